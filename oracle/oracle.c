@@ -1,0 +1,373 @@
+/*
+ * oracle.c -- plain FP64 CPU reference of the W4A16 quantized-expert MoE layer.
+ *
+ * TEST INFRASTRUCTURE.  Only the test-suite, the smoke check and the benchmark's
+ * CPU-baseline leg may load this library.  It shares no code, header, table or
+ * constant with the CUDA path; it is slow and written to be checked by eye.
+ *
+ * What it computes, and where each step comes from:
+ *
+ *  - W4A16: 4-bit integer weights, fp16 activations.
+ *      "GLM-5.3-Flash 320B MoEを4枚のCMP 170HXで動かすvLLMレシピ" (648news),
+ *      section "OpenAI互換APIで動く320BパラメータのMoE構成".
+ *  - int4 codes with one scale per output row (symmetric, no zero point).
+ *      "Show HN: 低速のコンピュータでGLM 5.2を動かす方法" (hakusoku), section
+ *      "実装済み機能", the int8/int4/int2 kernels with per-row scales.
+ *  - NVFP4 (E2M1 codes, one E4M3 scale per 16 elements, fp32 tensor scale) decoded
+ *    inside the matmul.  "GTX 1070向け35BパラメータMoEモデル推論エンジン公開"
+ *    (648news), section "VRAMとシステムメモリで重みを分割する設計" and the NVFP4
+ *    entry of "用語の注釈"; the bit layouts are those of the OCP Microscaling
+ *    Formats specification v1.0 (E2M1, E4M3 "FN").
+ *  - DeepSeek-V3-style sigmoid router with a shared expert.  hakusoku page,
+ *    section "実装済み機能".  The router formula is the DeepSeek-V3 one: sigmoid
+ *    scores, a per-expert bias that only affects selection, top-k, combine weights
+ *    = scores of the chosen experts normalised to sum 1 and multiplied by the
+ *    routed scaling factor.  No group-limited routing (one group).
+ *  - Batch MoE union: every unique expert of a batch is read once and applied to
+ *    all positions routed to it.  hakusoku page, section "実装済み機能".
+ *  - Deterministic MoE block order.  648news GLM-5.3 page, section
+ *    "Ampere世代のGPU向けに最適化された独自カーネル群".
+ *
+ * Readings taken where the pages are silent (each also listed in the design notes):
+ *  - nibble order: element 2b in the low nibble of byte b, 2b+1 in the high nibble;
+ *    int4 codes are two's complement (0x8..0xF -> -8..-1).
+ *  - NVFP4 blocks of 16 run along K of each output row, same nibble order.
+ *  - router logits are accumulated in fp64 and rounded to fp32; sigmoid in fp64
+ *    rounded to fp32; selection score = fp32 add of score and bias; top-k ties go
+ *    to the lower expert index; combine weight w = scaling * (s_j / sum_j s_j) in
+ *    fp64, stored as fp32.
+ *  - grouping: counts, exclusive offsets, permutation of assignment ids
+ *    a = t*k + j ordered by expert, ascending a inside an expert.
+ *  - expert FFN: g = W_g x, u = W_u x, h = SiLU(g) * u, y_e = W_d h, all fp64,
+ *    sums in ascending index order.
+ *  - combine: y_t = shared(x_t) + sum_{j=0..k-1} w_tj * y_{e_tj}(x_t), the shared
+ *    expert with weight 1.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "oracle.h"
+
+/* ------------------------------------------------------------ scalar decodes */
+
+double orc_half_to_double(uint16_t h)
+{
+    int s = (h >> 15) & 1, e = (h >> 10) & 31, m = h & 1023;
+    double v;
+    if (e == 0) v = ldexp((double)m, -24);                 /* subnormal: m * 2^-24 */
+    else if (e == 31) v = m ? NAN : INFINITY;
+    else v = ldexp((double)(1024 + m), e - 25);            /* (1 + m/1024) * 2^(e-15) */
+    return s ? -v : v;
+}
+
+int orc_int4_at(const uint8_t *row, long k)
+{
+    unsigned b = row[k >> 1];
+    int n = (k & 1) ? (int)(b >> 4) : (int)(b & 15);
+    return n >= 8 ? n - 16 : n;
+}
+
+double orc_e2m1_to_double(unsigned code)
+{
+    int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double v = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);   /* bias 1 */
+    return s ? -v : v;
+}
+
+double orc_e4m3_to_double(uint8_t b)
+{
+    int s = (b >> 7) & 1, e = (b >> 3) & 15, m = b & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = (e == 0) ? ldexp((double)m, -9)                     /* m/8 * 2^-6 */
+                        : ldexp(1.0 + m / 8.0, e - 7);             /* bias 7 */
+    return s ? -v : v;
+}
+
+/* dequantised weight (row n, column k) of one matrix */
+static double wq(const orc_matrix *M, long n, long k)
+{
+    const uint8_t *row = M->codes + (size_t)n * (size_t)(M->K / 2);
+    if (M->format == ORC_INT4) {
+        return (double)orc_int4_at(row, k) * (double)M->row_scale[n];
+    } else {
+        unsigned b = row[k >> 1];
+        unsigned c = (k & 1) ? (b >> 4) : (b & 15);
+        uint8_t sb = M->block_scale[(size_t)n * (size_t)(M->K / 16) + (size_t)(k / 16)];
+        return orc_e2m1_to_double(c) * orc_e4m3_to_double(sb) * (double)M->tensor_scale;
+    }
+}
+
+/* all dequantised weights of one matrix, [N][K] */
+void orc_dequant_matrix(const orc_matrix *M, double *out)
+{
+    for (long n = 0; n < M->N; n++)
+        for (long k = 0; k < M->K; k++) out[(size_t)n * (size_t)M->K + (size_t)k] = wq(M, n, k);
+}
+
+/* ------------------------------------------------------------------ router */
+
+void orc_router_logits(const uint16_t *x, int T, int H, const float *Wr, int E, float *logits)
+{
+    for (int t = 0; t < T; t++)
+        for (int e = 0; e < E; e++) {
+            double acc = 0.0;
+            for (int h = 0; h < H; h++)
+                acc += (double)Wr[(size_t)e * H + h] * orc_half_to_double(x[(size_t)t * H + h]);
+            logits[(size_t)t * E + e] = (float)acc;
+        }
+}
+
+float orc_sigmoid_f32(float logit)
+{
+    return (float)(1.0 / (1.0 + exp(-(double)logit)));
+}
+
+void orc_route(const float *logits, const float *bias, int T, int E, int k, double scaling,
+               int32_t *topk_idx, float *topk_w, float *sel_out, float *gap_out)
+{
+    float *s = (float *)malloc(sizeof(float) * (size_t)E);
+    float *sel = (float *)malloc(sizeof(float) * (size_t)E);
+    char *taken = (char *)malloc((size_t)E);
+    for (int t = 0; t < T; t++) {
+        for (int e = 0; e < E; e++) {
+            s[e] = orc_sigmoid_f32(logits[(size_t)t * E + e]);
+            sel[e] = s[e] + bias[e];                 /* one fp32 add */
+            if (sel_out) sel_out[(size_t)t * E + e] = sel[e];
+        }
+        memset(taken, 0, (size_t)E);
+        float last = 0.0f;
+        for (int j = 0; j < k; j++) {                /* k passes of an argmax */
+            int best = -1;
+            for (int e = 0; e < E; e++)
+                if (!taken[e] && (best < 0 || sel[e] > sel[best])) best = e;
+            taken[best] = 1;
+            topk_idx[(size_t)t * k + j] = best;
+            last = sel[best];
+        }
+        double sum = 0.0;
+        for (int j = 0; j < k; j++) sum += (double)s[topk_idx[(size_t)t * k + j]];
+        for (int j = 0; j < k; j++)
+            topk_w[(size_t)t * k + j] =
+                (float)(scaling * ((double)s[topk_idx[(size_t)t * k + j]] / sum));
+        if (gap_out) {
+            /* margin between the k-th chosen and the best unchosen selection score */
+            float next = -INFINITY;
+            for (int e = 0; e < E; e++)
+                if (!taken[e] && sel[e] > next) next = sel[e];
+            gap_out[t] = (k < E) ? (float)((double)last - (double)next) : INFINITY;
+        }
+    }
+    free(s);
+    free(sel);
+    free(taken);
+}
+
+/* ---------------------------------------------------------------- grouping */
+
+void orc_group(const int32_t *topk_idx, int T, int k, int E, int32_t *counts, int32_t *offsets,
+               int32_t *perm, int32_t *unique, int32_t *n_unique)
+{
+    int n = T * k;
+    for (int e = 0; e < E; e++) counts[e] = 0;
+    for (int a = 0; a < n; a++) counts[topk_idx[a]]++;
+    offsets[0] = 0;
+    for (int e = 0; e < E; e++) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t *fill = (int32_t *)calloc((size_t)E, sizeof(int32_t));
+    for (int a = 0; a < n; a++) {                      /* ascending a: stable */
+        int e = topk_idx[a];
+        perm[offsets[e] + fill[e]++] = a;
+    }
+    free(fill);
+    int u = 0;
+    for (int e = 0; e < E; e++)
+        if (counts[e] > 0) unique[u++] = e;
+    *n_unique = u;
+}
+
+/* -------------------------------------------------------------- expert FFN */
+
+void orc_expert_ffn(const orc_matrix *Wg, const orc_matrix *Wu, const orc_matrix *Wd,
+                    const double *x, double *h_out, double *y)
+{
+    int I = Wg->N, H = Wg->K;
+    double *h = (double *)malloc(sizeof(double) * (size_t)I);
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < I; n++) {
+        double g = 0.0, u = 0.0;
+        for (int kk = 0; kk < H; kk++) {
+            g += wq(Wg, n, kk) * x[kk];
+            u += wq(Wu, n, kk) * x[kk];
+        }
+        h[n] = g / (1.0 + exp(-g)) * u;               /* SiLU(g) * u */
+    }
+#pragma omp parallel for schedule(static)
+    for (int m = 0; m < Wd->N; m++) {
+        double acc = 0.0;
+        for (int n = 0; n < I; n++) acc += wq(Wd, m, n) * h[n];
+        y[m] = acc;
+    }
+    if (h_out) memcpy(h_out, h, sizeof(double) * (size_t)I);
+    free(h);
+}
+
+static orc_matrix routed_matrix(const orc_layer *L, int which, int e)
+{
+    orc_matrix M;
+    memset(&M, 0, sizeof M);
+    M.format = L->format;
+    int rows = which == 2 ? L->H : L->I;
+    int K = which == 2 ? L->I : L->H;
+    M.N = rows;
+    M.K = K;
+    const uint8_t *codes = which == 0 ? L->g : which == 1 ? L->u : L->d;
+    M.codes = codes + (size_t)e * (size_t)rows * (size_t)(K / 2);
+    if (L->format == ORC_INT4) {
+        const float *sc = which == 0 ? L->sg : which == 1 ? L->su : L->sd;
+        M.row_scale = sc + (size_t)e * (size_t)rows;
+    } else {
+        const uint8_t *bs = which == 0 ? L->bg : which == 1 ? L->bu : L->bd;
+        const float *ts = which == 0 ? L->tg : which == 1 ? L->tu : L->td;
+        M.block_scale = bs + (size_t)e * (size_t)rows * (size_t)(K / 16);
+        M.tensor_scale = ts[e];
+    }
+    return M;
+}
+
+static orc_matrix shared_matrix(const orc_layer *L, int which)
+{
+    orc_matrix M;
+    memset(&M, 0, sizeof M);
+    M.format = L->format;
+    M.N = which == 2 ? L->H : L->I_sh;
+    M.K = which == 2 ? L->I_sh : L->H;
+    M.codes = which == 0 ? L->sh_g : which == 1 ? L->sh_u : L->sh_d;
+    if (L->format == ORC_INT4) {
+        M.row_scale = which == 0 ? L->sh_sg : which == 1 ? L->sh_su : L->sh_sd;
+    } else {
+        M.block_scale = which == 0 ? L->sh_bg : which == 1 ? L->sh_bu : L->sh_bd;
+        M.tensor_scale = which == 0 ? L->sh_tg : which == 1 ? L->sh_tu : L->sh_td;
+    }
+    return M;
+}
+
+void orc_routed_expert(const orc_layer *L, int e, const double *x, double *h_out, double *y)
+{
+    orc_matrix g = routed_matrix(L, 0, e), u = routed_matrix(L, 1, e), d = routed_matrix(L, 2, e);
+    orc_expert_ffn(&g, &u, &d, x, h_out, y);
+}
+
+void orc_shared_expert(const orc_layer *L, const double *x, double *h_out, double *y)
+{
+    orc_matrix g = shared_matrix(L, 0), u = shared_matrix(L, 1), d = shared_matrix(L, 2);
+    orc_expert_ffn(&g, &u, &d, x, h_out, y);
+}
+
+/* ------------------------------------------------------------------ drivers */
+
+static void decode_tokens(const uint16_t *x, int T, int H, double *xd)
+{
+    for (size_t i = 0; i < (size_t)T * H; i++) xd[i] = orc_half_to_double(x[i]);
+}
+
+static void route_all(const orc_layer *L, const uint16_t *x, int T, const float *logits_in,
+                      orc_result *R)
+{
+    if (logits_in)
+        memcpy(R->logits, logits_in, sizeof(float) * (size_t)T * L->E);
+    else
+        orc_router_logits(x, T, L->H, L->Wr, L->E, R->logits);
+    orc_route(R->logits, L->bias, T, L->E, L->k, L->scaling, R->topk_idx, R->topk_w, R->sel,
+              R->gap);
+}
+
+static void combine(const orc_layer *L, int T, const double *y_assign, const double *y_shared,
+                    const float *topk_w, double *y)
+{
+    int H = L->H, k = L->k;
+    for (int t = 0; t < T; t++)
+        for (int m = 0; m < H; m++) {
+            double acc = L->n_shared ? y_shared[(size_t)t * H + m] : 0.0;
+            for (int j = 0; j < k; j++)
+                acc += (double)topk_w[(size_t)t * k + j] * y_assign[((size_t)t * k + j) * H + m];
+            y[(size_t)t * H + m] = acc;
+        }
+}
+
+/* Batched driver: group the assignments by expert and apply every unique expert
+ * once, to all the tokens routed to it. */
+void orc_forward(const orc_layer *L, const uint16_t *x, int T, const float *logits_in,
+                 orc_result *R)
+{
+    int H = L->H, k = L->k, E = L->E;
+    double *xd = (double *)malloc(sizeof(double) * (size_t)T * H);
+    decode_tokens(x, T, H, xd);
+    route_all(L, x, T, logits_in, R);
+    orc_group(R->topk_idx, T, k, E, R->counts, R->offsets, R->perm, R->unique, &R->n_unique);
+    for (int ui = 0; ui < R->n_unique; ui++) {
+        int e = R->unique[ui];
+        for (int p = R->offsets[e]; p < R->offsets[e + 1]; p++) {
+            int a = R->perm[p], t = a / k;
+            orc_routed_expert(L, e, xd + (size_t)t * H,
+                              R->h_assign ? R->h_assign + (size_t)a * L->I : NULL,
+                              R->y_assign + (size_t)a * H);
+        }
+    }
+    if (L->n_shared)
+        for (int t = 0; t < T; t++)
+            orc_shared_expert(L, xd + (size_t)t * H,
+                              R->h_shared ? R->h_shared + (size_t)t * L->I_sh : NULL,
+                              R->y_shared + (size_t)t * H);
+    combine(L, T, R->y_assign, R->y_shared, R->topk_w, R->y);
+    free(xd);
+}
+
+/* Per-token driver: every token visits its own k experts in order j = 0..k-1. */
+void orc_forward_per_token(const orc_layer *L, const uint16_t *x, int T, const float *logits_in,
+                           orc_result *R)
+{
+    int H = L->H, k = L->k, E = L->E;
+    double *xd = (double *)malloc(sizeof(double) * (size_t)T * H);
+    decode_tokens(x, T, H, xd);
+    route_all(L, x, T, logits_in, R);
+    orc_group(R->topk_idx, T, k, E, R->counts, R->offsets, R->perm, R->unique, &R->n_unique);
+    for (int t = 0; t < T; t++) {
+        for (int j = 0; j < k; j++) {
+            int a = t * k + j;
+            orc_routed_expert(L, R->topk_idx[a], xd + (size_t)t * H,
+                              R->h_assign ? R->h_assign + (size_t)a * L->I : NULL,
+                              R->y_assign + (size_t)a * H);
+        }
+        if (L->n_shared)
+            orc_shared_expert(L, xd + (size_t)t * H,
+                              R->h_shared ? R->h_shared + (size_t)t * L->I_sh : NULL,
+                              R->y_shared + (size_t)t * H);
+    }
+    combine(L, T, R->y_assign, R->y_shared, R->topk_w, R->y);
+    free(xd);
+}
+
+/* One token's output, for sampled checks at full size: routes token t of x
+ * (using logits_in row t when given) and evaluates only that token. */
+void orc_forward_token(const orc_layer *L, const uint16_t *x_t, const float *logits_t,
+                       int32_t *topk_idx, float *topk_w, float *gap, double *y)
+{
+    int H = L->H, k = L->k, E = L->E;
+    float *logits = (float *)malloc(sizeof(float) * (size_t)E);
+    if (logits_t) memcpy(logits, logits_t, sizeof(float) * (size_t)E);
+    else orc_router_logits(x_t, 1, H, L->Wr, E, logits);
+    orc_route(logits, L->bias, 1, E, k, L->scaling, topk_idx, topk_w, NULL, gap);
+    double *xd = (double *)malloc(sizeof(double) * (size_t)H);
+    double *ye = (double *)malloc(sizeof(double) * (size_t)H);
+    decode_tokens(x_t, 1, H, xd);
+    for (int m = 0; m < H; m++) y[m] = 0.0;
+    if (L->n_shared) orc_shared_expert(L, xd, NULL, y);
+    for (int j = 0; j < k; j++) {
+        orc_routed_expert(L, topk_idx[j], xd, NULL, ye);
+        for (int m = 0; m < H; m++) y[m] += (double)topk_w[j] * ye[m];
+    }
+    free(logits);
+    free(xd);
+    free(ye);
+}
