@@ -1,0 +1,211 @@
+/*
+ * moe.h -- C ABI of the W4A16 quantized-expert Mixture-of-Experts decode layer
+ *          for NVIDIA B200 (sm_100a).
+ *
+ * The layer (one call = one MoE layer over T tokens):
+ *   1. router:  logit[t,e] = sum_h W_r[e,h] * x[t,h]   (fp32 weights, fp16 activations,
+ *               fp32 accumulation)
+ *   2. scores:  s = sigmoid(logit); selection score sel = s + bias[e]; the k experts with
+ *               the largest sel (descending, equal scores -> lower expert index);
+ *               combine weights w_j = routed_scaling * s_j / sum_j' s_j'
+ *   3. grouping: the T*k assignments a = t*k + j are grouped by expert so that every
+ *               unique expert is read once and applied to all its tokens
+ *   4. experts: h = SiLU(x W_g^T) * (x W_u^T) rounded to fp16, y_e = h W_d^T, weights
+ *               dequantised inside the matmul, fp32 accumulation
+ *   5. combine: y[t] = shared(x_t) + sum_{j=0..k-1} w_tj * y_{e_tj}(x_t), in that order,
+ *               stored as fp16.
+ *
+ * Sources (web pages on W4A16 quantised-expert inference):
+ *  - W4A16 = INT4 weights, FP16 activations; custom kernels fusing MoE routing for small
+ *    batches; deterministic MoE block order: "GLM-5.3-Flash 320B MoEを4枚のCMP 170HXで
+ *    動かすvLLMレシピ" (648news), sections "OpenAI互換APIで動く320BパラメータのMoE構成" and
+ *    "Ampere世代のGPU向けに最適化された独自カーネル群".
+ *  - DeepSeek-V3-style sigmoid router, shared expert, int4 with per-row scales, batch MoE
+ *    union: "Show HN: 低速のコンピュータでGLM 5.2を動かす方法" (hakusoku), section
+ *    "実装済み機能".
+ *  - NVFP4 weights decoded in registers inside the matmul: "GTX 1070向け35Bパラメータ
+ *    MoEモデル推論エンジン公開" (648news), section "VRAMとシステムメモリで重みを分割する
+ *    設計" and "用語の注釈" (NVFP4).
+ *  - 256 experts of about 19 MB per layer: hakusoku page, section "Colibrì: 消費者PCで
+ *    744BパラメータGLM-5.2を動かす革新的エンジン".
+ *
+ * Conventions for every call below:
+ *  - All tensor pointers are DEVICE pointers unless the name ends in _host.  They are
+ *    borrowed: the library never frees them.  Weight pointers given to moe_layer_create
+ *    must stay valid and unchanged for the life of the handle.
+ *  - Activations are fp16 given as their uint16_t bit patterns, row-major [T][H].
+ *  - Quantised matrices are row-major with K (the input dimension) contiguous; two 4-bit
+ *    codes per byte, element 2b in the LOW nibble of byte b.  int4 codes are two's
+ *    complement in [-8, 7] with one fp32 scale per output row.  NVFP4 codes are E2M1 with
+ *    one E4M3 (OCP "FN") scale byte per 16 consecutive K elements of a row and one fp32
+ *    scale per (expert, matrix).
+ *  - Every call except create/destroy/get_device_status is asynchronous on the caller's
+ *    stream, allocates nothing and never synchronises the host, so it may be captured in
+ *    a CUDA graph.  A non-zero return means nothing was enqueued.
+ *  - Errors found on the device (a bounded wait that gave up, an index out of range)
+ *    never trap: kernels record a MOE_ERR_* code in the handle's status word and return.
+ *    Read it with moe_get_device_status.
+ *  - Results are deterministic: the same inputs give bit-identical outputs (no float
+ *    atomics, fixed reduction orders).
+ */
+#ifndef MOE_W4A16_H
+#define MOE_W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Compatible with cudaStream_t / CUstream; NULL is the legacy default stream. */
+typedef struct CUstream_st *moe_stream_t;
+
+/* ---------------------------------------------------------------- status codes */
+enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,     /* a pointer, size or shape is invalid (host check) */
+    MOE_ERR_UNSUPPORTED = 2,     /* valid request this build does not implement */
+    MOE_ERR_WORKSPACE = 3,       /* workspace missing, misaligned or too small */
+    MOE_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed */
+    MOE_ERR_DEVICE_TIMEOUT = 5,  /* a device-side wait exceeded its iteration limit */
+    MOE_ERR_DEVICE_BOUNDS = 6    /* a device-side index check failed; access skipped */
+};
+
+/* weight formats */
+enum {
+    MOE_FMT_INT4_ROWSCALE = 0,   /* int4 codes + fp32 scale per output row */
+    MOE_FMT_NVFP4 = 1            /* E2M1 codes + E4M3 per 16 K-elements + fp32 per matrix */
+};
+
+/* Shape and hyper-parameters of one layer. */
+typedef struct moe_layer_desc {
+    int hidden;            /* H: model width, fan-in of gate/up, fan-out of down */
+    int inter;             /* I: intermediate width of a routed expert */
+    int inter_shared;      /* I_sh: intermediate width of the shared expert */
+    int n_experts;         /* E: routed experts, 1..1024 */
+    int top_k;             /* k: experts per token, 1..min(E, 32) */
+    int n_shared;          /* shared experts: 0 or 1 */
+    float routed_scaling;  /* multiplies the normalised combine weights (e.g. 2.5) */
+    int format;            /* MOE_FMT_* */
+    int max_tokens;        /* largest T any call on this handle will pass, >= 1 */
+} moe_layer_desc;
+
+/* Device pointers to one layer's parameters (borrowed; see conventions).
+ * Routed tensors have a leading expert dimension E; shared ones do not.
+ *   router_w     fp32 [E][H]              router_bias fp32 [E]
+ *   gate, up     u8   [E][I][H/2]         down        u8   [E][H][I/2]
+ *   int4:  gate_scale, up_scale fp32 [E][I];  down_scale fp32 [E][H]
+ *   NVFP4: gate_bscale, up_bscale u8 [E][I][H/16]; down_bscale u8 [E][H][I/16];
+ *          gate_tscale, up_tscale, down_tscale fp32 [E]
+ *   shared_*: the same without E, with I_sh rows (gate/up) or I_sh/2 bytes (down);
+ *          shared NVFP4 tensor scales are fp32 [1].
+ * Pointers that the chosen format or n_shared does not use may be NULL.  Every pointer
+ * must be 16-byte aligned. */
+typedef struct moe_weights {
+    const float *router_w;
+    const float *router_bias;
+    const uint8_t *gate, *up, *down;
+    const float *gate_scale, *up_scale, *down_scale;
+    const uint8_t *gate_bscale, *up_bscale, *down_bscale;
+    const float *gate_tscale, *up_tscale, *down_tscale;
+    const uint8_t *shared_gate, *shared_up, *shared_down;
+    const float *shared_gate_scale, *shared_up_scale, *shared_down_scale;
+    const uint8_t *shared_gate_bscale, *shared_up_bscale, *shared_down_bscale;
+    const float *shared_gate_tscale, *shared_up_tscale, *shared_down_tscale;
+} moe_weights;
+
+typedef struct moe_layer moe_layer;   /* opaque handle */
+
+/* ---------------------------------------------------------------- lifetime */
+
+/* Validates desc and weights and builds the handle: TMA descriptors over the caller's
+ * weights and a device status word (the only allocation the library makes).
+ * Requirements: H and I (and I_sh) multiples of 64 (int4) or 256 (NVFP4) -- the NVFP4
+ * block-scale rows must be 16-byte multiples -- H <= 16384, I, I_sh <= 16384,
+ * 1 <= E <= 1024, 1 <= k <= min(E, 32), n_shared in {0, 1}, 1 <= max_tokens <= 65536,
+ * all pointers 16-byte aligned.  Uses the current CUDA device.
+ * Returns MOE_OK and *out, or an error code and *out = NULL. */
+int moe_layer_create(const moe_layer_desc *desc, const moe_weights *weights, moe_layer **out);
+
+/* Frees the handle (and its status word).  The caller must ensure no call on it is
+ * still running on the GPU.  NULL is accepted. */
+int moe_layer_destroy(moe_layer *layer);
+
+/* Bytes of device workspace any call with T tokens needs (0 if T is out of range).
+ * One workspace serves every entry point; it must be 256-byte aligned, and must not be
+ * used by two calls that may run concurrently.  It holds a few completion counters that
+ * must be ZERO before the workspace's first use (one cudaMemset of the whole buffer);
+ * every call leaves them at zero again.  After a device-side error
+ * (moe_get_device_status != MOE_OK) zero it again before reuse. */
+size_t moe_workspace_size(const moe_layer *layer, int T);
+
+/* ---------------------------------------------------------------- staged steps */
+
+/* Steps 1-2.  x [T][H] fp16.  If logits_in is non-NULL ([T][E] fp32) the router GEMV is
+ * skipped and these logits are used (bit-exact selection from given logits).  If
+ * logits_out is non-NULL the fp32 logits are written there.  Outputs: topk_idx int32
+ * [T][k] (descending selection score), topk_w fp32 [T][k].  0 <= T <= max_tokens. */
+int moe_route(const moe_layer *layer, const uint16_t *x, int T, const float *logits_in,
+              float *logits_out, int32_t *topk_idx, float *topk_w, void *workspace,
+              size_t workspace_bytes, moe_stream_t stream);
+
+/* Step 3.  topk_idx [T][k] with values in [0, E) (out-of-range values set
+ * MOE_ERR_DEVICE_BOUNDS and are dropped).  Outputs (int32): counts [E], offsets [E+1]
+ * (exclusive prefix sum of counts), perm [T*k] (assignment ids a = t*k + j ordered by
+ * expert, ascending a inside an expert), unique [E] (experts with counts > 0,
+ * ascending; entries past n_unique are unspecified), n_unique [1]. */
+int moe_group(const moe_layer *layer, const int32_t *topk_idx, int T, int32_t *counts,
+              int32_t *offsets, int32_t *perm, int32_t *unique, int32_t *n_unique,
+              void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* Step 4 (and the shared expert).  Uses offsets [E+1] and perm [T*k] as moe_group
+ * writes them.  y_assign fp32 [T*k][H]: row a = t*k + j holds expert topk_idx[t][j]
+ * applied to x[t] (unscaled).  y_shared fp32 [T][H] receives the shared expert (may be
+ * NULL when n_shared = 0). */
+int moe_expert_ffn(const moe_layer *layer, const uint16_t *x, int T, const int32_t *offsets,
+                   const int32_t *perm, float *y_assign, float *y_shared, void *workspace,
+                   size_t workspace_bytes, moe_stream_t stream);
+
+/* Step 5.  y [T][H] fp16 = y_shared[t] + sum_j topk_w[t][j] * y_assign[t*k + j], summed
+ * in fp32 in the order shared, j = 0 .. k-1.  y_shared may be NULL when n_shared = 0. */
+int moe_combine(const moe_layer *layer, const float *y_assign, const float *y_shared,
+                const float *topk_w, int T, uint16_t *y, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- fused layer */
+
+/* Steps 1-5 in as few launches as the path allows.  x [T][H] fp16 in, y [T][H] fp16
+ * out (x and y may not overlap).  Equal within tolerance to the staged path. */
+int moe_forward(const moe_layer *layer, const uint16_t *x, int T, uint16_t *y,
+                void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* moe_forward with HOST activations: enqueues the host->device copy of x_host, the
+ * layer and the device->host copy into y_host on the stream (x and y are staged in the
+ * workspace).  Returns once enqueued; synchronise the stream before reading y_host.
+ * Host buffers should be page-locked for the copies to be asynchronous. */
+int moe_forward_host(const moe_layer *layer, const uint16_t *x_host, int T, uint16_t *y_host,
+                     void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- diagnostics */
+
+/* Human-readable name of a MOE_* status code (static storage). */
+const char *moe_status_string(int status);
+
+/* Synchronises the device, returns in *status the first device-side error recorded on
+ * this handle since the last call (MOE_OK if none) and clears it.  For tests and
+ * debugging, not for the hot path. */
+int moe_get_device_status(const moe_layer *layer, int *status);
+
+/* Test hook for the bounded waits: launches one block whose consumer waits on an
+ * mbarrier that nothing completes, with an iteration limit of max_iters.  The kernel
+ * gives up, records MOE_ERR_DEVICE_TIMEOUT in the status word and returns. */
+int moe_debug_wait_timeout(const moe_layer *layer, long long max_iters, moe_stream_t stream);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_W4A16_H */

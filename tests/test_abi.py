@@ -1,0 +1,125 @@
+"""The C-ABI library: it loads without a GPU, exports every symbol ``include/moe.h``
+declares, and its host-side validation rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import w4a16_quantized_expert_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b(moe_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("moe_layer_create", "moe_layer_destroy", "moe_workspace_size", "moe_route",
+                     "moe_group", "moe_expert_ffn", "moe_combine", "moe_forward"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = moe.lib()
+    missing = [n for n in declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_python_binding_has_the_same_names():
+    for n in declared_functions():
+        assert hasattr(moe, n), n
+
+
+def test_status_strings_and_version():
+    assert moe.status_string(moe.MOE_OK) == "MOE_OK"
+    assert moe.status_string(moe.MOE_ERR_DEVICE_TIMEOUT) == "MOE_ERR_DEVICE_TIMEOUT"
+    assert moe.status_string(99) == "MOE_ERR_UNKNOWN"
+    assert moe.moe_version() >= 100
+
+
+def _desc(**kw):
+    d = dict(hidden=256, inter=128, inter_shared=128, n_experts=16, top_k=2, n_shared=1,
+             routed_scaling=2.5, format=0, max_tokens=4)
+    d.update(kw)
+    return moe.moe_layer_desc(**d)
+
+
+def _weights(fmt=0, n_shared=1, misalign=None, drop=None):
+    w = moe.moe_weights()
+    for i, f in enumerate(moe.WEIGHT_FIELDS):
+        setattr(w, f, 0x100000 + 0x1000 * i)
+    if misalign:
+        setattr(w, misalign, getattr(w, misalign) + 4)
+    if drop:
+        setattr(w, drop, None)
+    return w
+
+
+def _create(desc, w):
+    h = ctypes.c_void_p()
+    rc = moe.lib().moe_layer_create(ctypes.byref(desc), ctypes.byref(w), ctypes.byref(h))
+    return rc, h.value
+
+
+@pytest.mark.parametrize("bad", [
+    dict(hidden=0), dict(hidden=96), dict(hidden=16384 + 64), dict(inter=100),
+    dict(n_experts=0), dict(n_experts=1025), dict(top_k=0), dict(top_k=33),
+    dict(top_k=17), dict(n_shared=2), dict(inter_shared=50), dict(max_tokens=0),
+    dict(max_tokens=70000), dict(format=7), dict(routed_scaling=float("nan")),
+    dict(format=1, hidden=320), dict(format=1, inter=128),
+])
+def test_create_rejects_bad_shapes(bad):
+    rc, h = _create(_desc(**bad), _weights())
+    assert rc == moe.MOE_ERR_INVALID_ARG and h is None
+
+
+@pytest.mark.parametrize("field", ["router_w", "gate", "down_scale", "shared_up"])
+def test_create_rejects_missing_or_misaligned_pointers(field):
+    rc, _ = _create(_desc(), _weights(drop=field))
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    rc, _ = _create(_desc(), _weights(misalign=field))
+    assert rc == moe.MOE_ERR_INVALID_ARG
+
+
+def test_unused_pointers_may_be_null():
+    # int4 without a shared expert ignores the NVFP4 and shared fields; with no GPU the
+    # call gets past validation and fails at the first CUDA call instead
+    w = _weights()
+    for f in moe.WEIGHT_FIELDS:
+        if "bscale" in f or "tscale" in f or f.startswith("shared"):
+            setattr(w, f, None)
+    rc, h = _create(_desc(n_shared=0), w)
+    try:
+        import torch
+        gpu = torch.cuda.is_available()
+    except Exception:
+        gpu = False
+    if not gpu:
+        assert rc == moe.MOE_ERR_CUDA and h is None
+
+
+def test_null_handle_and_out_of_range_T():
+    L = moe.lib()
+    assert L.moe_workspace_size(None, 1) == 0
+    assert L.moe_forward(None, None, 1, None, None, 0, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_route(None, None, 1, None, None, None, None, None, 0, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_destroy(None) == moe.MOE_OK
+    st = ctypes.c_int(0)
+    assert L.moe_get_device_status(None, ctypes.byref(st)) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_product_path_has_no_oracle_or_fallback():
+    """The package never imports the oracle and has no CPU compute path."""
+    pkg = os.path.join(ROOT, "w4a16_quantized_expert_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
+                assert "liboracle" not in txt, f

@@ -1,0 +1,248 @@
+"""GPU parity: every step of the layer through the C ABI against the FP64 oracle on the
+same seeded inputs (see ``gpu_cases.py`` for the comparison rules)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import w4a16_quantized_expert_b200 as moe
+from gpu_cases import Case, check_weights, check_y, y_to_f64
+
+pytestmark = pytest.mark.gpu
+
+W = synth.WORKLOADS
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    return Case(W["tiny"], max_tokens=64)
+
+
+# ------------------------------------------------------------------ routing
+def _route_from_logits(case, T):
+    ws = case.dev.workspace(T)
+    ref = case.oracle_forward()
+    li = torch.from_numpy(ref["logits"]).cuda()
+    idx, w, lo = case.dev.route(None, T, ws, logits_in=li, want_logits=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), ref["topk_idx"]), "topk_idx differs"
+    check_weights(w.cpu().numpy(), ref["topk_w"].astype(np.float64))
+    assert np.array_equal(lo.cpu().numpy(), ref["logits"]), "logits_out copy"
+    return ref
+
+
+def test_route_bitexact_from_oracle_logits_tiny(tiny):
+    _route_from_logits(tiny, tiny.T)
+
+
+@pytest.mark.parametrize("name,T", [("decode8", 8), ("nvfp4_16", 16), ("tiny", 37)])
+def test_route_bitexact_from_oracle_logits(name, T):
+    w = W[name]
+    case = Case(w, T=T, experts="routed") if name != "tiny" else Case(w, T=T)
+    _route_from_logits(case, T)
+
+
+def test_route_gemv_logits(tiny):
+    T = tiny.T
+    ws = tiny.dev.workspace(T)
+    idx, w, lo = tiny.dev.route(tiny.x_dev, T, ws, want_logits=True)
+    ref = tiny.oracle_forward()
+    lo = lo.cpu().numpy()
+    assert np.abs(lo - ref["logits"]).max() <= 1e-5 * np.abs(ref["logits"]).max() + 1e-6
+    keep = ref["gap"] >= 1e-4
+    assert np.array_equal(idx.cpu().numpy()[keep], ref["topk_idx"][keep])
+
+
+# ------------------------------------------------------------------ grouping
+@pytest.mark.parametrize("T,k,E,mode", [(4, 2, 16, "rand"), (1, 8, 256, "rand"), (16, 8, 256, "rand"),
+                                        (512, 8, 256, "rand"), (40, 4, 16, "hot"), (9, 3, 1024, "rand")])
+def test_group_bitexact(T, k, E, mode):
+    rng = np.random.default_rng(T * 1000 + E)
+    if mode == "hot":
+        idx = np.stack([np.concatenate([[0], rng.choice(np.arange(1, E), k - 1, replace=False)])
+                        for _ in range(T)]).astype(np.int32)
+    else:
+        idx = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    w = synth.WORKLOADS["tiny"].with_(E=E, k=k)
+    host = {"Wr": np.zeros((E, 256), np.float32), "bias": np.zeros(E, np.float32)}
+    host.update(synth.make_experts(w, experts=[]))
+    from w4a16_quantized_expert_b200.device import DeviceLayer
+    dev = DeviceLayer(oracle.desc_of(w), host, max_tokens=T)
+    ws = dev.workspace(T)
+    counts, offsets, perm, unique, nu = dev.group(torch.from_numpy(idx).cuda(), T, ws)
+    c_ref, o_ref, p_ref, u_ref = oracle.default().group(idx, E)
+    assert np.array_equal(counts.cpu().numpy(), c_ref)
+    assert np.array_equal(offsets.cpu().numpy(), o_ref)
+    assert np.array_equal(perm.cpu().numpy()[: T * k], p_ref)
+    n = int(nu.item())
+    assert n == len(u_ref) and np.array_equal(unique.cpu().numpy()[:n], u_ref)
+    assert moe.moe_get_device_status(dev.handle) == moe.MOE_OK
+
+
+def test_group_out_of_range_index_is_reported_not_faulted(tiny):
+    idx = torch.tensor([[0, 99], [3, -2], [5, 6], [7, 1]], dtype=torch.int32, device="cuda")
+    ws = tiny.dev.workspace(4)
+    counts, offsets, perm, unique, nu = tiny.dev.group(idx, 4, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(tiny.dev.handle) == moe.MOE_ERR_DEVICE_BOUNDS
+    assert int(offsets[-1].item()) == 6        # the two bad assignments were dropped
+
+
+# ------------------------------------------------------------------ experts
+def _ffn_vs_oracle(case, T):
+    ref = case.oracle_forward()
+    ws = case.dev.workspace(T)
+    offsets = torch.from_numpy(ref["offsets"]).cuda()
+    perm = torch.from_numpy(ref["perm"]).cuda()
+    ya, ys = case.dev.expert_ffn(case.x_dev, T, offsets, perm, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(case.dev.handle) == moe.MOE_OK
+    ya = ya.cpu().numpy().astype(np.float64)
+    scale = np.abs(ref["y_assign"]).max()
+    err = np.abs(ya - ref["y_assign"]).max() / scale
+    assert err <= 4e-3, f"y_assign error {err:.3g}"
+    if case.desc["n_shared"]:
+        ys = ys.cpu().numpy().astype(np.float64)
+        err = np.abs(ys - ref["y_shared"]).max() / np.abs(ref["y_shared"]).max()
+        assert err <= 4e-3, f"y_shared error {err:.3g}"
+    return ref
+
+
+def test_expert_ffn_tiny(tiny):
+    _ffn_vs_oracle(tiny, tiny.T)
+
+
+@pytest.mark.parametrize("name,T", [("decode8", 8), ("nvfp4_16", 16), ("nvfp4_1", 1)])
+def test_expert_ffn(name, T):
+    _ffn_vs_oracle(Case(W[name], T=T, experts="routed"), T)
+
+
+def test_combine_tiny(tiny):
+    T = tiny.T
+    ref = tiny.oracle_forward()
+    ya = torch.from_numpy(ref["y_assign"].astype(np.float32)).cuda()
+    ys = torch.from_numpy(ref["y_shared"].astype(np.float32)).cuda()
+    w = torch.from_numpy(ref["topk_w"]).cuda()
+    y = tiny.dev.combine(ya, ys, w, T)
+    check_y(y_to_f64(y), ref["y"], np.full(T, 1.0))
+
+
+# ------------------------------------------------------------------ fused layer
+def _forward(case, T=None):
+    T = case.T if T is None else T
+    ws = case.dev.workspace(T)
+    y = case.dev.forward(case.x_dev[:T], ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(case.dev.handle) == moe.MOE_OK
+    return y, ws
+
+
+def test_forward_tiny(tiny):
+    y, _ = _forward(tiny)
+    ref = tiny.oracle_forward()
+    check_y(y_to_f64(y), ref["y"], ref["gap"])
+
+
+@pytest.mark.parametrize("name", ["decode1", "decode8", "nvfp4_1", "nvfp4_16"])
+def test_forward_full_size(name):
+    case = Case(W[name], experts="routed")
+    y, _ = _forward(case)
+    ref = case.oracle_forward()
+    excluded, err = check_y(y_to_f64(y), ref["y"], ref["gap"])
+    print(f"{name}: excluded {excluded}/{case.T}, rel err {err:.3g}")
+
+
+def test_forward_prefill512_sampled():
+    case = Case(W["prefill512"])
+    y, _ = _forward(case)
+    tokens = [0, 1, 63, 64, 255, 300, 510, 511]
+    ref = case.oracle_forward(tokens=tokens)
+    excluded, err = check_y(y_to_f64(y)[tokens], ref["y"], ref["gap"])
+    print(f"prefill512 sampled: excluded {excluded}/{len(tokens)}, rel err {err:.3g}")
+
+
+@pytest.mark.parametrize("T", [1, 2, 15, 16, 17, 33, 64])
+def test_forward_ragged_T(tiny, T):
+    case = Case(W["tiny"], T=T, max_tokens=64, batch=T)
+    y, _ = _forward(case)
+    ref = case.oracle_forward()
+    check_y(y_to_f64(y), ref["y"], ref["gap"])
+
+
+def test_forward_T0_is_noop(tiny):
+    ws = tiny.dev.workspace(0)
+    y = torch.zeros((0, 256), dtype=torch.uint16, device="cuda")
+    moe.moe_forward(tiny.dev.handle, tiny.x_dev.data_ptr(), 0, y.data_ptr(), ws.data_ptr(), ws.numel(), 0)
+
+
+def test_staged_equals_fused(tiny):
+    T = tiny.T
+    ws = tiny.dev.workspace(T)
+    y_fused = tiny.dev.forward(tiny.x_dev, ws)
+    idx, w, _ = tiny.dev.route(tiny.x_dev, T, ws)
+    counts, offsets, perm, unique, nu = tiny.dev.group(idx, T, ws)
+    ya, ys = tiny.dev.expert_ffn(tiny.x_dev, T, offsets, perm, ws)
+    y_staged = tiny.dev.combine(ya, ys, w, T)
+    torch.cuda.synchronize()
+    a, b = y_to_f64(y_fused), y_to_f64(y_staged)
+    assert np.abs(a - b).max() <= 1e-3 * np.abs(a).max()
+
+
+def test_determinism_bit_identical():
+    case = Case(W["decode8"], experts="routed")
+    y1, ws = _forward(case)
+    y2 = case.dev.forward(case.x_dev, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_forward_host_matches_forward(tiny):
+    T = tiny.T
+    ws = tiny.dev.workspace(T)
+    y_dev = tiny.dev.forward(tiny.x_dev, ws)
+    xh = torch.from_numpy(tiny.x.copy()).pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    tiny.dev.forward_host(xh, yh, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y_dev.cpu(), yh)
+
+
+# ------------------------------------------------------------------ special shapes
+def _special(E, k, n_shared, scaling, fmt=0, bias_hot=None, T=6):
+    H, I = (256, 128) if fmt == 0 else (512, 256)
+    w = synth.Workload("special", T, H, I, I, E, k, n_shared, scaling, fmt, "uniform", 99)
+    host = synth.make_layer(w)
+    if bias_hot is not None:
+        host["bias"] = np.full(E, -1.0, np.float32)
+        host["bias"][bias_hot] = 1.0
+    case = Case.__new__(Case)
+    case.w, case.T, case.desc = w, T, oracle.desc_of(w)
+    case.x = synth.make_tokens(w, T)
+    case.host = host
+    from w4a16_quantized_expert_b200.device import DeviceLayer
+    case.dev = DeviceLayer(case.desc, host, max_tokens=T)
+    case.x_dev = torch.from_numpy(case.x.copy()).cuda()
+    return case
+
+
+@pytest.mark.parametrize("E,k,n_shared,scaling,fmt,hot", [
+    (1, 1, 0, 1.0, 0, None),       # dense SwiGLU special case
+    (8, 8, 1, 2.5, 0, None),       # k = E: every expert on every token
+    (16, 4, 0, 2.5, 0, [3, 5, 7, 9]),   # every token on the same four experts
+    (32, 8, 1, 2.5, 1, None),      # NVFP4 with a small shape
+    (5, 2, 1, 1.0, 0, None),       # E not a multiple of 32
+])
+def test_forward_special_shapes(E, k, n_shared, scaling, fmt, hot):
+    case = _special(E, k, n_shared, scaling, fmt, hot)
+    y, _ = _forward(case)
+    ref = oracle.default().forward(case.desc, case.host, case.x)
+    check_y(y_to_f64(y), ref["y"], ref["gap"])
+
+
+def test_device_wait_timeout_is_reported(tiny):
+    moe.moe_debug_wait_timeout(tiny.dev.handle, 1 << 20, 0)
+    assert moe.moe_get_device_status(tiny.dev.handle) == moe.MOE_ERR_DEVICE_TIMEOUT
+    # the context stays usable
+    y, _ = _forward(tiny)
+    assert y.shape == (tiny.T, 256)

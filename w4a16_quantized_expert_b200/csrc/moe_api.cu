@@ -1,0 +1,476 @@
+// moe_api.cu -- the C ABI declared in include/moe.h: validation, TMA descriptors over
+// the caller's weights, workspace layout and the launch sequence of each entry point.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "moe_internal.h"
+
+namespace moe {
+cudaError_t launch_router(const RouterParams &p, int grid_x, int grid_y, cudaStream_t s);
+cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
+cudaError_t launch_combine(const CombineParams &p, cudaStream_t s);
+cudaError_t launch_ffn(const LayerMaps &maps, const FfnParams &p, bool gate_up, int grid, bool pdl,
+                       cudaStream_t s);
+cudaError_t ffn_occupancy(int fmt, bool gu, int *blocks_per_sm);
+cudaError_t launch_wait_timeout(int *status, unsigned long long max_iters, cudaStream_t s);
+
+namespace {
+
+constexpr int kRouterEpc = 2;   // router experts per CTA
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// ------------------------------------------------------------------ workspace layout
+// The counter block sits first and depends only on the handle, so counters keep their
+// place (and their zero value) whatever T successive calls use.
+struct Ws {
+    size_t ctr_tiles, ctr_group, ctr_rows, ctr_end;
+    size_t logits, topk_idx, topk_w, counts, offsets, perm, unique, n_unique;
+    size_t h, h_sh, y_assign, y_shared, x_stage, y_stage, total;
+};
+
+Ws ws_layout(const moe_layer_desc &d, int T)
+{
+    Ws w;
+    size_t o = 0;
+    const int max_tiles = (d.max_tokens + kRouterTokTile - 1) / kRouterTokTile;
+    w.ctr_tiles = o; o += (size_t)max_tiles * 4;
+    w.ctr_group = o; o += 4;
+    w.ctr_rows = o; o += (size_t)(d.hidden / kRowTile) * 4;
+    o = up256(o);
+    w.ctr_end = o;
+    const size_t Tk = (size_t)T * d.top_k;
+    w.logits = o; o = up256(o + (size_t)T * d.n_experts * 4);
+    w.topk_idx = o; o = up256(o + Tk * 4);
+    w.topk_w = o; o = up256(o + Tk * 4);
+    w.counts = o; o = up256(o + (size_t)d.n_experts * 4);
+    w.offsets = o; o = up256(o + (size_t)(d.n_experts + 1) * 4);
+    w.perm = o; o = up256(o + Tk * 4);
+    w.unique = o; o = up256(o + (size_t)d.n_experts * 4);
+    w.n_unique = o; o = up256(o + 4);
+    w.h = o; o = up256(o + Tk * d.inter * 2);
+    w.h_sh = o; o = up256(o + (size_t)T * d.inter_shared * 2 * (d.n_shared ? 1 : 0));
+    w.y_assign = o; o = up256(o + Tk * d.hidden * 4);
+    w.y_shared = o; o = up256(o + (size_t)T * d.hidden * 4 * (d.n_shared ? 1 : 0));
+    w.x_stage = o; o = up256(o + (size_t)T * d.hidden * 2);
+    w.y_stage = o; o = up256(o + (size_t)T * d.hidden * 2);
+    w.total = o;
+    return w;
+}
+
+template <typename P>
+P *at(void *ws, size_t off) { return reinterpret_cast<P *>(static_cast<char *>(ws) + off); }
+
+// ------------------------------------------------------------------ TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// bytes [experts][rows][row_bytes], box {box_inner bytes, 16 rows, 1 expert}
+bool make_map(CUtensorMap *m, const void *base, int row_bytes, int rows, int experts, int box_inner,
+              bool swizzle128)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)rows, (cuuint64_t)experts};
+    cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)row_bytes * (cuuint64_t)rows};
+    cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)kRowTile, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int validate_desc(const moe_layer_desc *d)
+{
+    if (!d) return MOE_ERR_INVALID_ARG;
+    const int kmul = d->format == MOE_FMT_NVFP4 ? 256 : 64;
+    if (d->format != MOE_FMT_INT4_ROWSCALE && d->format != MOE_FMT_NVFP4) return MOE_ERR_INVALID_ARG;
+    if (d->hidden <= 0 || d->hidden > 16384 || d->hidden % kmul) return MOE_ERR_INVALID_ARG;
+    if (d->inter <= 0 || d->inter > 16384 || d->inter % kmul) return MOE_ERR_INVALID_ARG;
+    if (d->n_shared != 0 && d->n_shared != 1) return MOE_ERR_INVALID_ARG;
+    if (d->n_shared && (d->inter_shared <= 0 || d->inter_shared > 16384 || d->inter_shared % kmul))
+        return MOE_ERR_INVALID_ARG;
+    if (d->n_experts < 1 || d->n_experts > kMaxExperts) return MOE_ERR_INVALID_ARG;
+    if (d->top_k < 1 || d->top_k > kMaxTopK || d->top_k > d->n_experts) return MOE_ERR_INVALID_ARG;
+    if (d->max_tokens < 1 || d->max_tokens > 65536) return MOE_ERR_INVALID_ARG;
+    if (!(d->routed_scaling == d->routed_scaling)) return MOE_ERR_INVALID_ARG;   // NaN
+    return MOE_OK;
+}
+
+int validate_weights(const moe_layer_desc *d, const moe_weights *w)
+{
+    if (!w) return MOE_ERR_INVALID_ARG;
+    const void *req[32];
+    int n = 0;
+    req[n++] = w->router_w; req[n++] = w->router_bias;
+    req[n++] = w->gate; req[n++] = w->up; req[n++] = w->down;
+    if (d->format == MOE_FMT_INT4_ROWSCALE) {
+        req[n++] = w->gate_scale; req[n++] = w->up_scale; req[n++] = w->down_scale;
+    } else {
+        req[n++] = w->gate_bscale; req[n++] = w->up_bscale; req[n++] = w->down_bscale;
+        req[n++] = w->gate_tscale; req[n++] = w->up_tscale; req[n++] = w->down_tscale;
+    }
+    if (d->n_shared) {
+        req[n++] = w->shared_gate; req[n++] = w->shared_up; req[n++] = w->shared_down;
+        if (d->format == MOE_FMT_INT4_ROWSCALE) {
+            req[n++] = w->shared_gate_scale; req[n++] = w->shared_up_scale; req[n++] = w->shared_down_scale;
+        } else {
+            req[n++] = w->shared_gate_bscale; req[n++] = w->shared_up_bscale; req[n++] = w->shared_down_bscale;
+            req[n++] = w->shared_gate_tscale; req[n++] = w->shared_up_tscale; req[n++] = w->shared_down_tscale;
+        }
+    }
+    for (int i = 0; i < n; ++i)
+        if (!req[i] || !aligned16(req[i])) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+int check_ws(const moe_layer *L, int T, void *ws, size_t bytes)
+{
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_WORKSPACE;
+    if (bytes < ws_layout(L->desc, T).total) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+LayerWeights layer_weights(const moe_layer *L)
+{
+    LayerWeights lw;
+    const moe_weights &w = L->w;
+    lw.router_w = w.router_w;
+    lw.router_bias = w.router_bias;
+    if (L->desc.format == MOE_FMT_NVFP4) {
+        lw.g_scale = w.gate_tscale; lw.u_scale = w.up_tscale; lw.d_scale = w.down_tscale;
+        lw.sh_g_scale = w.shared_gate_tscale; lw.sh_u_scale = w.shared_up_tscale;
+        lw.sh_d_scale = w.shared_down_tscale;
+    } else {
+        lw.g_scale = w.gate_scale; lw.u_scale = w.up_scale; lw.d_scale = w.down_scale;
+        lw.sh_g_scale = w.shared_gate_scale; lw.sh_u_scale = w.shared_up_scale;
+        lw.sh_d_scale = w.shared_down_scale;
+    }
+    return lw;
+}
+
+RouterParams router_params(const moe_layer *L, const uint16_t *x, int T, void *ws)
+{
+    const Ws W = ws_layout(L->desc, T);
+    RouterParams p = {};
+    p.x = x;
+    p.w = L->w.router_w;
+    p.bias = L->w.router_bias;
+    p.tile_counters = at<unsigned int>(ws, W.ctr_tiles);
+    p.group_counter = at<unsigned int>(ws, W.ctr_group);
+    p.status = L->d_status;
+    p.T = T;
+    p.H = L->desc.hidden;
+    p.E = L->desc.n_experts;
+    p.k = L->desc.top_k;
+    p.scaling = L->desc.routed_scaling;
+    p.experts_per_cta = kRouterEpc;
+    return p;
+}
+
+FfnParams ffn_params(const moe_layer *L, const uint16_t *x, int T, void *ws)
+{
+    const Ws W = ws_layout(L->desc, T);
+    FfnParams p = {};
+    p.T = T;
+    p.H = L->desc.hidden;
+    p.I = L->desc.inter;
+    p.I_sh = L->desc.inter_shared;
+    p.E = L->desc.n_experts;
+    p.k = L->desc.top_k;
+    p.n_shared = L->desc.n_shared;
+    p.fmt = L->desc.format;
+    p.x = x;
+    p.wt = layer_weights(L);
+    p.h = at<__half>(ws, W.h);
+    p.h_sh = at<__half>(ws, W.h_sh);
+    p.row_counters = at<unsigned int>(ws, W.ctr_rows);
+    p.status = L->d_status;
+    return p;
+}
+
+int ffn_grid(const moe_layer *L, bool gu) { return gu ? L->grid_gate_up : L->grid_down; }
+
+int run_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s)
+{
+    const Ws W = ws_layout(L->desc, T);
+    RouterParams rp = router_params(L, x, T, ws);
+    rp.logits = at<float>(ws, W.logits);
+    rp.topk_idx = at<int32_t>(ws, W.topk_idx);
+    rp.topk_w = at<float>(ws, W.topk_w);
+    rp.counts = at<int32_t>(ws, W.counts);
+    rp.offsets = at<int32_t>(ws, W.offsets);
+    rp.perm = at<int32_t>(ws, W.perm);
+    rp.unique = at<int32_t>(ws, W.unique);
+    rp.n_unique = at<int32_t>(ws, W.n_unique);
+    rp.do_gemv = 1;
+    rp.do_group = 1;
+    const int gx = (L->desc.n_experts + kRouterEpc - 1) / kRouterEpc;
+    const int gy = (T + kRouterTokTile - 1) / kRouterTokTile;
+    cudaError_t e = launch_router(rp, gx, gy, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+    FfnParams fp = ffn_params(L, x, T, ws);
+    fp.offsets = rp.offsets;
+    fp.perm = rp.perm;
+    fp.topk_w = rp.topk_w;
+    fp.y_assign = at<float>(ws, W.y_assign);
+    fp.y_shared = at<float>(ws, W.y_shared);
+    fp.y = y;
+    fp.fuse_combine = 1;
+    e = launch_ffn(L->maps, fp, true, ffn_grid(L, true), true, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    e = launch_ffn(L->maps, fp, false, ffn_grid(L, false), true, s);
+    return cuda_status(e);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_version(void) { return 100; }
+
+const char *moe_status_string(int status)
+{
+    switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+    case MOE_ERR_DEVICE_BOUNDS: return "MOE_ERR_DEVICE_BOUNDS";
+    default: return "MOE_ERR_UNKNOWN";
+    }
+}
+
+int moe_layer_create(const moe_layer_desc *desc, const moe_weights *weights, moe_layer **out)
+{
+    if (!out) return MOE_ERR_INVALID_ARG;
+    *out = nullptr;
+    int rc = validate_desc(desc);
+    if (rc) return rc;
+    rc = validate_weights(desc, weights);
+    if (rc) return rc;
+    moe_layer *L = new (std::nothrow) moe_layer();
+    if (!L) return MOE_ERR_CUDA;
+    L->desc = *desc;
+    L->w = *weights;
+    if (cudaGetDevice(&L->device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, L->device) != cudaSuccess) {
+        delete L;
+        return MOE_ERR_CUDA;
+    }
+    const moe_layer_desc &d = *desc;
+    const moe_weights &w = *weights;
+    const int H = d.hidden, I = d.inter, Is = d.inter_shared, E = d.n_experts;
+    bool ok = make_map(&L->maps.g, w.gate, H / 2, I, E, 128, true) &&
+              make_map(&L->maps.u, w.up, H / 2, I, E, 128, true) &&
+              make_map(&L->maps.d, w.down, I / 2, H, E, 128, true);
+    if (ok && d.n_shared)
+        ok = make_map(&L->maps.sh_g, w.shared_gate, H / 2, Is, 1, 128, true) &&
+             make_map(&L->maps.sh_u, w.shared_up, H / 2, Is, 1, 128, true) &&
+             make_map(&L->maps.sh_d, w.shared_down, Is / 2, H, 1, 128, true);
+    if (ok && d.format == MOE_FMT_NVFP4) {
+        ok = make_map(&L->maps.gb, w.gate_bscale, H / 16, I, E, 32, false) &&
+             make_map(&L->maps.ub, w.up_bscale, H / 16, I, E, 32, false) &&
+             make_map(&L->maps.db, w.down_bscale, I / 16, H, E, 32, false);
+        if (ok && d.n_shared)
+            ok = make_map(&L->maps.sh_gb, w.shared_gate_bscale, H / 16, Is, 1, 32, false) &&
+                 make_map(&L->maps.sh_ub, w.shared_up_bscale, H / 16, Is, 1, 32, false) &&
+                 make_map(&L->maps.sh_db, w.shared_down_bscale, Is / 16, H, 1, 32, false);
+    }
+    if (!ok) {
+        delete L;
+        return MOE_ERR_CUDA;
+    }
+    int occ_gu = 0, occ_d = 0;
+    if (ffn_occupancy(d.format, true, &occ_gu) != cudaSuccess ||
+        ffn_occupancy(d.format, false, &occ_d) != cudaSuccess || occ_gu < 1 || occ_d < 1) {
+        delete L;
+        return MOE_ERR_CUDA;
+    }
+    L->grid_gate_up = L->num_sms * occ_gu;
+    L->grid_down = L->num_sms * occ_d;
+    if (cudaMalloc(&L->d_status, 256) != cudaSuccess) {
+        delete L;
+        return MOE_ERR_CUDA;
+    }
+    if (cudaMemset(L->d_status, 0, 256) != cudaSuccess) {
+        cudaFree(L->d_status);
+        delete L;
+        return MOE_ERR_CUDA;
+    }
+    *out = L;
+    return MOE_OK;
+}
+
+int moe_layer_destroy(moe_layer *L)
+{
+    if (!L) return MOE_OK;
+    cudaFree(L->d_status);
+    delete L;
+    return MOE_OK;
+}
+
+size_t moe_workspace_size(const moe_layer *L, int T)
+{
+    if (!L || T < 0 || T > L->desc.max_tokens) return 0;
+    return ws_layout(L->desc, T).total;
+}
+
+int moe_route(const moe_layer *L, const uint16_t *x, int T, const float *logits_in, float *logits_out,
+              int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    if (!L || T < 0 || T > L->desc.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if ((!x && !logits_in) || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (x && !aligned16(x)) return MOE_ERR_INVALID_ARG;
+    int rc = check_ws(L, T, ws, ws_bytes);
+    if (rc) return rc;
+    const Ws W = ws_layout(L->desc, T);
+    RouterParams p = router_params(L, x, T, ws);
+    p.logits_in = logits_in;
+    p.logits = logits_in ? logits_out : (logits_out ? logits_out : at<float>(ws, W.logits));
+    p.topk_idx = topk_idx;
+    p.topk_w = topk_w;
+    p.do_gemv = logits_in ? 0 : 1;
+    p.do_group = 0;
+    const int gx = logits_in ? 1 : (L->desc.n_experts + kRouterEpc - 1) / kRouterEpc;
+    const int gy = (T + kRouterTokTile - 1) / kRouterTokTile;
+    return cuda_status(launch_router(p, gx, gy, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_group(const moe_layer *L, const int32_t *topk_idx, int T, int32_t *counts, int32_t *offsets,
+              int32_t *perm, int32_t *unique, int32_t *n_unique, void *ws, size_t ws_bytes,
+              moe_stream_t stream)
+{
+    if (!L || T < 0 || T > L->desc.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (!counts || !offsets || !unique || !n_unique || (T > 0 && (!topk_idx || !perm)))
+        return MOE_ERR_INVALID_ARG;
+    int rc = check_ws(L, T, ws, ws_bytes);
+    if (rc) return rc;
+    GroupParams p = {};
+    p.topk_idx = topk_idx;
+    p.counts = counts;
+    p.offsets = offsets;
+    p.perm = perm;
+    p.unique = unique;
+    p.n_unique = n_unique;
+    p.status = L->d_status;
+    p.T = T;
+    p.k = L->desc.top_k;
+    p.E = L->desc.n_experts;
+    return cuda_status(launch_group(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_expert_ffn(const moe_layer *L, const uint16_t *x, int T, const int32_t *offsets, const int32_t *perm,
+                   float *y_assign, float *y_shared, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    if (!L || T < 0 || T > L->desc.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !aligned16(x) || !offsets || !perm || !y_assign) return MOE_ERR_INVALID_ARG;
+    if (L->desc.n_shared && !y_shared) return MOE_ERR_INVALID_ARG;
+    int rc = check_ws(L, T, ws, ws_bytes);
+    if (rc) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    FfnParams fp = ffn_params(L, x, T, ws);
+    fp.offsets = offsets;
+    fp.perm = perm;
+    fp.y_assign = y_assign;
+    fp.y_shared = y_shared;
+    fp.fuse_combine = 0;
+    cudaError_t e = launch_ffn(L->maps, fp, true, ffn_grid(L, true), false, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    return cuda_status(launch_ffn(L->maps, fp, false, ffn_grid(L, false), true, s));
+}
+
+int moe_combine(const moe_layer *L, const float *y_assign, const float *y_shared, const float *topk_w,
+                int T, uint16_t *y, moe_stream_t stream)
+{
+    if (!L || T < 0 || T > L->desc.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!y_assign || !topk_w || !y || (L->desc.n_shared && !y_shared)) return MOE_ERR_INVALID_ARG;
+    CombineParams p = {};
+    p.y_assign = y_assign;
+    p.y_shared = y_shared;
+    p.topk_w = topk_w;
+    p.y = y;
+    p.T = T;
+    p.H = L->desc.hidden;
+    p.k = L->desc.top_k;
+    p.n_shared = L->desc.n_shared;
+    return cuda_status(launch_combine(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void *ws, size_t ws_bytes,
+                moe_stream_t stream)
+{
+    if (!L || T < 0 || T > L->desc.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !y || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+    int rc = check_ws(L, T, ws, ws_bytes);
+    if (rc) return rc;
+    return run_forward(L, x, T, y, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_forward_host(const moe_layer *L, const uint16_t *x_host, int T, uint16_t *y_host, void *ws,
+                     size_t ws_bytes, moe_stream_t stream)
+{
+    if (!L || T < 0 || T > L->desc.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x_host || !y_host) return MOE_ERR_INVALID_ARG;
+    int rc = check_ws(L, T, ws, ws_bytes);
+    if (rc) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Ws W = ws_layout(L->desc, T);
+    const size_t bytes = (size_t)T * L->desc.hidden * 2;
+    uint16_t *xd = at<uint16_t>(ws, W.x_stage), *yd = at<uint16_t>(ws, W.y_stage);
+    if (cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
+    rc = run_forward(L, xd, T, yd, ws, s);
+    if (rc) return rc;
+    return cuda_status(cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s));
+}
+
+int moe_get_device_status(const moe_layer *L, int *status)
+{
+    if (!L || !status) return MOE_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, L->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemset(L->d_status, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    *status = v;
+    return MOE_OK;
+}
+
+int moe_debug_wait_timeout(const moe_layer *L, long long max_iters, moe_stream_t stream)
+{
+    if (!L || max_iters < 1) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_wait_timeout(L->d_status, (unsigned long long)max_iters,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

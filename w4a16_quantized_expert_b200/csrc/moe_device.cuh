@@ -1,0 +1,196 @@
+// moe_device.cuh -- device-side building blocks shared by the MoE kernels (sm_100a).
+//
+// mbarrier waits are bounded (iteration count and %globaltimer deadline); a wait that
+// gives up records MOE_ERR_DEVICE_TIMEOUT in the layer's status word and lets the
+// kernel return instead of hanging.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ------------------------------------------------------------------ limits & status
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s: never reached when healthy
+constexpr unsigned long long kWaitMaxIters = 1ull << 30;
+
+__device__ __forceinline__ void record_error(int *status, int code)
+{
+    if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ------------------------------------------------------------------ mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 1000000;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Returns false (after recording
+// MOE_ERR_DEVICE_TIMEOUT) if the barrier did not complete in time.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *status,
+                                          unsigned long long timeout_ns = kWaitTimeoutNs,
+                                          unsigned long long max_iters = kWaitMaxIters)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (unsigned long long it = 1; it < max_iters; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15) == 0 && globaltimer_ns() - t0 > timeout_ns) break;
+    }
+    record_error(status, MOE_ERR_DEVICE_TIMEOUT);
+    return false;
+}
+
+// ------------------------------------------------------------------ TMA
+__device__ __forceinline__ uint64_t l2_evict_first_policy()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// 3-D tiled bulk tensor copy global -> shared, completing on an mbarrier (no multicast).
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *map, uint64_t *bar,
+                                            int c0, int c1, int c2, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
+        "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ------------------------------------------------------------------ PDL
+// Programmatic dependent launch: wait for the prerequisite grid (no-op without one)
+// and allow dependents to be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;"); }
+
+// ------------------------------------------------------------------ warp MMA
+__device__ __forceinline__ void ldmatrix_x4(uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3,
+                                            uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// D = A(16x16, f16, row) * B(16x8, f16, col) + D, fp32 accumulate.
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ------------------------------------------------------------------ dequantisation
+// int4 (two's complement, 8 codes in a 32-bit word, element i in bits 4i..4i+3) to four
+// fp16 pairs, exactly.  Each code is turned into offset binary (q + 8), placed in the
+// mantissa of the fp16 number 1024 (exponent trick: 0x6400 | m == 1024 + m), and the
+// bias is removed with one fp16 subtract (low nibbles) or one fma with 1/16 (high
+// nibbles, which sit 4 bits higher).  Output pairs hold elements (0,4), (1,5), (2,6),
+// (3,7) of the word: callers order the other operand the same way.
+__device__ __forceinline__ void dequant_int4_word(uint32_t w, uint32_t (&r)[4])
+{
+    w ^= 0x88888888u;
+    const uint32_t hi = w >> 8;
+    uint32_t t0 = (w & 0x000F000Fu) | 0x64006400u;
+    uint32_t t1 = (w & 0x00F000F0u) | 0x64006400u;
+    uint32_t t2 = (hi & 0x000F000Fu) | 0x64006400u;
+    uint32_t t3 = (hi & 0x00F000F0u) | 0x64006400u;
+    const uint32_t k1032 = 0x64086408u;   // 1032.0 in both halves
+    const uint32_t k1_16 = 0x2C002C00u;   // 0.0625
+    const uint32_t km72 = 0xD480D480u;    // -72.0
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r[0]) : "r"(t0), "r"(k1032));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[1]) : "r"(t1), "r"(k1_16), "r"(km72));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r[2]) : "r"(t2), "r"(k1032));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[3]) : "r"(t3), "r"(k1_16), "r"(km72));
+}
+
+// NVFP4 word (8 E2M1 codes) times one E4M3 block scale (given as an fp16 pair) to four
+// fp16 pairs, exactly (an E2M1 value times an E4M3 value has at most 6 significant bits
+// and lies in [2^-10, 2688]).  Output pairs hold elements (0,1), (2,3), (4,5), (6,7).
+__device__ __forceinline__ void dequant_nvfp4_word(uint32_t w, uint32_t scale2, uint32_t (&r)[4])
+{
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+        : "r"(w));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) asm("mul.rn.f16x2 %0, %0, %1;" : "+r"(r[i]) : "r"(scale2));
+}
+
+// one E4M3 byte -> the fp16 pair (v, v)
+__device__ __forceinline__ uint32_t e4m3_to_half2(uint32_t byte)
+{
+    uint32_t r;
+    const uint16_t two = static_cast<uint16_t>(byte | (byte << 8));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(two));
+    return r;
+}
+
+// (a.lo16, b.lo16) and (a.hi16, b.hi16)
+__device__ __forceinline__ uint32_t pack_lo(uint32_t a, uint32_t b) { return __byte_perm(a, b, 0x5410); }
+__device__ __forceinline__ uint32_t pack_hi(uint32_t a, uint32_t b) { return __byte_perm(a, b, 0x7632); }
+
+}  // namespace moe

@@ -1,0 +1,99 @@
+// moe_internal.h -- parameter blocks shared by the host dispatch and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 32;
+constexpr int kRouterTokTile = 16;     // tokens per router CTA
+constexpr int kRowTile = 16;           // output rows per expert work item (mma M)
+constexpr int kTokChunk = 32;          // tokens per expert work item (4 mma N-tiles)
+
+// Matrices of one layer in one format.  Routed tensors carry a leading expert index.
+struct LayerWeights {
+    const float *router_w, *router_bias;
+    // row scales (int4) or tensor scales (NVFP4), routed [E][rows] / [E], shared
+    const float *g_scale, *u_scale, *d_scale;
+    const float *sh_g_scale, *sh_u_scale, *sh_d_scale;
+};
+
+// TMA descriptors over the quantised weights (3-D: K bytes, rows, experts).
+struct LayerMaps {
+    CUtensorMap g, u, d;           // routed codes
+    CUtensorMap sh_g, sh_u, sh_d;  // shared codes (expert extent 1)
+    CUtensorMap gb, ub, db;        // NVFP4 routed block scales
+    CUtensorMap sh_gb, sh_ub, sh_db;
+};
+
+struct RouterParams {
+    const uint16_t *x;       // [T][H]
+    const float *w;          // [E][H]
+    const float *bias;       // [E]
+    const float *logits_in;  // optional [T][E]
+    float *logits;           // [T][E] (workspace or caller)
+    int32_t *topk_idx;       // [T][k]
+    float *topk_w;           // [T][k]
+    // grouping outputs (only when do_group)
+    int32_t *counts, *offsets, *perm, *unique, *n_unique;
+    unsigned int *tile_counters;  // [ceil(T/16)] expert-group CTAs done per token tile
+    unsigned int *group_counter;  // token tiles whose top-k is done
+    int *status;
+    int T, H, E, k;
+    float scaling;
+    int experts_per_cta;
+    int do_gemv, do_group;
+};
+
+struct GroupParams {
+    const int32_t *topk_idx;
+    int32_t *counts, *offsets, *perm, *unique, *n_unique;
+    int *status;
+    int T, k, E;
+};
+
+struct FfnParams {
+    // problem
+    int T, H, I, I_sh, E, k, n_shared, fmt;
+    const uint16_t *x;         // [T][H]
+    const int32_t *offsets;    // [E+1]
+    const int32_t *perm;       // [T*k]
+    const float *topk_w;       // [T][k] (fused combine only)
+    LayerWeights wt;
+    // intermediate / outputs
+    __half *h;                 // [T*k][I], rows in perm order, columns in mma order
+    __half *h_sh;              // [T][I_sh]
+    float *y_assign;           // [T*k][H]
+    float *y_shared;           // [T][H]
+    uint16_t *y;               // [T][H] fp16 (fused combine)
+    unsigned int *row_counters;  // [H/16] (fused combine)
+    int *status;
+    int fuse_combine;
+};
+
+struct CombineParams {
+    const float *y_assign, *y_shared, *topk_w;
+    uint16_t *y;
+    int T, H, k, n_shared;
+};
+
+}  // namespace moe
+
+// the opaque handle
+struct moe_layer {
+    moe_layer_desc desc;
+    moe_weights w;
+    moe::LayerMaps maps;
+    int *d_status;
+    int device;
+    int num_sms;
+    int grid_gate_up;   // persistent grid of the expert kernels (SMs x resident CTAs)
+    int grid_down;
+};
