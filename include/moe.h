@@ -201,6 +201,15 @@ int moe_get_device_status(const moe_layer *layer, int *status);
  * gives up, records MOE_ERR_DEVICE_TIMEOUT in the status word and returns. */
 int moe_debug_wait_timeout(const moe_layer *layer, long long max_iters, moe_stream_t stream);
 
+/* moe_forward for per-kernel timing: the same kernels on the same work, launched without
+ * programmatic dependent launch so that events[0..3] (cudaEvent_t handles, recorded on
+ * the stream) bracket them: [0] before the router, [1] after the router / before the
+ * expert gate/up kernel, [2] after gate/up / before the down kernel (which also
+ * combines), [3] after it.  For benchmarks and profiling, not for the hot path. */
+int moe_forward_timed(const moe_layer *layer, const uint16_t *x, int T, uint16_t *y,
+                      void *workspace, size_t workspace_bytes, moe_stream_t stream,
+                      void *const events[4]);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int moe_version(void);
 

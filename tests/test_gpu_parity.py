@@ -246,3 +246,13 @@ def test_device_wait_timeout_is_reported(tiny):
     # the context stays usable
     y, _ = _forward(tiny)
     assert y.shape == (tiny.T, 256)
+
+
+def test_handles_with_different_expert_counts_coexist(tiny):
+    """Kernel launch limits are per function: a later handle with a smaller E must not
+    break launches of an earlier handle with a larger one."""
+    small = _special(5, 2, 1, 1.0)
+    y_small, _ = _forward(small)
+    y, _ = _forward(tiny)
+    ref = tiny.oracle_forward()
+    check_y(y_to_f64(y), ref["y"], ref["gap"])

@@ -11,7 +11,8 @@ import ctypes
 import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libmoe.so")
+# W4A16_MOE_LIB selects another build of the same library (e.g. for A/B profiling)
+LIB_PATH = os.environ.get("W4A16_MOE_LIB") or os.path.join(PKG, "libmoe.so")
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1
@@ -80,10 +81,11 @@ def lib():
         L.moe_combine.argtypes = [vp, vp, vp, vp, c_int, vp, vp]
         L.moe_forward.argtypes = [vp, vp, c_int, vp, vp, c_size, vp]
         L.moe_forward_host.argtypes = [vp, vp, c_int, vp, vp, c_size, vp]
+        L.moe_forward_timed.argtypes = [vp, vp, c_int, vp, vp, c_size, vp, ctypes.POINTER(vp)]
         L.moe_get_device_status.argtypes = [vp, ctypes.POINTER(c_int)]
         L.moe_debug_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
         for f in ("moe_layer_create", "moe_layer_destroy", "moe_route", "moe_group",
-                  "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
+                  "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host", "moe_forward_timed",
                   "moe_get_device_status", "moe_debug_wait_timeout"):
             getattr(L, f).restype = c_int
         _lib = L
@@ -147,6 +149,11 @@ def moe_forward(layer, x, T, y, ws, ws_bytes, stream=0):
 def moe_forward_host(layer, x_host, T, y_host, ws, ws_bytes, stream=0):
     _check(lib().moe_forward_host(layer, x_host, T, y_host, ws, ws_bytes, stream),
            "moe_forward_host")
+
+
+def moe_forward_timed(layer, x, T, y, ws, ws_bytes, stream, events):
+    ev = (vp * 4)(*events)
+    _check(lib().moe_forward_timed(layer, x, T, y, ws, ws_bytes, stream, ev), "moe_forward_timed")
 
 
 def moe_get_device_status(layer) -> int:

@@ -6,22 +6,21 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <new>
 
 #include "moe_internal.h"
 
 namespace moe {
-cudaError_t launch_router(const RouterParams &p, int grid_x, int grid_y, cudaStream_t s);
+cudaError_t launch_router(const RouterParams &p, cudaStream_t s);
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams &p, cudaStream_t s);
-cudaError_t launch_ffn(const LayerMaps &maps, const FfnParams &p, bool gate_up, int grid, bool pdl,
+cudaError_t launch_ffn(const LayerMaps &maps, const FfnParams &p, bool gate_up, int ks, int grid, bool pdl,
                        cudaStream_t s);
-cudaError_t ffn_occupancy(int fmt, bool gu, int *blocks_per_sm);
+cudaError_t ffn_prepare(int fmt, int E, int occ[2][2][2]);
 cudaError_t launch_wait_timeout(int *status, unsigned long long max_iters, cudaStream_t s);
 
 namespace {
-
-constexpr int kRouterEpc = 2;   // router experts per CTA
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -30,9 +29,9 @@ size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
 // The counter block sits first and depends only on the handle, so counters keep their
 // place (and their zero value) whatever T successive calls use.
 struct Ws {
-    size_t ctr_tiles, ctr_group, ctr_rows, ctr_end;
-    size_t logits, topk_idx, topk_w, counts, offsets, perm, unique, n_unique;
-    size_t h, h_sh, y_assign, y_shared, x_stage, y_stage, total;
+    size_t ctr_tiles, ctr_group, ctr_rows, zrow, ctr_end;
+    size_t logits, score, sel, topk_idx, topk_w, counts, offsets, perm, unique, n_unique;
+    size_t x_perm, h, h_sh, y_assign, y_shared, x_stage, y_stage, total;
 };
 
 Ws ws_layout(const moe_layer_desc &d, int T)
@@ -44,9 +43,13 @@ Ws ws_layout(const moe_layer_desc &d, int T)
     w.ctr_group = o; o += 4;
     w.ctr_rows = o; o += (size_t)(d.hidden / kRowTile) * 4;
     o = up256(o);
+    // a row of zeros read by padding token columns (never written)
+    w.zrow = o; o = up256(o + (size_t)std::max(d.hidden, std::max(d.inter, d.inter_shared)) * 2);
     w.ctr_end = o;
     const size_t Tk = (size_t)T * d.top_k;
     w.logits = o; o = up256(o + (size_t)T * d.n_experts * 4);
+    w.score = o; o = up256(o + (size_t)T * d.n_experts * 4);
+    w.sel = o; o = up256(o + (size_t)T * d.n_experts * 4);
     w.topk_idx = o; o = up256(o + Tk * 4);
     w.topk_w = o; o = up256(o + Tk * 4);
     w.counts = o; o = up256(o + (size_t)d.n_experts * 4);
@@ -54,6 +57,7 @@ Ws ws_layout(const moe_layer_desc &d, int T)
     w.perm = o; o = up256(o + Tk * 4);
     w.unique = o; o = up256(o + (size_t)d.n_experts * 4);
     w.n_unique = o; o = up256(o + 4);
+    w.x_perm = o; o = up256(o + (size_t)T * d.hidden * 2);
     w.h = o; o = up256(o + Tk * d.inter * 2);
     w.h_sh = o; o = up256(o + (size_t)T * d.inter_shared * 2 * (d.n_shared ? 1 : 0));
     w.y_assign = o; o = up256(o + Tk * d.hidden * 4);
@@ -142,6 +146,10 @@ int validate_weights(const moe_layer_desc *d, const moe_weights *w)
     return MOE_OK;
 }
 
+// tokens per expert work item: 8 for decode-sized batches (a one-n-tile kernel with few
+// registers; a bucket of more tokens becomes several items), 32 otherwise
+int tok_chunk(int T) { return T <= 16 ? 8 : kTokChunk; }
+
 int check_ws(const moe_layer *L, int T, void *ws, size_t bytes)
 {
     if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_WORKSPACE;
@@ -176,6 +184,8 @@ RouterParams router_params(const moe_layer *L, const uint16_t *x, int T, void *w
     p.x = x;
     p.w = L->w.router_w;
     p.bias = L->w.router_bias;
+    p.score = at<float>(ws, W.score);
+    p.sel = at<float>(ws, W.sel);
     p.tile_counters = at<unsigned int>(ws, W.ctr_tiles);
     p.group_counter = at<unsigned int>(ws, W.ctr_group);
     p.status = L->d_status;
@@ -184,7 +194,6 @@ RouterParams router_params(const moe_layer *L, const uint16_t *x, int T, void *w
     p.E = L->desc.n_experts;
     p.k = L->desc.top_k;
     p.scaling = L->desc.routed_scaling;
-    p.experts_per_cta = kRouterEpc;
     return p;
 }
 
@@ -200,7 +209,12 @@ FfnParams ffn_params(const moe_layer *L, const uint16_t *x, int T, void *ws)
     p.k = L->desc.top_k;
     p.n_shared = L->desc.n_shared;
     p.fmt = L->desc.format;
+    p.dk = {0x000F000Fu, 0x00F000F0u, 0x64086408u, 0x64806480u, 0x64086408u, 0x2C002C00u, 0xD480D480u};
+    p.tok_chunk = tok_chunk(T);
     p.x = x;
+    p.xb = x;
+    p.xb_perm = 0;
+    p.zrow = at<uint16_t>(ws, W.zrow);
     p.wt = layer_weights(L);
     p.h = at<__half>(ws, W.h);
     p.h_sh = at<__half>(ws, W.h_sh);
@@ -209,10 +223,49 @@ FfnParams ffn_params(const moe_layer *L, const uint16_t *x, int T, void *ws)
     return p;
 }
 
-int ffn_grid(const moe_layer *L, bool gu) { return gu ? L->grid_gate_up : L->grid_down; }
+// Warp layout of an expert launch: KS = 1 (each warp owns 16 rows over the whole K) when
+// its 64-row items fill the persistent grid about as evenly as 16-row items would, else
+// KS = 4 (16-row items, K split four ways).  The number of non-empty experts is known
+// only on the device, so the bound min(E, T*k) is used.
+struct Launch {
+    int ks, grid;
+};
 
-int run_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s)
+Launch ffn_launch(const moe_layer *L, int T, bool gu)
 {
+    const moe_layer_desc &d = L->desc;
+    const int tc = tok_chunk(T);
+    const int wide = tc > 8;
+    const long slots = (long)std::min<long>(d.n_experts, (long)T * d.top_k);
+    const long chunks_sh = (T + tc - 1) / tc;
+    const long rows = gu ? d.inter : d.hidden;
+    const long rows_sh = gu ? d.inter_shared : d.hidden;
+    auto items = [&](int rw) {
+        return slots * (rows / (kRowTile * rw)) + (d.n_shared ? (rows_sh / (kRowTile * rw)) * chunks_sh : 0);
+    };
+    // balance per SM (the CTAs of one SM share its bandwidth): items per SM vs. average
+    auto eff = [&](long n) {
+        const long per_sm = (n + L->num_sms - 1) / L->num_sms;
+        return (double)n / (double)(per_sm * L->num_sms);
+    };
+    const long i1 = items(4), i4 = items(1);
+#ifdef MOE_FORCE_KS
+    if (MOE_FORCE_KS == 4) return {4, L->num_sms * L->occ[wide][gu][1]};
+    return {1, L->num_sms * L->occ[wide][gu][0]};
+#endif
+    if (i1 >= L->num_sms && eff(i1) >= 0.85 * eff(i4)) return {1, L->num_sms * L->occ[wide][gu][0]};
+    return {4, L->num_sms * L->occ[wide][gu][1]};
+}
+
+int run_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s,
+                void *const *events = nullptr)
+{
+    const bool pdl = events == nullptr;
+    auto rec = [&](int i) {
+        // external record nodes when captured, so the events also time graph replays
+        if (events) cudaEventRecordWithFlags(reinterpret_cast<cudaEvent_t>(events[i]), s, cudaEventRecordExternal);
+    };
+    rec(0);
     const Ws W = ws_layout(L->desc, T);
     RouterParams rp = router_params(L, x, T, ws);
     rp.logits = at<float>(ws, W.logits);
@@ -225,22 +278,31 @@ int run_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void 
     rp.n_unique = at<int32_t>(ws, W.n_unique);
     rp.do_gemv = 1;
     rp.do_group = 1;
-    const int gx = (L->desc.n_experts + kRouterEpc - 1) / kRouterEpc;
-    const int gy = (T + kRouterTokTile - 1) / kRouterTokTile;
-    cudaError_t e = launch_router(rp, gx, gy, s);
+    if (L->desc.format == MOE_FMT_INT4_ROWSCALE) rp.x_perm = at<uint16_t>(ws, W.x_perm);
+    cudaError_t e = launch_router(rp, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    rec(1);
 
     FfnParams fp = ffn_params(L, x, T, ws);
     fp.offsets = rp.offsets;
     fp.perm = rp.perm;
     fp.topk_w = rp.topk_w;
+    fp.unique = rp.unique;
+    if (rp.x_perm) {
+        fp.xb = rp.x_perm;
+        fp.xb_perm = 1;
+    }
+    fp.n_unique = rp.n_unique;
     fp.y_assign = at<float>(ws, W.y_assign);
     fp.y_shared = at<float>(ws, W.y_shared);
     fp.y = y;
     fp.fuse_combine = 1;
-    e = launch_ffn(L->maps, fp, true, ffn_grid(L, true), true, s);
+    const Launch lg = ffn_launch(L, T, true), ld = ffn_launch(L, T, false);
+    e = launch_ffn(L->maps, fp, true, lg.ks, lg.grid, pdl, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_ffn(L->maps, fp, false, ffn_grid(L, false), true, s);
+    rec(2);
+    e = launch_ffn(L->maps, fp, false, ld.ks, ld.grid, pdl, s);
+    rec(3);
     return cuda_status(e);
 }
 
@@ -295,26 +357,26 @@ int moe_layer_create(const moe_layer_desc *desc, const moe_weights *weights, moe
              make_map(&L->maps.sh_u, w.shared_up, H / 2, Is, 1, 128, true) &&
              make_map(&L->maps.sh_d, w.shared_down, Is / 2, H, 1, 128, true);
     if (ok && d.format == MOE_FMT_NVFP4) {
-        ok = make_map(&L->maps.gb, w.gate_bscale, H / 16, I, E, 32, false) &&
-             make_map(&L->maps.ub, w.up_bscale, H / 16, I, E, 32, false) &&
-             make_map(&L->maps.db, w.down_bscale, I / 16, H, E, 32, false);
+        ok = make_map(&L->maps.gb, w.gate_bscale, H / 16, I, E, 16, false) &&
+             make_map(&L->maps.ub, w.up_bscale, H / 16, I, E, 16, false) &&
+             make_map(&L->maps.db, w.down_bscale, I / 16, H, E, 16, false);
         if (ok && d.n_shared)
-            ok = make_map(&L->maps.sh_gb, w.shared_gate_bscale, H / 16, Is, 1, 32, false) &&
-                 make_map(&L->maps.sh_ub, w.shared_up_bscale, H / 16, Is, 1, 32, false) &&
-                 make_map(&L->maps.sh_db, w.shared_down_bscale, Is / 16, H, 1, 32, false);
+            ok = make_map(&L->maps.sh_gb, w.shared_gate_bscale, H / 16, Is, 1, 16, false) &&
+                 make_map(&L->maps.sh_ub, w.shared_up_bscale, H / 16, Is, 1, 16, false) &&
+                 make_map(&L->maps.sh_db, w.shared_down_bscale, Is / 16, H, 1, 16, false);
     }
     if (!ok) {
         delete L;
         return MOE_ERR_CUDA;
     }
-    int occ_gu = 0, occ_d = 0;
-    if (ffn_occupancy(d.format, true, &occ_gu) != cudaSuccess ||
-        ffn_occupancy(d.format, false, &occ_d) != cudaSuccess || occ_gu < 1 || occ_d < 1) {
+    bool occ_ok = ffn_prepare(d.format, d.n_experts, L->occ) == cudaSuccess;
+    for (int a = 0; a < 2; ++a)
+        for (int b = 0; b < 2; ++b)
+            for (int c = 0; c < 2; ++c) occ_ok = occ_ok && L->occ[a][b][c] >= 1;
+    if (!occ_ok) {
         delete L;
         return MOE_ERR_CUDA;
     }
-    L->grid_gate_up = L->num_sms * occ_gu;
-    L->grid_down = L->num_sms * occ_d;
     if (cudaMalloc(&L->d_status, 256) != cudaSuccess) {
         delete L;
         return MOE_ERR_CUDA;
@@ -359,9 +421,7 @@ int moe_route(const moe_layer *L, const uint16_t *x, int T, const float *logits_
     p.topk_w = topk_w;
     p.do_gemv = logits_in ? 0 : 1;
     p.do_group = 0;
-    const int gx = logits_in ? 1 : (L->desc.n_experts + kRouterEpc - 1) / kRouterEpc;
-    const int gy = (T + kRouterTokTile - 1) / kRouterTokTile;
-    return cuda_status(launch_router(p, gx, gy, reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_router(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int moe_group(const moe_layer *L, const int32_t *topk_idx, int T, int32_t *counts, int32_t *offsets,
@@ -403,9 +463,10 @@ int moe_expert_ffn(const moe_layer *L, const uint16_t *x, int T, const int32_t *
     fp.y_assign = y_assign;
     fp.y_shared = y_shared;
     fp.fuse_combine = 0;
-    cudaError_t e = launch_ffn(L->maps, fp, true, ffn_grid(L, true), false, s);
+    const Launch lg = ffn_launch(L, T, true), ld = ffn_launch(L, T, false);
+    cudaError_t e = launch_ffn(L->maps, fp, true, lg.ks, lg.grid, false, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    return cuda_status(launch_ffn(L->maps, fp, false, ffn_grid(L, false), true, s));
+    return cuda_status(launch_ffn(L->maps, fp, false, ld.ks, ld.grid, true, s));
 }
 
 int moe_combine(const moe_layer *L, const float *y_assign, const float *y_shared, const float *topk_w,
@@ -435,6 +496,18 @@ int moe_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void 
     int rc = check_ws(L, T, ws, ws_bytes);
     if (rc) return rc;
     return run_forward(L, x, T, y, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_forward_timed(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void *ws, size_t ws_bytes,
+                      moe_stream_t stream, void *const events[4])
+{
+    if (!L || T < 0 || T > L->desc.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (!events || !events[0] || !events[1] || !events[2] || !events[3]) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !y || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+    int rc = check_ws(L, T, ws, ws_bytes);
+    if (rc) return rc;
+    return run_forward(L, x, T, y, ws, reinterpret_cast<cudaStream_t>(stream), events);
 }
 
 int moe_forward_host(const moe_layer *L, const uint16_t *x_host, int T, uint16_t *y_host, void *ws,

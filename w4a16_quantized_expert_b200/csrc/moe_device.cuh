@@ -140,27 +140,40 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a
 }
 
 // ------------------------------------------------------------------ dequantisation
+// Constants of the int4 dequantisation.  They are passed to the kernels at run time so
+// that each lives in one register (or a constant-bank operand) for the whole kernel: as
+// compile-time literals the compiler splits the fused logic ops and rematerialises the
+// literals, which doubles the instruction count of the inner loop.
+struct DequantK {
+    uint32_t m_lo;    // 0x000F000F: low nibble of bytes 0 and 2
+    uint32_t m_hi;    // 0x00F000F0: high nibble of bytes 0 and 2
+    uint32_t x_lo;    // 0x64086408: 0x6400 (fp16 1024) | bit 3 of the low nibble
+    uint32_t x_hi;    // 0x64806480: 0x6400 | bit 3 of the high nibble
+    uint32_t h1032;   // fp16x2 1032
+    uint32_t h1_16;   // fp16x2 1/16
+    uint32_t hm72;    // fp16x2 -72
+};
+
 // int4 (two's complement, 8 codes in a 32-bit word, element i in bits 4i..4i+3) to four
-// fp16 pairs, exactly.  Each code is turned into offset binary (q + 8), placed in the
-// mantissa of the fp16 number 1024 (exponent trick: 0x6400 | m == 1024 + m), and the
-// bias is removed with one fp16 subtract (low nibbles) or one fma with 1/16 (high
-// nibbles, which sit 4 bits higher).  Output pairs hold elements (0,4), (1,5), (2,6),
-// (3,7) of the word: callers order the other operand the same way.
-__device__ __forceinline__ void dequant_int4_word(uint32_t w, uint32_t (&r)[4])
+// fp16 pairs, exactly.  Each code q is placed in the mantissa of the fp16 number 1024
+// (exponent trick: 0x6400 | m == 1024 + m) as q + 8: flipping bit 3 of a two's complement
+// nibble gives q + 8, and since the flip bit lies under the mask and 0x6400 outside it,
+// (w & mask) ^ (0x6400 | flip) is a single 3-input logic op.  The bias is then removed
+// with one fp16 subtract (low nibbles) or one fma with 1/16 (high nibbles, which sit
+// 4 bits higher).  Five integer and four fp16 ops per 8 weights.  Output pairs hold
+// elements (0,4), (1,5), (2,6), (3,7) of the word: callers order the other operand alike.
+__device__ __forceinline__ void dequant_int4_word(uint32_t w, uint32_t (&r)[4], const DequantK &k)
 {
-    w ^= 0x88888888u;
     const uint32_t hi = w >> 8;
-    uint32_t t0 = (w & 0x000F000Fu) | 0x64006400u;
-    uint32_t t1 = (w & 0x00F000F0u) | 0x64006400u;
-    uint32_t t2 = (hi & 0x000F000Fu) | 0x64006400u;
-    uint32_t t3 = (hi & 0x00F000F0u) | 0x64006400u;
-    const uint32_t k1032 = 0x64086408u;   // 1032.0 in both halves
-    const uint32_t k1_16 = 0x2C002C00u;   // 0.0625
-    const uint32_t km72 = 0xD480D480u;    // -72.0
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r[0]) : "r"(t0), "r"(k1032));
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[1]) : "r"(t1), "r"(k1_16), "r"(km72));
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r[2]) : "r"(t2), "r"(k1032));
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[3]) : "r"(t3), "r"(k1_16), "r"(km72));
+    uint32_t t0, t1, t2, t3;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t0) : "r"(w), "r"(k.m_lo), "r"(k.x_lo));   // (a & b) ^ c
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t1) : "r"(w), "r"(k.m_hi), "r"(k.x_hi));
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t2) : "r"(hi), "r"(k.m_lo), "r"(k.x_lo));
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t3) : "r"(hi), "r"(k.m_hi), "r"(k.x_hi));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r[0]) : "r"(t0), "r"(k.h1032));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[1]) : "r"(t1), "r"(k.h1_16), "r"(k.hm72));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r[2]) : "r"(t2), "r"(k.h1032));
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[3]) : "r"(t3), "r"(k.h1_16), "r"(k.hm72));
 }
 
 // NVFP4 word (8 E2M1 codes) times one E4M3 block scale (given as an fp16 pair) to four
@@ -187,6 +200,13 @@ __device__ __forceinline__ uint32_t e4m3_to_half2(uint32_t byte)
     const uint16_t two = static_cast<uint16_t>(byte | (byte << 8));
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(two));
     return r;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
 }
 
 // (a.lo16, b.lo16) and (a.hi16, b.hi16)

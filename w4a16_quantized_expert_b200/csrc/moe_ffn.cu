@@ -9,71 +9,107 @@
 // decoded in registers, never expanded to fp16 in memory: "GTX 1070向け35Bパラメータ
 // MoEモデル推論エンジン公開" (648news), "VRAMとシステムメモリで重みを分割する設計".
 //
-// Design (B200): the weight stream is the whole cost (2 flop per weight per token), so
-// every byte is read from HBM exactly once, by TMA, into a ring of shared-memory stages
-// (128-byte swizzled 16-row x 128-byte boxes, an L2 evict-first hint), while four
-// consumer warps turn the nibbles into fp16 in registers and feed them to mma.sync
-// m16n8k16 (the tensor cores are used as a wide dot-product engine: 256 weights per
-// instruction, which keeps the issue slots well below the HBM rate; CUDA-core FMA would
-// need ~3 instructions per weight and fall behind HBM).  Work items are
-// (expert slot, 16 output rows, up to 32 tokens); a persistent grid walks them with a
-// fixed stride, so the result does not depend on timing.  Split-K runs across the four
-// consumer warps and is reduced in a fixed order through shared memory.
+// Design (B200).  The weight stream is the whole cost (2 flop per weight per token), so
+// every byte is read from HBM once, by TMA, into a ring of shared-memory stages, while
+// four consumer warps turn nibbles into fp16 in registers and feed mma.sync m16n8k16:
+// the tensor cores serve as a wide dot-product engine (256 weights per instruction),
+// which keeps the issue slots below the HBM rate -- CUDA-core FMA would need about three
+// instructions per weight and fall behind.
 //
-// gate/up kernel: h = SiLU(g * sg) * (u * su) rounded to fp16, stored per bucket
-//                 position with each 8-column group in mma B-fragment order.
-// down kernel:    y_assign[a] = (W_d h) * sd (fp32); with fuse_combine, the last work
-//                 item of a 16-row tile also forms y = shared + sum_j w_j y_assign.
+// Warp layout RW x KS (RW * KS = 4 consumer warps).  A work item is (expert slot, 16*RW
+// output rows, up to 32 tokens).  Warp (rw, ks) owns rows [16 rw, 16 rw + 16) of the
+// item and K-box ks of every stage.  A stage holds, per matrix, RW*KS boxes of
+// 16 rows x 128 bytes (128-byte swizzle), i.e. 8 KB.  With KS = 1 every warp covers the
+// whole K of its rows, so the epilogue runs from registers with no cross-warp traffic;
+// with KS = 4 (small layers, to make enough items) the four K-slices are reduced in a
+// fixed order through shared memory.  The host picks RW per launch for load balance.
+// A persistent grid walks the items with a fixed stride, so results never depend on
+// timing.
 //
-// Programmatic dependent launch: the gate/up kernel starts the shared expert (which
-// needs no routing) before griddepcontrol.wait; the down kernel's producer streams its
-// weights before waiting for h.
+// gate/up: h = SiLU(g * sg) * (u * su) rounded to fp16, stored per bucket position with
+//          every 8-column group in the down kernel's B-fragment order.
+// down:    y_assign[a] = (W_d h) * sd in fp32; with fuse_combine, the last of the items
+//          writing a 16-row tile forms y = shared + sum_j w_j y_assign there.
+//
+// Programmatic dependent launch: the gate/up kernel runs the shared expert (no routing
+// needed) before griddepcontrol.wait; the down kernel's producer streams weights before
+// its consumers wait for h.
 #include <cuda_fp16.h>
 #include <math.h>
 
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
+#ifndef MOE_CHAINS
+#define MOE_CHAINS 1
+#endif
+#ifndef MOE_MIN_CTAS
+#define MOE_MIN_CTAS 2
+#endif
+
 namespace moe {
 
 constexpr int kConsumerWarps = 4;
 constexpr int kFfnThreads = (kConsumerWarps + 1) * 32;
-constexpr int kBoxBytes = 128;                 // K bytes per TMA box = swizzle span
-constexpr int kBoxesPerStage = 2;
-constexpr int kStageK = kBoxBytes * kBoxesPerStage;   // 256 bytes (512 weights) of K
-constexpr int kBoxSmem = kRowTile * kBoxBytes;        // 2 KB
-constexpr int kScaleRowBytes = kStageK / 8;           // NVFP4: one E4M3 per 16 weights
-constexpr int kScaleBoxSmem = kRowTile * kScaleRowBytes;   // 512 B
-constexpr int kStages = 6;
+constexpr int kBoxBytes = 128;          // K bytes per TMA box = swizzle span
+constexpr int kBoxSmem = kRowTile * kBoxBytes;     // 2 KB
+constexpr int kScaleBoxBytes = kBoxBytes / 8;      // NVFP4: one E4M3 per 16 weights = 16 B
+constexpr int kScaleBoxSmem = kRowTile * kScaleBoxBytes;   // 256 B
+constexpr int kMatStage = kConsumerWarps * kBoxSmem;       // 8 KB of codes per matrix
 
-template <int FMT, bool GU>
+template <int FMT, bool GU, int KS, int NNMAX>
 struct FfnCfg {
     static constexpr int kMats = GU ? 2 : 1;
+    static constexpr int kRW = kConsumerWarps / KS;
     static constexpr bool kNv = FMT == MOE_FMT_NVFP4;
-    static constexpr int kCodeBytes = kMats * kBoxesPerStage * kBoxSmem;
-    static constexpr int kStageBytes = kCodeBytes + (kNv ? kMats * 1024 : 0);
-    static constexpr int kRedFloats = kConsumerWarps * kMats * kTokChunk * kRowTile;
-    static constexpr size_t kSmem = 1024 /*align slack*/ + (size_t)kStages * kStageBytes +
-                                    (size_t)kRedFloats * 4 + (size_t)4 * (4 * (kMaxExperts + 2)) +
-                                    64 + (2 * kStages + 2) * 8;
+    static constexpr int kStageK = KS * kBoxBytes;        // K bytes per stage
+    static constexpr int kCodeBytes = kMats * kMatStage;
+    static constexpr int kScaleBytes = kNv ? kMats * kConsumerWarps * kScaleBoxSmem : 0;
+    // decode variant: the producer also copies each stage's slice of the (up to 8) token
+    // rows of the B operand into the stage, one 16-byte-padded row per token
+    static constexpr bool kSmemB = NNMAX == 1 && KS == 1;
+    static constexpr int kBRow = 4 * kStageK + 16;
+    static constexpr int kBOff = kCodeBytes + kScaleBytes;
+    static constexpr int kBBytes = kSmemB ? 8 * kBRow : 0;
+    static constexpr int kStageBytes = ((kCodeBytes + kScaleBytes + kBBytes) + 1023) / 1024 * 1024;
+    static constexpr int kStages = GU ? (kSmemB ? 3 : 4) : 5;   // 3 CTAs per SM where it matters
+    static constexpr int kZeroRow = kSmemB ? kBRow : 0;   // zero row read by padding lanes
+    static constexpr int kRedFloats = KS > 1 ? kConsumerWarps * kMats * kTokChunk * kRowTile : 0;
 };
+
+// dynamic shared memory of one CTA: ring + zero row + reduction + slot table + header/barriers
+template <int FMT, bool GU, int KS, int NNMAX>
+__host__ __device__ constexpr size_t ffn_smem(int E)
+{
+    using C = FfnCfg<FMT, GU, KS, NNMAX>;
+    return 1024 + (size_t)C::kStages * C::kStageBytes + C::kZeroRow + (size_t)C::kRedFloats * 4 +
+           (size_t)4 * 4 * (E + 2) + 64 + 8 + (2 * C::kStages + 2) * 8;
+}
+
+// 1-D bulk copy global -> shared completing on an mbarrier (16-byte aligned, size % 16 == 0)
+__device__ __forceinline__ void bulk_copy(void *smem_dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(smem_dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
 
 struct SlotTable {
     int *e;      // expert id, -1 = shared expert
     int *cnt;    // tokens in the bucket
     int *off;    // bucket start (position in perm)
     int *base;   // first item of the slot; base[n_slots] = total
-    int *hdr;    // [0] = n_slots, [1] = total items
+    int *hdr;    // [0] n_slots, [1] total items, [2] producer abort, [3] consumer fail
 };
 
 struct Item {
     int e;        // expert, -1 = shared
-    int row0;     // first output row
+    int row0;     // first output row of the item
     int tok0;     // first bucket position of the chunk (relative to the bucket)
     int ntok;     // tokens in the chunk (1..32)
     int boff;     // bucket start in perm order
     int K;        // input dimension of the matrix
-    int rows;
 };
 
 template <bool GU>
@@ -87,62 +123,44 @@ __device__ __forceinline__ int slot_K(const FfnParams &p, bool shared)
     return GU ? p.H : (shared ? p.I_sh : p.I);
 }
 
-template <bool GU>
+template <bool GU, int RW>
 __device__ __forceinline__ int shared_items(const FfnParams &p)
 {
     if (!p.n_shared) return 0;
-    return (slot_rows<GU>(p, true) / kRowTile) * ((p.T + kTokChunk - 1) / kTokChunk);
+    return (slot_rows<GU>(p, true) / (kRowTile * RW)) * ((p.T + p.tok_chunk - 1) / p.tok_chunk);
 }
 
-// Items of the shared slot are numbered first and need no routing information.
-template <bool GU>
-__device__ __forceinline__ Item shared_item(const FfnParams &p, int local)
+template <bool GU, int RW>
+__device__ __forceinline__ Item make_item(const FfnParams &p, int e, int cnt, int boff, int local)
 {
-    const int rows = slot_rows<GU>(p, true);
-    const int tiles = rows / kRowTile;
+    const bool shared = e < 0;
+    const int tiles = slot_rows<GU>(p, shared) / (kRowTile * RW);
     Item it;
-    it.e = -1;
-    it.row0 = (local % tiles) * kRowTile;
-    const int chunk = local / tiles;
-    it.tok0 = chunk * kTokChunk;
-    it.ntok = min(kTokChunk, p.T - it.tok0);
-    it.boff = 0;
-    it.K = slot_K<GU>(p, true);
-    it.rows = rows;
+    it.e = e;
+    it.row0 = (local % tiles) * kRowTile * RW;
+    it.tok0 = (local / tiles) * p.tok_chunk;
+    it.ntok = min(p.tok_chunk, cnt - it.tok0);
+    it.boff = boff;
+    it.K = slot_K<GU>(p, shared);
     return it;
 }
 
-template <bool GU>
+template <bool GU, int RW>
 __device__ Item decode_item(const FfnParams &p, const SlotTable &tb, int i)
 {
-    const int ns = tb.hdr[0];
-    int lo = 0, hi = ns - 1;   // last slot with base <= i
+    int lo = 0, hi = tb.hdr[0] - 1;   // last slot whose first item is <= i
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (tb.base[mid] <= i) lo = mid;
         else hi = mid - 1;
     }
-    const int s = lo;
-    const bool shared = tb.e[s] < 0;
-    const int rows = slot_rows<GU>(p, shared);
-    const int tiles = rows / kRowTile;
-    const int local = i - tb.base[s];
-    Item it;
-    it.e = tb.e[s];
-    it.row0 = (local % tiles) * kRowTile;
-    const int chunk = local / tiles;
-    it.tok0 = chunk * kTokChunk;
-    it.ntok = min(kTokChunk, tb.cnt[s] - it.tok0);
-    it.boff = tb.off[s];
-    it.K = slot_K<GU>(p, shared);
-    it.rows = rows;
-    return it;
+    return make_item<GU, RW>(p, tb.e[lo], tb.cnt[lo], tb.off[lo], i - tb.base[lo]);
 }
 
-// Slot table from the expert offsets: the shared expert first, then the non-empty
-// experts in ascending order.  Built by one warp.
-template <bool GU>
-__device__ void build_slot_table(const FfnParams &p, const SlotTable &tb)
+// Slot table: the shared expert first, then the non-empty experts in ascending order,
+// from the router's compact list when present, else by scanning the offsets.  One warp.
+template <bool GU, int RW>
+__device__ void build_slot_table(const FfnParams &p, const SlotTable &tb, int E)
 {
     const int lane = threadIdx.x & 31;
     int ns = 0, acc = 0;
@@ -154,24 +172,27 @@ __device__ void build_slot_table(const FfnParams &p, const SlotTable &tb)
             tb.base[0] = 0;
         }
         ns = 1;
-        acc = shared_items<GU>(p);
+        acc = shared_items<GU, RW>(p);
     }
-    const int rows = slot_rows<GU>(p, false);
-    const int tiles = rows / kRowTile;
-    for (int eb = 0; eb < p.E; eb += 32) {
-        const int e = eb + lane;
-        int cnt = 0, off = 0;
-        if (e < p.E) {
-            off = __ldcg(p.offsets + e);
-            cnt = __ldcg(p.offsets + e + 1) - off;
-            if (off < 0 || cnt < 0 || off + cnt > p.T * p.k) {   // inconsistent offsets
-                record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
+    const int tiles = slot_rows<GU>(p, false) / (kRowTile * RW);
+    const int n_scan = p.unique ? min(__ldcg(p.n_unique), E) : E;
+    for (int b = 0; b < n_scan; b += 32) {
+        const int j = b + lane;
+        int e = -1, cnt = 0, off = 0;
+        if (j < n_scan) {
+            e = p.unique ? __ldcg(p.unique + j) : j;
+            if (e >= 0 && e < E) {
+                off = __ldcg(p.offsets + e);
+                cnt = __ldcg(p.offsets + e + 1) - off;
+            }
+            if (e < 0 || e >= E || off < 0 || cnt < 0 || off + cnt > p.T * p.k) {
+                if (p.unique || cnt != 0) record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
                 cnt = 0;
             }
         }
         const bool has = cnt > 0;
         const unsigned bal = __ballot_sync(0xffffffffu, has);
-        const int nit = has ? tiles * ((cnt + kTokChunk - 1) / kTokChunk) : 0;
+        const int nit = has ? tiles * ((cnt + p.tok_chunk - 1) / p.tok_chunk) : 0;
         int incl = nit;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -196,6 +217,30 @@ __device__ void build_slot_table(const FfnParams &p, const SlotTable &tb)
     __syncwarp();
 }
 
+// B-operand row of bucket column `col` of an item: an x row (gate/up; the permuted copy
+// unless perm_b) or an h row (down); NULL for padding columns or a bad index
+template <bool GU>
+__device__ __forceinline__ const uint16_t *item_brow(const FfnParams &p, const Item &it, int col, bool perm_b)
+{
+    if (col >= it.ntok) return nullptr;
+    const bool sh = it.e < 0;
+    const int bpos = it.tok0 + col;
+    if (GU) {
+        int t = bpos;
+        if (!sh) {
+            const int a = __ldg(p.perm + it.boff + bpos);
+            t = (a >= 0 && a < p.T * p.k) ? a / p.k : -1;
+            if (t < 0) {
+                record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
+                return nullptr;
+            }
+        }
+        return (perm_b ? p.x : p.xb) + (size_t)t * p.H;
+    }
+    return sh ? reinterpret_cast<const uint16_t *>(p.h_sh) + (size_t)bpos * p.I_sh
+              : reinterpret_cast<const uint16_t *>(p.h) + (size_t)(it.boff + bpos) * p.I;
+}
+
 // position of h column n inside its 8-column group, in the order the down kernel's
 // B fragments want it (int4: pairs (0,4)(1,5)(2,6)(3,7); NVFP4: natural order)
 template <int FMT>
@@ -212,41 +257,368 @@ __device__ __forceinline__ void consumer_sync()
     asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
 }
 
-template <int FMT, bool GU>
-__global__ void __launch_bounds__(kFfnThreads) ffn_kernel(const __grid_constant__ LayerMaps maps,
+// int4: the fp32 scale of row `row`; NVFP4: the fp32 scale of the whole matrix
+template <int FMT>
+__device__ __forceinline__ float mat_scale(const float *scales, int e, int rows, int row)
+{
+    const int ez = e < 0 ? 0 : e;
+    if (FMT == MOE_FMT_NVFP4) return scales[ez];
+    return scales[(size_t)ez * rows + row];
+}
+
+// Per-thread constants of a consumer warp.
+struct Lane {
+    int lane, g, tq, warp, rw, ks, bx;
+    uint32_t off[4];   // swizzled ldmatrix offsets of chunk pairs 0..3 inside a box
+    DequantK dk;
+};
+
+// B-operand row of each of a thread's four n-tiles
+struct BRows {
+    const uint16_t *r[4];
+};
+
+// One chunk pair (64 weights of each of the warp's 16 rows and of each matrix): ldmatrix,
+// dequantise in registers, NN n-tiles of mma.  X0/X1 hold the n-tile-0 B fragments.
+// independent accumulator chains per (matrix, n-tile): mma.sync results feed the next
+// mma on the same accumulator, so one chain per matrix would serialise a stage's 16 mma
+template <int NN>
+struct Chains {
+    static constexpr int P = MOE_CHAINS;
+};
+
+template <int FMT, bool GU, int KS, int NN, bool PERM>
+__device__ __forceinline__ void chunk_pair(const unsigned char *st, uint32_t abase, const Lane &L, int q, int kel,
+                                           const uint4 &X0, const uint4 &X1, const BRows &brow,
+                                           float (&acc)[GU ? 2 : 1][NN][Chains<NN>::P][4])
+{
+    using C = FfnCfg<FMT, GU, KS, 1>;   // the values used here do not depend on NNMAX
+    uint32_t A[C::kMats][2][2][4];   // [mat][chunk][row g / g+8][pairs]
+#pragma unroll
+    for (int m = 0; m < C::kMats; ++m) {
+        uint32_t r0, r1, r2, r3;
+        ldmatrix_x4(r0, r1, r2, r3, abase + m * kMatStage + L.off[q]);
+        if constexpr (C::kNv) {
+            const unsigned char *sc = st + C::kCodeBytes + (m * kConsumerWarps + L.bx) * kScaleBoxSmem;
+            const int b0 = 4 * q + (L.tq >> 1);       // block of (chunk 2q, word tq)
+            const uint32_t s00 = e4m3_to_half2(sc[L.g * kScaleBoxBytes + b0]);
+            const uint32_t s10 = e4m3_to_half2(sc[(L.g + 8) * kScaleBoxBytes + b0]);
+            const uint32_t s01 = e4m3_to_half2(sc[L.g * kScaleBoxBytes + b0 + 2]);
+            const uint32_t s11 = e4m3_to_half2(sc[(L.g + 8) * kScaleBoxBytes + b0 + 2]);
+            dequant_nvfp4_word(r0, s00, A[m][0][0]);
+            dequant_nvfp4_word(r1, s10, A[m][0][1]);
+            dequant_nvfp4_word(r2, s01, A[m][1][0]);
+            dequant_nvfp4_word(r3, s11, A[m][1][1]);
+        } else {
+            dequant_int4_word(r0, A[m][0][0], L.dk);
+            dequant_int4_word(r1, A[m][0][1], L.dk);
+            dequant_int4_word(r2, A[m][1][0], L.dk);
+            dequant_int4_word(r3, A[m][1][1], L.dk);
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < NN; ++n) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const uint4 X = n == 0 ? (c == 0 ? X0 : X1)
+                                   : __ldg(reinterpret_cast<const uint4 *>(brow.r[n] + kel + 32 * c + 8 * L.tq));
+            uint32_t b00, b01, b10, b11;
+            if constexpr (PERM) {
+                b00 = pack_lo(X.x, X.z);
+                b01 = pack_hi(X.x, X.z);
+                b10 = pack_lo(X.y, X.w);
+                b11 = pack_hi(X.y, X.w);
+            } else {
+                b00 = X.x;
+                b01 = X.y;
+                b10 = X.z;
+                b11 = X.w;
+            }
+            constexpr int P = Chains<NN>::P;
+#pragma unroll
+            for (int m = 0; m < C::kMats; ++m) {
+                mma_16816(acc[m][n][(2 * c) % P], A[m][c][0][0], A[m][c][1][0], A[m][c][0][1], A[m][c][1][1], b00, b01);
+                mma_16816(acc[m][n][(2 * c + 1) % P], A[m][c][0][2], A[m][c][1][2], A[m][c][0][3], A[m][c][1][3], b10, b11);
+            }
+        }
+    }
+}
+
+// One warp's share of one work item: the stages of the item (for each stage the B
+// fragments of the warp's K range are fetched before its weights are waited for, since
+// they do not depend on them), then the epilogue.  NN: n-tiles of 8 tokens.  PERM: the
+// int4 gate/up B operand arrives in natural order and is permuted here to the dequant
+// pair order (0,4)(1,5)(2,6)(3,7); otherwise it is already in fragment order.
+// Returns false (every consumer warp alike) when a wait gave up.
+template <int FMT, bool GU, int KS, int NNMAX, int NN, bool PERM>
+__device__ __forceinline__ bool consume_item(const FfnParams &p, const SlotTable tb, const Item it,
+                                          unsigned char *ring, uint64_t *full, uint64_t *empty, int &stage,
+                                          uint32_t &phase, const Lane L, const BRows brow, uint32_t zsm,
+                                          float *red, volatile int *cfail, volatile int *abort_flag)
+{
+    using C = FfnCfg<FMT, GU, KS, NNMAX>;
+    constexpr int S = C::kStages;
+    constexpr int RW = C::kRW;
+    const bool sh = it.e < 0;
+    const int Kb = it.K / 2;
+    const int nst = (Kb + C::kStageK - 1) / C::kStageK;
+    constexpr int P = Chains<NN>::P;
+    float part[C::kMats][NN][P][4];
+#pragma unroll
+    for (int m = 0; m < C::kMats; ++m)
+#pragma unroll
+        for (int n = 0; n < NN; ++n)
+#pragma unroll
+            for (int j = 0; j < P; ++j)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) part[m][n][j][c] = 0.f;
+
+    bool ok = true;
+    if constexpr (C::kSmemB) {
+        // B fragments from the stage's token rows in shared memory (padding lanes read
+        // the zero row)
+        for (int s = 0; s < nst; ++s) {
+            const int kbox = s * C::kStageK;
+            if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
+            const unsigned char *st = ring + (size_t)stage * C::kStageBytes;
+            const uint32_t abase = smem_u32(st + L.bx * kBoxSmem);
+            const uint32_t bsm = (L.g < it.ntok ? smem_u32(st + C::kBOff + L.g * C::kBRow) : zsm) + 16 * L.tq;
+            if (kbox + kBoxBytes <= Kb) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    chunk_pair<FMT, GU, KS, NN, PERM>(st, abase, L, q, 0, lds128(bsm + 128 * q),
+                                                      lds128(bsm + 128 * q + 64), brow, part);
+            } else {
+                const int npairs = kbox < Kb ? (Kb - kbox) / 32 : 0;
+                for (int q = 0; q < npairs; ++q)
+                    chunk_pair<FMT, GU, KS, NN, PERM>(st, abase, L, q, 0, lds128(bsm + 128 * q),
+                                                      lds128(bsm + 128 * q + 64), brow, part);
+            }
+            __syncwarp();
+            if (L.lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+    } else
+    for (int s = 0; s < nst; ++s) {
+        const int kbox = s * C::kStageK + L.ks * kBoxBytes;     // K byte of this warp's box
+        const uint16_t *b0 = brow.r[0] + 2 * kbox + 8 * L.tq;
+        if (kbox + kBoxBytes <= Kb) {
+            // full box: four chunk pairs, fully unrolled
+            uint4 xb[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) xb[c] = __ldg(reinterpret_cast<const uint4 *>(b0 + 32 * c));
+            if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
+            const unsigned char *st = ring + (size_t)stage * C::kStageBytes;
+            const uint32_t abase = smem_u32(st + L.bx * kBoxSmem);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                chunk_pair<FMT, GU, KS, NN, PERM>(st, abase, L, q, 2 * kbox + 64 * q, xb[2 * q], xb[2 * q + 1], brow, part);
+        } else {
+            // the last, partial box (or none): K is a multiple of 64, so whole chunk pairs
+            if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
+            const unsigned char *st = ring + (size_t)stage * C::kStageBytes;
+            const uint32_t abase = smem_u32(st + L.bx * kBoxSmem);
+            const int npairs = kbox < Kb ? (Kb - kbox) / 32 : 0;
+            for (int q = 0; q < npairs; ++q) {
+                const uint4 x0 = __ldg(reinterpret_cast<const uint4 *>(b0 + 64 * q));
+                const uint4 x1 = __ldg(reinterpret_cast<const uint4 *>(b0 + 64 * q + 32));
+                chunk_pair<FMT, GU, KS, NN, PERM>(st, abase, L, q, 2 * kbox + 64 * q, x0, x1, brow, part);
+            }
+        }
+        __syncwarp();
+        if (L.lane == 0) mbar_arrive(&empty[stage]);
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+    }
+    if (!ok) {
+        *cfail = 1;
+        *abort_flag = 1;
+    }
+    // the partial chains, summed in a fixed order
+    float acc[C::kMats][NN][4];
+#pragma unroll
+    for (int m = 0; m < C::kMats; ++m)
+#pragma unroll
+        for (int n = 0; n < NN; ++n)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float v = part[m][n][0][c];
+#pragma unroll
+                for (int j = 1; j < P; ++j) v += part[m][n][j][c];
+                acc[m][n][c] = v;
+            }
+
+    const int rows_all = slot_rows<GU>(p, sh);
+    const float *sc0 = GU ? (sh ? p.wt.sh_g_scale : p.wt.g_scale) : (sh ? p.wt.sh_d_scale : p.wt.d_scale);
+    const float *sc1 = sh ? p.wt.sh_u_scale : p.wt.u_scale;
+    const int tid = threadIdx.x;
+    if constexpr (KS == 1) {
+        // ------------------------------------------------ epilogue from registers
+        consumer_sync();   // only to agree on failure: all warps ran the same stages
+        if (*cfail) return false;
+#pragma unroll
+        for (int n = 0; n < NN; ++n)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int col = 8 * n + 2 * L.tq + (c & 1);
+                if (col >= it.ntok) continue;
+                const int row = it.row0 + L.rw * kRowTile + L.g + (c >> 1) * 8;
+                const int bpos = it.tok0 + col;
+                if (GU) {
+                    const float gv = acc[0][n][c] * mat_scale<FMT>(sc0, it.e, rows_all, row);
+                    const float uv = acc[C::kMats - 1][n][c] * mat_scale<FMT>(sc1, it.e, rows_all, row);
+                    const float hv = gv / (1.f + expf(-gv)) * uv;
+                    __half *dst = sh ? p.h_sh + (size_t)bpos * p.I_sh : p.h + (size_t)(it.boff + bpos) * p.I;
+                    dst[h_pos<FMT>(row)] = __float2half_rn(hv);
+                } else {
+                    const float yv = acc[0][n][c] * mat_scale<FMT>(sc0, it.e, rows_all, row);
+                    if (sh) {
+                        p.y_shared[(size_t)bpos * p.H + row] = yv;
+                    } else {
+                        const int a = __ldg(p.perm + it.boff + bpos);
+                        if (a >= 0 && a < p.T * p.k) p.y_assign[(size_t)a * p.H + row] = yv;
+                        else record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
+                    }
+                }
+            }
+        if (!GU && p.fuse_combine) {
+            // the last of the items writing this warp's 16-row tile combines it
+            const int tile = (it.row0 + L.rw * kRowTile) / kRowTile;
+            __threadfence();
+            __syncwarp();
+            unsigned last = 0;
+            if (L.lane == 0) {
+                int target = 0;
+                for (int s2 = 0; s2 < tb.hdr[0]; ++s2) target += (tb.cnt[s2] + p.tok_chunk - 1) / p.tok_chunk;
+                const unsigned old = atomicInc(p.row_counters + tile, (unsigned)target - 1u);
+                last = (old == (unsigned)target - 1u);
+            }
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (last) {
+                __threadfence();
+                for (int o = L.lane; o < p.T * kRowTile; o += 32) {
+                    const int t = o / kRowTile, row = tile * kRowTile + o % kRowTile;
+                    float yv = p.n_shared ? __ldcg(p.y_shared + (size_t)t * p.H + row) : 0.f;
+                    for (int j = 0; j < p.k; ++j)
+                        yv = fmaf(__ldg(p.topk_w + (size_t)t * p.k + j),
+                                  __ldcg(p.y_assign + ((size_t)t * p.k + j) * p.H + row), yv);
+                    p.y[(size_t)t * p.H + row] = __half_as_ushort(__float2half_rn(yv));
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ K-split epilogue (KS = 4)
+        // partial sums of the four K-slices -> shared memory [warp][mat][col][row]
+#pragma unroll
+        for (int m = 0; m < C::kMats; ++m)
+#pragma unroll
+            for (int n = 0; n < NN; ++n) {
+                float *r = red + ((L.warp * C::kMats + m) * kTokChunk) * kRowTile;
+                const int c0 = 8 * n + 2 * L.tq;
+                r[c0 * kRowTile + L.g] = acc[m][n][0];
+                r[(c0 + 1) * kRowTile + L.g] = acc[m][n][1];
+                r[c0 * kRowTile + L.g + 8] = acc[m][n][2];
+                r[(c0 + 1) * kRowTile + L.g + 8] = acc[m][n][3];
+            }
+        consumer_sync();
+        if (*cfail) return false;
+        for (int o = tid; o < it.ntok * kRowTile; o += kConsumerWarps * 32) {
+            const int r = o % kRowTile, col = o / kRowTile;
+            const int row = it.row0 + r;
+            float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                v0 += red[((w * C::kMats + 0) * kTokChunk + col) * kRowTile + r];
+                if (GU) v1 += red[((w * C::kMats + 1) * kTokChunk + col) * kRowTile + r];
+            }
+            const int bpos = it.tok0 + col;
+            if (GU) {
+                const float gv = v0 * mat_scale<FMT>(sc0, it.e, rows_all, row);
+                const float uv = v1 * mat_scale<FMT>(sc1, it.e, rows_all, row);
+                const float hv = gv / (1.f + expf(-gv)) * uv;
+                __half *dst = sh ? p.h_sh + (size_t)bpos * p.I_sh : p.h + (size_t)(it.boff + bpos) * p.I;
+                dst[h_pos<FMT>(row)] = __float2half_rn(hv);
+            } else {
+                const float yv = v0 * mat_scale<FMT>(sc0, it.e, rows_all, row);
+                if (sh) {
+                    p.y_shared[(size_t)bpos * p.H + row] = yv;
+                } else {
+                    const int a = __ldg(p.perm + it.boff + bpos);
+                    if (a >= 0 && a < p.T * p.k) p.y_assign[(size_t)a * p.H + row] = yv;
+                    else record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
+                }
+            }
+        }
+        consumer_sync();
+        if (!GU && p.fuse_combine) {
+            __shared__ int s_last;
+            const int tile = it.row0 / kRowTile;
+            if (tid == 0) {
+                int target = 0;
+                for (int s2 = 0; s2 < tb.hdr[0]; ++s2) target += (tb.cnt[s2] + p.tok_chunk - 1) / p.tok_chunk;
+                __threadfence();
+                const unsigned old = atomicInc(p.row_counters + tile, (unsigned)target - 1u);
+                s_last = (old == (unsigned)target - 1u);
+            }
+            consumer_sync();
+            if (s_last) {
+                __threadfence();
+                for (int o = tid; o < p.T * kRowTile; o += kConsumerWarps * 32) {
+                    const int t = o / kRowTile, row = it.row0 + o % kRowTile;
+                    float yv = p.n_shared ? __ldcg(p.y_shared + (size_t)t * p.H + row) : 0.f;
+                    for (int j = 0; j < p.k; ++j)
+                        yv = fmaf(__ldg(p.topk_w + (size_t)t * p.k + j),
+                                  __ldcg(p.y_assign + ((size_t)t * p.k + j) * p.H + row), yv);
+                    p.y[(size_t)t * p.H + row] = __half_as_ushort(__float2half_rn(yv));
+                }
+            }
+            consumer_sync();
+        }
+    }
+    (void)RW;
+    return true;
+}
+
+template <int FMT, bool GU, int KS, int NNMAX>
+__global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __grid_constant__ LayerMaps maps,
                                                           const FfnParams p)
 {
-    using C = FfnCfg<FMT, GU>;
+    using C = FfnCfg<FMT, GU, KS, NNMAX>;
+    constexpr int RW = C::kRW;
+    constexpr int S = C::kStages;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char *smem = reinterpret_cast<unsigned char *>(
+    unsigned char *ring = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char *ring = smem;
-    float *red = reinterpret_cast<float *>(ring + (size_t)kStages * C::kStageBytes);
+    unsigned char *zrow_sm = ring + (size_t)S * C::kStageBytes;
+    float *red = reinterpret_cast<float *>(zrow_sm + C::kZeroRow);
     int *tbl = reinterpret_cast<int *>(red + C::kRedFloats);
+    const int E = p.E;
     SlotTable tb;
     tb.e = tbl;
-    tb.cnt = tbl + (kMaxExperts + 2);
-    tb.off = tbl + 2 * (kMaxExperts + 2);
-    tb.base = tbl + 3 * (kMaxExperts + 2);
-    tb.hdr = tbl + 4 * (kMaxExperts + 2);
+    tb.cnt = tbl + (E + 2);
+    tb.off = tbl + 2 * (E + 2);
+    tb.base = tbl + 3 * (E + 2);
+    tb.hdr = tbl + 4 * (E + 2);
     volatile int *abort_flag = tb.hdr + 2;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(tb.hdr + 16);
-    uint64_t *full = bars, *empty = bars + kStages, *table_ready = bars + 2 * kStages;
+    volatile int *cfail = tb.hdr + 3;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(
+        (reinterpret_cast<uintptr_t>(tb.hdr + 16) + 7) & ~uintptr_t(7));
+    uint64_t *full = bars, *empty = bars + S, *table_ready = bars + 2 * S;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x;
     // Only the gate/up kernel runs shared-expert items before the slot table exists (they
     // need no routing).  The down kernel builds its table at once (no wait involved) and
     // its fused combine reads the table, so every one of its items goes through it.
-    const int n_sh_items = GU ? shared_items<GU>(p) : 0;
+    const int n_pre = GU ? shared_items<GU, RW>(p) : 0;
 
+    for (int i = tid; i < C::kZeroRow / 4; i += kFfnThreads) reinterpret_cast<uint32_t *>(zrow_sm)[i] = 0u;
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
         }
         mbar_init(table_ready, 1);
-        *abort_flag = 0;
+        tb.hdr[2] = 0;
         tb.hdr[3] = 0;
         fence_mbar_init();
     }
@@ -265,15 +637,13 @@ __global__ void __launch_bounds__(kFfnThreads) ffn_kernel(const __grid_constant_
         const uint64_t pol = l2_evict_first_policy();
         int stage = 0;
         uint32_t phase = 0;
-        bool ok = true, have_table = false;
-        int total = n_sh_items;
-        int issued_phase[kStages];
-        bool unconfirmed[kStages];
-        for (int s = 0; s < kStages; ++s) unconfirmed[s] = false, issued_phase[s] = 0;
+        bool ok = true, have_table = false, pdl_done = GU;
+        int total = n_pre;
+        uint32_t unconfirmed = 0, issued_phase = 0;   // bit s: stage s in flight / its parity
         for (int i = blockIdx.x; ok; i += G) {
-            if (i >= n_sh_items && !have_table) {
+            if (i >= n_pre && !have_table) {
                 if (GU) pdl_wait();
-                build_slot_table<GU>(p, tb);
+                build_slot_table<GU, RW>(p, tb, E);
                 if (lane == 0) mbar_arrive(table_ready);
                 have_table = true;
                 total = tb.hdr[1];
@@ -281,67 +651,115 @@ __global__ void __launch_bounds__(kFfnThreads) ffn_kernel(const __grid_constant_
             }
             if (i >= total) break;
             if (lane == 0) {
-                const Item it = (i < n_sh_items) ? shared_item<GU>(p, i) : decode_item<GU>(p, tb, i);
+                const Item it = (i < n_pre) ? make_item<GU, RW>(p, -1, p.T, 0, i) : decode_item<GU, RW>(p, tb, i);
                 const bool sh = it.e < 0;
                 const int ez = sh ? 0 : it.e;
                 const int Kb = it.K / 2;
-                const int nst = (Kb + kStageK - 1) / kStageK;
+                const int nst = (Kb + C::kStageK - 1) / C::kStageK;
+                // decode variant: token rows of the B operand, copied stage by stage
+                const uint16_t *brows[8];
+                int nb = 0;
+                if constexpr (C::kSmemB) {
+                    const bool perm_b = GU && FMT == MOE_FMT_INT4_ROWSCALE && (i < n_pre || !p.xb_perm);
+                    nb = min(it.ntok, 8);
+                    for (int j = 0; j < 8; ++j) brows[j] = j < nb ? item_brow<GU>(p, it, j, perm_b) : nullptr;
+                }
+                // The down kernel starts early (programmatic launch) and its B operand, h,
+                // comes from the gate/up kernel: its first stages get their weights at once
+                // and their h rows only after the grid dependency is resolved.
+                const int defer = (!GU && C::kSmemB && !pdl_done) ? min(nst, S) : 0;
                 for (int s = 0; s < nst; ++s) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
-                    unconfirmed[stage] = false;
-                    const int kb0 = s * kStageK;
-                    const int nbox = min(kBoxesPerStage, (Kb - kb0 + kBoxBytes - 1) / kBoxBytes);
-                    uint32_t tx = C::kMats * nbox * kBoxSmem + (C::kNv ? C::kMats * kScaleBoxSmem : 0);
+                    unconfirmed &= ~(1u << stage);
+                    const int kb0 = s * C::kStageK;
+                    const int nks = min(KS, (Kb - kb0 + kBoxBytes - 1) / kBoxBytes);
+                    const uint32_t bbytes = 4u * (uint32_t)min(C::kStageK, Kb - kb0);
+                    uint32_t tx = (uint32_t)C::kMats * RW * nks * (kBoxSmem + (C::kNv ? kScaleBoxSmem : 0));
+                    if constexpr (C::kSmemB) {
+                        for (int j = 0; j < nb; ++j) tx += brows[j] ? bbytes : 0u;
+                    }
                     mbar_arrive_expect_tx(&full[stage], tx);
                     unsigned char *st = ring + (size_t)stage * C::kStageBytes;
 #pragma unroll
                     for (int m = 0; m < C::kMats; ++m) {
                         const CUtensorMap *map = sh ? (m ? mS1 : mS0) : (m ? mA1 : mA0);
-                        for (int b = 0; b < nbox; ++b)
-                            tma_load_3d(st + (m * kBoxesPerStage + b) * kBoxSmem, map, &full[stage],
-                                        kb0 + b * kBoxBytes, it.row0, ez, pol);
-                        if (C::kNv) {
-                            const CUtensorMap *bm = sh ? (m ? bS1 : bS0) : (m ? bA1 : bA0);
-                            tma_load_3d(st + C::kCodeBytes + m * 1024, bm, &full[stage],
-                                        s * kScaleRowBytes, it.row0, ez, pol);
+                        const CUtensorMap *bm = sh ? (m ? bS1 : bS0) : (m ? bA1 : bA0);
+                        for (int rw = 0; rw < RW; ++rw)
+                            for (int ks = 0; ks < nks; ++ks) {
+                                const int bx = rw * KS + ks;
+                                tma_load_3d(st + m * kMatStage + bx * kBoxSmem, map, &full[stage],
+                                            kb0 + ks * kBoxBytes, it.row0 + rw * kRowTile, ez, pol);
+                                if (C::kNv)
+                                    tma_load_3d(st + C::kCodeBytes + (m * kConsumerWarps + bx) * kScaleBoxSmem, bm,
+                                                &full[stage], (kb0 + ks * kBoxBytes) / 8, it.row0 + rw * kRowTile,
+                                                ez, pol);
+                            }
+                    }
+                    if constexpr (C::kSmemB) {
+                        if (s >= defer) {
+                            for (int j = 0; j < nb; ++j)
+                                if (brows[j]) bulk_copy(st + C::kBOff + j * C::kBRow, brows[j] + 2 * kb0, bbytes, &full[stage]);
+                        }
+                        if (defer && s == defer - 1) {
+                            // h is complete once the gate/up grid is: the deferred rows now
+                            pdl_wait();
+                            pdl_done = true;
+                            int st2 = stage - (defer - 1);
+                            if (st2 < 0) st2 += S;
+                            for (int s2 = 0; s2 < defer; ++s2) {
+                                const int k2 = s2 * C::kStageK;
+                                const uint32_t b2 = 4u * (uint32_t)min(C::kStageK, Kb - k2);
+                                unsigned char *stg = ring + (size_t)st2 * C::kStageBytes;
+                                for (int j = 0; j < nb; ++j)
+                                    if (brows[j]) bulk_copy(stg + C::kBOff + j * C::kBRow, brows[j] + 2 * k2, b2, &full[st2]);
+                                if (++st2 == S) st2 = 0;
+                            }
                         }
                     }
-                    issued_phase[stage] = phase;
-                    unconfirmed[stage] = true;
-                    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    unconfirmed |= 1u << stage;
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) *abort_flag = 1;
             }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (*abort_flag) ok = false;
         }
-        if (!have_table && lane == 0) mbar_arrive(table_ready);  // nothing left: release consumers
+        if (!have_table && lane == 0) mbar_arrive(table_ready);  // release the consumers
         if (lane == 0 && !ok) {
             // let copies still in flight land before the CTA may exit
-            for (int s = 0; s < kStages; ++s)
-                if (unconfirmed[s]) mbar_wait(&full[s], issued_phase[s], p.status, 10000000ull);
+            for (int s = 0; s < S; ++s)
+                if (unconfirmed >> s & 1u) mbar_wait(&full[s], issued_phase >> s & 1u, p.status, 10000000ull);
         }
         return;
     }
 
     // ============================================================ consumer warps
-    const int g = lane >> 2, tq = lane & 3;
-    const int ctid = tid;   // 0..127
+    Lane L;
+    L.lane = lane;
+    L.g = lane >> 2;
+    L.tq = lane & 3;
+    L.warp = warp;
+    L.rw = warp / KS;
+    L.ks = warp % KS;
+    L.bx = L.rw * KS + L.ks;
+    L.dk = p.dk;
+    {
+        // ldmatrix: lane -> (row inside the 16-row box, first or second chunk of a pair)
+        const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int lch = lane >> 4;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) L.off[q] = lrow * kBoxBytes + ((((2 * q + lch) ^ (lrow & 7)) & 7) << 4);
+    }
     int stage = 0;
     uint32_t phase = 0;
     bool have_table = false;
-    int total = n_sh_items;
-    // ldmatrix lane address pieces
-    const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8;
-    const int lch = lane >> 4;
-    const int box = warp >> 1;
-    const int cbase = (warp & 1) * 4;
+    int total = n_pre;
 
     // cfail is written only by consumer warps and read only after a consumer barrier,
     // so all four warps take the same exit decision and meet at the same barriers.
-    volatile int *cfail = tb.hdr + 3;
     for (int i = blockIdx.x;; i += G) {
-        if (i >= n_sh_items && !have_table) {
+        if (i >= n_pre && !have_table) {
             if (!mbar_wait(table_ready, 0, p.status)) {
                 *cfail = 1;
                 *abort_flag = 1;
@@ -351,23 +769,22 @@ __global__ void __launch_bounds__(kFfnThreads) ffn_kernel(const __grid_constant_
             have_table = true;
             total = tb.hdr[1];
             if (GU) {
-                pdl_wait();     // h, topk and the routed buckets come from the router
+                pdl_wait();     // topk and the routed buckets come from the router
                 pdl_trigger();
             }
         }
         if (i >= total) break;
-        const Item it = (i < n_sh_items) ? shared_item<GU>(p, i) : decode_item<GU>(p, tb, i);
+        const Item it = (i < n_pre) ? make_item<GU, RW>(p, -1, p.T, 0, i) : decode_item<GU, RW>(p, tb, i);
         const bool sh = it.e < 0;
-        const int Kb = it.K / 2;
-        const int nst = (Kb + kStageK - 1) / kStageK;
-        const int nN = (it.ntok + 7) >> 3;
 
-        // B-operand rows of this thread's tokens (one per n-tile: column 8n + g)
-        const uint16_t *brow[4];
+        // B-operand rows of this thread's tokens (one per n-tile: column 8n + g); padding
+        // columns read a zero row, so no lane needs a select in the inner loop
+        const bool perm_b = GU && FMT == MOE_FMT_INT4_ROWSCALE && (i < n_pre || !p.xb_perm);
+        BRows brow;
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
-            const int col = 8 * n + g;
-            brow[n] = nullptr;
+            const int col = 8 * n + L.g;
+            brow.r[n] = p.zrow;
             if (col < it.ntok) {
                 const int bpos = it.tok0 + col;
                 if (GU) {
@@ -377,178 +794,34 @@ __global__ void __launch_bounds__(kFfnThreads) ffn_kernel(const __grid_constant_
                         t = (a >= 0 && a < p.T * p.k) ? a / p.k : -1;
                         if (t < 0) record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
                     }
-                    if (t >= 0) brow[n] = p.x + (size_t)t * p.H;
+                    if (t >= 0) brow.r[n] = (perm_b ? p.x : p.xb) + (size_t)t * p.H;
                 } else {
-                    brow[n] = sh ? reinterpret_cast<const uint16_t *>(p.h_sh) + (size_t)bpos * p.I_sh
+                    brow.r[n] = sh ? reinterpret_cast<const uint16_t *>(p.h_sh) + (size_t)bpos * p.I_sh
                                  : reinterpret_cast<const uint16_t *>(p.h) + (size_t)(it.boff + bpos) * p.I;
                 }
             }
         }
         if (!GU && i == blockIdx.x) pdl_wait();   // h is produced by the gate/up kernel
+        const uint32_t zsm = smem_u32(zrow_sm);
 
-        float acc[C::kMats][4][4];
-#pragma unroll
-        for (int m = 0; m < C::kMats; ++m)
-#pragma unroll
-            for (int n = 0; n < 4; ++n)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc[m][n][c] = 0.f;
-
-        bool ok = true;
-        for (int s = 0; s < nst; ++s) {
-            if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
-            const unsigned char *st = ring + (size_t)stage * C::kStageBytes;
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int cc = cbase + 2 * q;                       // chunk pair (cc, cc+1)
-                const int kbyte = s * kStageK + box * kBoxBytes + cc * 16;
-                if (kbyte >= Kb) continue;
-                const int ch = cc + lch;
-                const uint32_t off = lrow * kBoxBytes + (((ch ^ (lrow & 7)) & 7) << 4);
-                uint32_t A[C::kMats][2][2][4];   // [mat][chunk][row g / g+8][pairs]
-#pragma unroll
-                for (int m = 0; m < C::kMats; ++m) {
-                    uint32_t r0, r1, r2, r3;
-                    ldmatrix_x4(r0, r1, r2, r3,
-                                smem_u32(st + (m * kBoxesPerStage + box) * kBoxSmem) + off);
-                    if (C::kNv) {
-                        const unsigned char *sc = st + C::kCodeBytes + m * 1024;
-                        const int cis = box * 8 + cc;                 // chunk index in stage
-                        const int b0 = 2 * cis + (tq >> 1);
-                        const uint32_t s00 = e4m3_to_half2(sc[g * kScaleRowBytes + b0]);
-                        const uint32_t s10 = e4m3_to_half2(sc[(g + 8) * kScaleRowBytes + b0]);
-                        const uint32_t s01 = e4m3_to_half2(sc[g * kScaleRowBytes + b0 + 2]);
-                        const uint32_t s11 = e4m3_to_half2(sc[(g + 8) * kScaleRowBytes + b0 + 2]);
-                        dequant_nvfp4_word(r0, s00, A[m][0][0]);
-                        dequant_nvfp4_word(r1, s10, A[m][0][1]);
-                        dequant_nvfp4_word(r2, s01, A[m][1][0]);
-                        dequant_nvfp4_word(r3, s11, A[m][1][1]);
-                    } else {
-                        dequant_int4_word(r0, A[m][0][0]);
-                        dequant_int4_word(r1, A[m][0][1]);
-                        dequant_int4_word(r2, A[m][1][0]);
-                        dequant_int4_word(r3, A[m][1][1]);
-                    }
-                }
-                const int kel = 2 * kbyte;   // first weight index of chunk cc
-#pragma unroll
-                for (int n = 0; n < 4; ++n) {
-                    if (n >= nN) break;
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint4 X = make_uint4(0, 0, 0, 0);
-                        if (brow[n]) X = __ldg(reinterpret_cast<const uint4 *>(brow[n] + kel + 32 * c + 8 * tq));
-                        uint32_t b00, b01, b10, b11;
-                        if (GU && FMT == MOE_FMT_INT4_ROWSCALE) {
-                            b00 = pack_lo(X.x, X.z);
-                            b01 = pack_hi(X.x, X.z);
-                            b10 = pack_lo(X.y, X.w);
-                            b11 = pack_hi(X.y, X.w);
-                        } else {
-                            b00 = X.x;
-                            b01 = X.y;
-                            b10 = X.z;
-                            b11 = X.w;
-                        }
-#pragma unroll
-                        for (int m = 0; m < C::kMats; ++m) {
-                            mma_16816(acc[m][n], A[m][c][0][0], A[m][c][1][0], A[m][c][0][1],
-                                      A[m][c][1][1], b00, b01);
-                            mma_16816(acc[m][n], A[m][c][0][2], A[m][c][1][2], A[m][c][0][3],
-                                      A[m][c][1][3], b10, b11);
-                        }
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);
-            if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        const int nN = (it.ntok + 7) >> 3;
+        bool ok;
+        constexpr bool kPerm = GU && FMT == MOE_FMT_INT4_ROWSCALE;
+#define MOE_CONSUME(NN, PERM)                                                                                   \
+    consume_item<FMT, GU, KS, NNMAX, NN, PERM>(p, tb, it, ring, full, empty, stage, phase, L, brow, zsm, red, cfail, \
+                                               abort_flag)
+        // NNMAX = 1: items of at most 8 tokens (decode), one n-tile, few registers.
+        // NNMAX = 4: items of up to 32 tokens; 2 and 3 n-tiles run the 4-tile code
+        // (padding columns read the zero row), which keeps the kernel small.
+        if constexpr (NNMAX == 1) {
+            if (kPerm && perm_b) ok = MOE_CONSUME(1, kPerm);
+            else ok = MOE_CONSUME(1, false);
+        } else {
+            if (kPerm && perm_b) ok = nN == 1 ? MOE_CONSUME(1, kPerm) : MOE_CONSUME(4, kPerm);
+            else ok = nN == 1 ? MOE_CONSUME(1, false) : MOE_CONSUME(4, false);
         }
-        if (!ok) {
-            *cfail = 1;
-            *abort_flag = 1;
-        }
-
-        // ---------------------------------------------------------------- epilogue
-        // partial sums of the four K-slices -> shared memory [warp][mat][col][row]
-#pragma unroll
-        for (int m = 0; m < C::kMats; ++m)
-#pragma unroll
-            for (int n = 0; n < 4; ++n) {
-                if (n >= nN) break;
-                float *r = red + ((warp * C::kMats + m) * kTokChunk) * kRowTile;
-                const int c0 = 8 * n + 2 * tq;
-                r[c0 * kRowTile + g] = acc[m][n][0];
-                r[(c0 + 1) * kRowTile + g] = acc[m][n][1];
-                r[c0 * kRowTile + g + 8] = acc[m][n][2];
-                r[(c0 + 1) * kRowTile + g + 8] = acc[m][n][3];
-            }
-        consumer_sync();
-        if (*cfail) break;
-        for (int o = ctid; o < it.ntok * kRowTile; o += kConsumerWarps * 32) {
-            const int r = o % kRowTile, col = o / kRowTile;
-            const int row = it.row0 + r;
-            float v0 = 0.f, v1 = 0.f;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) {
-                v0 += red[((w * C::kMats + 0) * kTokChunk + col) * kRowTile + r];
-                if (GU) v1 += red[((w * C::kMats + 1) * kTokChunk + col) * kRowTile + r];
-            }
-            const int bpos = it.tok0 + col;
-            if (GU) {
-                float sg, su;
-                if (FMT == MOE_FMT_NVFP4) {
-                    sg = sh ? p.wt.sh_g_scale[0] : p.wt.g_scale[it.e];
-                    su = sh ? p.wt.sh_u_scale[0] : p.wt.u_scale[it.e];
-                } else {
-                    sg = sh ? p.wt.sh_g_scale[row] : p.wt.g_scale[(size_t)it.e * p.I + row];
-                    su = sh ? p.wt.sh_u_scale[row] : p.wt.u_scale[(size_t)it.e * p.I + row];
-                }
-                const float gv = v0 * sg, uv = v1 * su;
-                const float hv = gv / (1.f + expf(-gv)) * uv;
-                __half *dst = sh ? p.h_sh + (size_t)bpos * p.I_sh : p.h + (size_t)(it.boff + bpos) * p.I;
-                dst[h_pos<FMT>(row)] = __float2half_rn(hv);
-            } else {
-                float sd;
-                if (FMT == MOE_FMT_NVFP4) sd = sh ? p.wt.sh_d_scale[0] : p.wt.d_scale[it.e];
-                else sd = sh ? p.wt.sh_d_scale[row] : p.wt.d_scale[(size_t)it.e * p.H + row];
-                const float yv = v0 * sd;
-                if (sh) {
-                    p.y_shared[(size_t)bpos * p.H + row] = yv;
-                } else {
-                    const int a = __ldg(p.perm + it.boff + bpos);
-                    if (a >= 0 && a < p.T * p.k) p.y_assign[(size_t)a * p.H + row] = yv;
-                    else record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
-                }
-            }
-        }
-        consumer_sync();
-
-        if (!GU && p.fuse_combine) {
-            // the last item to finish a 16-row tile combines it: y = shared + sum_j w_j y_j
-            __shared__ int s_last;
-            const int tile = it.row0 / kRowTile;
-            if (ctid == 0) {
-                int target = 0;   // items that write this row tile: every token chunk of every slot
-                for (int s2 = 0; s2 < tb.hdr[0]; ++s2) target += (tb.cnt[s2] + kTokChunk - 1) / kTokChunk;
-                __threadfence();
-                const unsigned old = atomicInc(p.row_counters + tile, (unsigned)target - 1u);
-                s_last = (old == (unsigned)target - 1u);
-            }
-            consumer_sync();
-            if (s_last) {
-                __threadfence();
-                for (int o = ctid; o < p.T * kRowTile; o += kConsumerWarps * 32) {
-                    const int t = o / kRowTile, row = it.row0 + o % kRowTile;
-                    float yv = p.n_shared ? __ldcg(p.y_shared + (size_t)t * p.H + row) : 0.f;
-                    for (int j = 0; j < p.k; ++j)
-                        yv = fmaf(__ldg(p.topk_w + (size_t)t * p.k + j),
-                                  __ldcg(p.y_assign + ((size_t)t * p.k + j) * p.H + row), yv);
-                    p.y[(size_t)t * p.H + row] = __half_as_ushort(__float2half_rn(yv));
-                }
-            }
-            consumer_sync();
-        }
+#undef MOE_CONSUME
+        if (!ok) break;
     }
 }
 
@@ -565,63 +838,76 @@ __global__ void wait_timeout_kernel(int *status, unsigned long long max_iters)
 }
 
 // ---------------------------------------------------------------------------- launchers
-template <int FMT, bool GU>
-static cudaError_t launch_ffn_t(const LayerMaps &maps, const FfnParams &p, int grid, bool pdl,
-                                cudaStream_t s)
+template <int FMT, bool GU, int KS, int NNMAX>
+static cudaError_t launch_t(const LayerMaps &maps, const FfnParams &p, int grid, bool pdl, cudaStream_t s)
 {
-    using C = FfnCfg<FMT, GU>;
-    auto kern = ffn_kernel<FMT, GU>;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kFfnThreads);
-    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.dynamicSmemBytes = ffn_smem<FMT, GU, KS, NNMAX>(p.E);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, maps, p);
+    return cudaLaunchKernelEx(&cfg, ffn_kernel<FMT, GU, KS, NNMAX>, maps, p);
 }
 
-size_t ffn_smem_bytes(int fmt, bool gu)
+template <int FMT, bool GU, int KS, int NNMAX>
+static cudaError_t prepare_t(int E, int *blocks_per_sm)
 {
-    if (fmt == MOE_FMT_NVFP4) return gu ? FfnCfg<1, true>::kSmem : FfnCfg<1, false>::kSmem;
-    return gu ? FfnCfg<0, true>::kSmem : FfnCfg<0, false>::kSmem;
+    // the limit is a property of the kernel, shared by every handle: set it for the
+    // largest expert count; the occupancy is that of this handle's launches
+    const size_t smem = ffn_smem<FMT, GU, KS, NNMAX>(E);
+    cudaError_t e = cudaFuncSetAttribute(ffn_kernel<FMT, GU, KS, NNMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)ffn_smem<FMT, GU, KS, NNMAX>(kMaxExperts));
+    if (e != cudaSuccess) return e;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, ffn_kernel<FMT, GU, KS, NNMAX>, kFfnThreads,
+                                                         smem);
 }
 
-cudaError_t ffn_occupancy(int fmt, bool gu, int *blocks_per_sm)
+// Sets the shared-memory limits of the expert kernels of a format and returns their
+// resident CTAs per SM: occ[nnmax == 4][gate_up][ks == 4].
+template <int FMT>
+static cudaError_t prepare_fmt(int E, int occ[2][2][2])
 {
-    const size_t smem = ffn_smem_bytes(fmt, gu);
     cudaError_t e;
-    if (fmt == MOE_FMT_NVFP4) {
-        if (gu) {
-            cudaFuncSetAttribute(ffn_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, ffn_kernel<1, true>, kFfnThreads, smem);
-        } else {
-            cudaFuncSetAttribute(ffn_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, ffn_kernel<1, false>, kFfnThreads, smem);
-        }
-    } else {
-        if (gu) {
-            cudaFuncSetAttribute(ffn_kernel<0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, ffn_kernel<0, true>, kFfnThreads, smem);
-        } else {
-            cudaFuncSetAttribute(ffn_kernel<0, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, ffn_kernel<0, false>, kFfnThreads, smem);
-        }
-    }
-    return e;
+    if ((e = prepare_t<FMT, true, 1, 1>(E, &occ[0][1][0])) != cudaSuccess) return e;
+    if ((e = prepare_t<FMT, true, 4, 1>(E, &occ[0][1][1])) != cudaSuccess) return e;
+    if ((e = prepare_t<FMT, false, 1, 1>(E, &occ[0][0][0])) != cudaSuccess) return e;
+    if ((e = prepare_t<FMT, false, 4, 1>(E, &occ[0][0][1])) != cudaSuccess) return e;
+    if ((e = prepare_t<FMT, true, 1, 4>(E, &occ[1][1][0])) != cudaSuccess) return e;
+    if ((e = prepare_t<FMT, true, 4, 4>(E, &occ[1][1][1])) != cudaSuccess) return e;
+    if ((e = prepare_t<FMT, false, 1, 4>(E, &occ[1][0][0])) != cudaSuccess) return e;
+    return prepare_t<FMT, false, 4, 4>(E, &occ[1][0][1]);
 }
 
-cudaError_t launch_ffn(const LayerMaps &maps, const FfnParams &p, bool gate_up, int grid, bool pdl,
+cudaError_t ffn_prepare(int fmt, int E, int occ[2][2][2])
+{
+    return fmt == MOE_FMT_NVFP4 ? prepare_fmt<MOE_FMT_NVFP4>(E, occ) : prepare_fmt<MOE_FMT_INT4_ROWSCALE>(E, occ);
+}
+
+template <int FMT>
+static cudaError_t launch_fmt(const LayerMaps &maps, const FfnParams &p, bool gu, int ks, int grid, bool pdl,
+                              cudaStream_t s)
+{
+    const bool wide = p.tok_chunk > 8;
+    if (gu) {
+        if (ks == 1) return wide ? launch_t<FMT, true, 1, 4>(maps, p, grid, pdl, s) : launch_t<FMT, true, 1, 1>(maps, p, grid, pdl, s);
+        return wide ? launch_t<FMT, true, 4, 4>(maps, p, grid, pdl, s) : launch_t<FMT, true, 4, 1>(maps, p, grid, pdl, s);
+    }
+    if (ks == 1) return wide ? launch_t<FMT, false, 1, 4>(maps, p, grid, pdl, s) : launch_t<FMT, false, 1, 1>(maps, p, grid, pdl, s);
+    return wide ? launch_t<FMT, false, 4, 4>(maps, p, grid, pdl, s) : launch_t<FMT, false, 4, 1>(maps, p, grid, pdl, s);
+}
+
+// p.tok_chunk (8 or 32) selects the kernel variant: 8-token items for decode batches,
+// 32-token items otherwise.
+cudaError_t launch_ffn(const LayerMaps &maps, const FfnParams &p, bool gate_up, int ks, int grid, bool pdl,
                        cudaStream_t s)
 {
-    if (p.fmt == MOE_FMT_NVFP4)
-        return gate_up ? launch_ffn_t<1, true>(maps, p, grid, pdl, s)
-                       : launch_ffn_t<1, false>(maps, p, grid, pdl, s);
-    return gate_up ? launch_ffn_t<0, true>(maps, p, grid, pdl, s)
-                   : launch_ffn_t<0, false>(maps, p, grid, pdl, s);
+    return p.fmt == MOE_FMT_NVFP4 ? launch_fmt<MOE_FMT_NVFP4>(maps, p, gate_up, ks, grid, pdl, s)
+                                  : launch_fmt<MOE_FMT_INT4_ROWSCALE>(maps, p, gate_up, ks, grid, pdl, s);
 }
 
 cudaError_t launch_wait_timeout(int *status, unsigned long long max_iters, cudaStream_t s)

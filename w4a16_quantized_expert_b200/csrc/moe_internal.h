@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include "../../include/moe.h"
+#include "moe_device.cuh"
 
 namespace moe {
 
@@ -35,20 +36,22 @@ struct LayerMaps {
 
 struct RouterParams {
     const uint16_t *x;       // [T][H]
+    uint16_t *x_perm;        // optional [T][H]: x with every 8-group in int4 B-fragment order
     const float *w;          // [E][H]
     const float *bias;       // [E]
     const float *logits_in;  // optional [T][E]
-    float *logits;           // [T][E] (workspace or caller)
+    float *logits;           // [T][E] (workspace or caller; may be NULL with logits_in)
+    float *score;            // [T][E] sigmoid scores (workspace)
+    float *sel;              // [T][E] selection scores s + bias (workspace)
     int32_t *topk_idx;       // [T][k]
     float *topk_w;           // [T][k]
     // grouping outputs (only when do_group)
     int32_t *counts, *offsets, *perm, *unique, *n_unique;
-    unsigned int *tile_counters;  // [ceil(T/16)] expert-group CTAs done per token tile
+    unsigned int *tile_counters;  // [ceil(T/16)] expert CTAs done per token tile
     unsigned int *group_counter;  // token tiles whose top-k is done
     int *status;
     int T, H, E, k;
     float scaling;
-    int experts_per_cta;
     int do_gemv, do_group;
 };
 
@@ -60,12 +63,19 @@ struct GroupParams {
 };
 
 struct FfnParams {
+    DequantK dk;               // int4 dequantisation constants (run-time values on purpose)
     // problem
     int T, H, I, I_sh, E, k, n_shared, fmt;
     const uint16_t *x;         // [T][H]
+    const uint16_t *xb;        // x in the B-fragment order of the int4 gate/up kernel, or x
+    const uint16_t *zrow;      // max(H, I, I_sh) zero halves (padding token columns)
+    int xb_perm;               // xb holds the permuted copy (else int4 gate/up permutes x)
+    int tok_chunk;             // tokens per work item: 8 (decode variant) or 32
     const int32_t *offsets;    // [E+1]
     const int32_t *perm;       // [T*k]
     const float *topk_w;       // [T][k] (fused combine only)
+    const int32_t *unique;     // optional compact list of non-empty experts (router output)
+    const int32_t *n_unique;
     LayerWeights wt;
     // intermediate / outputs
     __half *h;                 // [T*k][I], rows in perm order, columns in mma order
@@ -94,6 +104,5 @@ struct moe_layer {
     int *d_status;
     int device;
     int num_sms;
-    int grid_gate_up;   // persistent grid of the expert kernels (SMs x resident CTAs)
-    int grid_down;
+    int occ[2][2][2];   // resident CTAs per SM of the expert kernels [tok_chunk 32][gate_up][ks == 4]
 };

@@ -10,9 +10,13 @@
 // its tokens), in a fixed, deterministic order ("GLM-5.3-Flash 320B MoEを4枚のCMP
 // 170HXで動かすvLLMレシピ", section "Ampere世代のGPU向けに最適化された独自カーネル群").
 //
-// One launch serves moe_forward: CTAs (expert group, token tile) compute logits; the
-// last CTA to finish a token tile runs that tile's top-k; the last tile to finish runs
+// One launch serves moe_forward.  CTA (e, tile) computes expert e's logits for a tile of
+// up to 16 tokens (every weight load of the row in flight at once), then the sigmoid
+// and selection scores.  The last CTA of a tile runs that tile's top-k (a warp per
+// token, k rounds of redux.sync max/min on order-preserving keys); the last tile runs
 // the grouping.  Counters are reset by the CTA that consumes them (atomicInc wraps).
+// The kernel releases its programmatic dependents at once: the expert kernel starts the
+// shared expert while routing is still running.
 #include <cuda_fp16.h>
 #include <math.h>
 
@@ -21,58 +25,57 @@
 
 namespace moe {
 
-constexpr int kRouterThreads = 256;
-constexpr int kMaxEpc = 4;
+constexpr int kRouterThreads = 128;
+constexpr int kWPerThread = 16;          // float4 of a router row held per thread per pass
 
 __device__ __forceinline__ float sigmoid_ref(float logit)
 {
     return static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(logit))));
 }
 
+// order-preserving map of a float to an unsigned key (larger float -> larger key)
+__device__ __forceinline__ unsigned float_key(float v)
+{
+    const unsigned b = __float_as_uint(v);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
 // ---------------------------------------------------------------------------- top-k
-// One warp per token: k rounds of a warp-wide argmax over the selection scores.
-__device__ void topk_token(const float *logits_row, const float *bias, int E, int k,
+// One warp per token: k rounds, each one warp-wide max of the selection keys and one
+// min of the expert indices holding that max (equal scores -> lower expert index).
+__device__ void topk_token(const float *sel_row, const float *score_row, int E, int k,
                            float scaling, int32_t *idx_out, float *w_out)
 {
     const int lane = threadIdx.x & 31;
     constexpr int kPer = kMaxExperts / 32;
-    float sel[kPer];
-    uint32_t taken = 0;
+    const int nper = (E + 31) >> 5;
+    unsigned key[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
         const int e = lane + 32 * i;
-        sel[i] = -INFINITY;
-        if (e < E) sel[i] = sigmoid_ref(__ldcg(logits_row + e)) + bias[e];
+        key[i] = (i < nper && e < E) ? float_key(__ldcg(sel_row + e)) : 0u;
     }
+    uint32_t taken = 0;
     int my_idx = 0;
     for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
-        int be = 0x7fffffff;
+        unsigned bk = 0u, be = 0xffffffffu;
 #pragma unroll
         for (int i = 0; i < kPer; ++i) {
+            if (i >= nper) break;
             const int e = lane + 32 * i;
-            if (e < E && !(taken >> i & 1u) && (be == 0x7fffffff || sel[i] > bv)) {
-                bv = sel[i];
-                be = e;
+            if (e < E && !(taken >> i & 1u) && (be == 0xffffffffu || key[i] > bk)) {
+                bk = key[i];
+                be = (unsigned)e;
             }
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-            const bool take = (be == 0x7fffffff) ||
-                              (oe != 0x7fffffff && (ov > bv || (ov == bv && oe < be)));
-            if (take) {
-                bv = ov;
-                be = oe;
-            }
-        }
-        if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
-        if (lane == j) my_idx = be;
+        const unsigned kmax = __reduce_max_sync(0xffffffffu, bk);
+        const unsigned win = __reduce_min_sync(0xffffffffu, (be != 0xffffffffu && bk == kmax) ? be : 0xffffffffu);
+        if ((int)(win & 31u) == lane) taken |= 1u << (win >> 5);
+        if (lane == j) my_idx = (int)win;
     }
     // combine weights from the unbiased scores, summed in order j = 0..k-1
     double s_mine = 0.0;
-    if (lane < k) s_mine = static_cast<double>(sigmoid_ref(__ldcg(logits_row + my_idx)));
+    if (lane < k) s_mine = static_cast<double>(__ldcg(score_row + my_idx));
     double sum = 0.0;
     for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, s_mine, j);
     if (lane < k) {
@@ -102,39 +105,44 @@ __device__ void group_warp(const int32_t *topk_idx, int n, int E, int32_t *count
         if (e >= 0 && lane == __ffs(peers) - 1) sm_run[e] += __popc(peers);
         __syncwarp();
     }
-    // exclusive scan of counts -> offsets
-    int carry = 0;
-    for (int base = 0; base < E; base += 32) {
-        const int e = base + lane;
-        const int c = (e < E) ? sm_run[e] : 0;
-        int incl = c;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += v;
-        }
+    // exclusive scan of counts: lane handles experts [lane*P, lane*P + P)
+    const int P = (E + 31) >> 5;
+    const int e0 = lane * P;
+    int local = 0, nz = 0;
+    for (int i = 0; i < P; ++i) {
+        const int e = e0 + i;
         if (e < E) {
-            counts[e] = c;
-            offsets[e] = carry + incl - c;
-            sm_off[e] = carry + incl - c;
+            local += sm_run[e];
+            nz += sm_run[e] > 0;
         }
-        carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) {
-        offsets[E] = carry;
-        sm_off[E] = carry;
+    int incl = local, incl_nz = nz;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        const int u = __shfl_up_sync(0xffffffffu, incl_nz, off);
+        if (lane >= off) {
+            incl += v;
+            incl_nz += u;
+        }
     }
-    __syncwarp();
-    // unique experts, ascending
-    int nu = 0;
-    for (int base = 0; base < E; base += 32) {
-        const int e = base + lane;
-        const bool has = e < E && sm_run[e] > 0;
-        const unsigned b = __ballot_sync(0xffffffffu, has);
-        if (has) unique[nu + __popc(b & ((1u << lane) - 1u))] = e;
-        nu += __popc(b);
+    int run = incl - local, ur = incl_nz - nz;
+    for (int i = 0; i < P; ++i) {
+        const int e = e0 + i;
+        if (e < E) {
+            const int c = sm_run[e];
+            counts[e] = c;
+            offsets[e] = run;
+            sm_off[e] = run;
+            if (c > 0) unique[ur++] = e;
+            run += c;
+        }
     }
-    if (lane == 0) *n_unique = nu;
+    if (lane == 31) {
+        offsets[E] = incl;
+        sm_off[E] = incl;
+        *n_unique = incl_nz;
+    }
     __syncwarp();
     for (int e = lane; e < E; e += 32) sm_run[e] = 0;
     __syncwarp();
@@ -157,70 +165,89 @@ __device__ void group_warp(const int32_t *topk_idx, int n, int E, int32_t *count
 // ---------------------------------------------------------------------------- kernels
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p)
 {
-    __shared__ float red[kRouterThreads / 32][kMaxEpc * kRouterTokTile];
+    __shared__ float red[kRouterThreads / 32][kRouterTokTile];
     __shared__ int s_flag;
     __shared__ int sm_run[kMaxExperts];
     __shared__ int sm_off[kMaxExperts + 1];
 
+    pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tt = blockIdx.y;
     const int t0 = tt * kRouterTokTile;
     const int nt = min(kRouterTokTile, p.T - t0);
 
     if (p.do_gemv) {
-        const int e0 = blockIdx.x * p.experts_per_cta;
-        const int ne = min(p.experts_per_cta, p.E - e0);
-        float acc[kMaxEpc][kRouterTokTile];
-#pragma unroll
-        for (int i = 0; i < kMaxEpc; ++i)
-#pragma unroll
-            for (int t = 0; t < kRouterTokTile; ++t) acc[i][t] = 0.f;
+        // ------------------------------------------------ logits of expert e, this tile
+        const int e = blockIdx.x;
+        const float4 *wrow = reinterpret_cast<const float4 *>(p.w + (size_t)e * p.H);
         const int H4 = p.H >> 2;
-        for (int h4 = tid; h4 < H4; h4 += kRouterThreads) {
-            float4 wv[kMaxEpc];
+        float acc[kRouterTokTile];
 #pragma unroll
-            for (int i = 0; i < kMaxEpc; ++i)
-                if (i < ne) wv[i] = __ldg(reinterpret_cast<const float4 *>(p.w + (size_t)(e0 + i) * p.H) + h4);
+        for (int t = 0; t < kRouterTokTile; ++t) acc[t] = 0.f;
+        for (int base = 0; base < H4; base += kRouterThreads * kWPerThread) {
+            float4 wv[kWPerThread];
+#pragma unroll
+            for (int j = 0; j < kWPerThread; ++j) {
+                const int h4 = base + j * kRouterThreads + tid;
+                wv[j] = (h4 < H4) ? __ldg(wrow + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
 #pragma unroll
             for (int t = 0; t < kRouterTokTile; ++t) {
                 if (t < nt) {
-                    const uint2 xr = __ldg(reinterpret_cast<const uint2 *>(p.x + (size_t)(t0 + t) * p.H) + h4);
-                    const float2 xa = __half22float2(*reinterpret_cast<const __half2 *>(&xr.x));
-                    const float2 xb = __half22float2(*reinterpret_cast<const __half2 *>(&xr.y));
+                    const uint2 *xrow = reinterpret_cast<const uint2 *>(p.x + (size_t)(t0 + t) * p.H);
+                    float a = acc[t];
 #pragma unroll
-                    for (int i = 0; i < kMaxEpc; ++i)
-                        if (i < ne) {
-                            float a = acc[i][t];
-                            a = fmaf(wv[i].x, xa.x, a);
-                            a = fmaf(wv[i].y, xa.y, a);
-                            a = fmaf(wv[i].z, xb.x, a);
-                            a = fmaf(wv[i].w, xb.y, a);
-                            acc[i][t] = a;
+                    for (int j = 0; j < kWPerThread; ++j) {
+                        const int h4 = base + j * kRouterThreads + tid;
+                        if (h4 < H4) {
+                            const uint2 xr = __ldg(xrow + h4);
+                            const float2 xa = __half22float2(*reinterpret_cast<const __half2 *>(&xr.x));
+                            const float2 xb = __half22float2(*reinterpret_cast<const __half2 *>(&xr.y));
+                            a = fmaf(wv[j].x, xa.x, a);
+                            a = fmaf(wv[j].y, xa.y, a);
+                            a = fmaf(wv[j].z, xb.x, a);
+                            a = fmaf(wv[j].w, xb.y, a);
                         }
+                    }
+                    acc[t] = a;
+                }
+            }
+        }
+        if (p.x_perm && e == 0) {
+            // x with every 8-group as (0,4)(1,5)(2,6)(3,7): the B-fragment order of the int4
+            // gate/up kernel, so that its inner loop needs no permutes
+            const int H8 = p.H >> 3;
+            for (int t = 0; t < nt; ++t) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)(t0 + t) * p.H);
+                uint4 *dst = reinterpret_cast<uint4 *>(p.x_perm + (size_t)(t0 + t) * p.H);
+                for (int i = tid; i < H8; i += kRouterThreads) {
+                    const uint4 v = __ldg(src + i);
+                    dst[i] = make_uint4(pack_lo(v.x, v.z), pack_hi(v.x, v.z), pack_lo(v.y, v.w), pack_hi(v.y, v.w));
                 }
             }
         }
         // deterministic block reduction: butterfly inside warps, then warps in order
 #pragma unroll
-        for (int i = 0; i < kMaxEpc; ++i)
-#pragma unroll
-            for (int t = 0; t < kRouterTokTile; ++t) {
-                float v = acc[i][t];
+        for (int t = 0; t < kRouterTokTile; ++t) {
+            if (t < nt) {
+                float v = acc[t];
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                if (lane == 0) red[warp][i * kRouterTokTile + t] = v;
-            }
-        __syncthreads();
-        if (tid < p.experts_per_cta * kRouterTokTile) {
-            const int i = tid / kRouterTokTile, t = tid % kRouterTokTile;
-            if (i < ne && t < nt) {
-                float v = 0.f;
-#pragma unroll
-                for (int w = 0; w < kRouterThreads / 32; ++w) v += red[w][tid];
-                p.logits[(size_t)(t0 + t) * p.E + e0 + i] = v;
+                if (lane == 0) red[warp][t] = v;
             }
         }
-        // last CTA of this token tile runs its top-k
+        __syncthreads();
+        if (tid < nt) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kRouterThreads / 32; ++w) v += red[w][tid];
+            const size_t o = (size_t)(t0 + tid) * p.E + e;
+            const float s = sigmoid_ref(v);
+            p.logits[o] = v;
+            p.score[o] = s;
+            p.sel[o] = s + p.bias[e];
+        }
+        // the last CTA of this token tile runs its top-k
         __threadfence();
         __syncthreads();
         if (tid == 0) {
@@ -230,19 +257,26 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p)
         __syncthreads();
         if (!s_flag) return;
         __threadfence();
+    } else {
+        // ------------------------------------------------ scores from given logits
+        for (int i = tid; i < nt * p.E; i += kRouterThreads) {
+            const size_t o = (size_t)t0 * p.E + i;
+            const float l = p.logits_in[o];
+            const float s = sigmoid_ref(l);
+            if (p.logits) p.logits[o] = l;
+            p.score[o] = s;
+            p.sel[o] = s + p.bias[i % p.E];
+        }
+        __threadfence();
+        __syncthreads();
     }
 
-    const float *logits = p.do_gemv ? p.logits : p.logits_in;
     for (int t = warp; t < nt; t += kRouterThreads / 32)
-        topk_token(logits + (size_t)(t0 + t) * p.E, p.bias, p.E, p.k, p.scaling,
-                   p.topk_idx + (size_t)(t0 + t) * p.k, p.topk_w + (size_t)(t0 + t) * p.k);
-    if (p.logits_in && p.logits && tid < 32) {   // copy given logits when asked to
-        for (int i = lane; i < nt * p.E; i += 32)
-            p.logits[(size_t)t0 * p.E + i] = p.logits_in[(size_t)t0 * p.E + i];
-    }
+        topk_token(p.sel + (size_t)(t0 + t) * p.E, p.score + (size_t)(t0 + t) * p.E, p.E, p.k,
+                   p.scaling, p.topk_idx + (size_t)(t0 + t) * p.k, p.topk_w + (size_t)(t0 + t) * p.k);
     if (!p.do_group) return;
 
-    // last token tile runs the grouping
+    // the last token tile runs the grouping
     __threadfence();
     __syncthreads();
     if (tid == 0) {
@@ -277,9 +311,11 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p)
 }
 
 // ---------------------------------------------------------------------------- launchers
-cudaError_t launch_router(const RouterParams &p, int grid_x, int grid_y, cudaStream_t s)
+cudaError_t launch_router(const RouterParams &p, cudaStream_t s)
 {
-    router_kernel<<<dim3(grid_x, grid_y), kRouterThreads, 0, s>>>(p);
+    const int gx = p.do_gemv ? p.E : 1;
+    const int gy = (p.T + kRouterTokTile - 1) / kRouterTokTile;
+    router_kernel<<<dim3(gx, gy), kRouterThreads, 0, s>>>(p);
     return cudaGetLastError();
 }
 
