@@ -558,6 +558,8 @@ def main():
     ap.add_argument("--layers", type=int, default=None, help="rotating layer copies")
     ap.add_argument("--experts", type=int, default=None,
                     help="override E (smaller profiling-size layers; not a bench line)")
+    ap.add_argument("--hidden", type=int, default=None, help="override H (profiling only)")
+    ap.add_argument("--inter", type=int, default=None, help="override I and I_sh (profiling only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
@@ -565,6 +567,9 @@ def main():
     d = DEFAULTS.get(w.name, (1000, 50, 8))
     if args.experts:
         w = w.with_(E=args.experts, k=min(w.k, args.experts), name=f"{w.name}_e{args.experts}")
+    if args.hidden or args.inter:
+        w = w.with_(H=args.hidden or w.H, I=args.inter or w.I, I_sh=args.inter or w.I_sh,
+                    name=f"{w.name}_h{args.hidden or w.H}_i{args.inter or w.I}")
     if args.steps is None:
         args.steps = d[0]
     if args.warmup is None:
