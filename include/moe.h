@@ -150,6 +150,30 @@ int moe_route(const moe_layer *layer, const uint16_t *x, int T, const float *log
               float *logits_out, int32_t *topk_idx, float *topk_w, void *workspace,
               size_t workspace_bytes, moe_stream_t stream);
 
+/* moe_route without a workspace: the same kernel and the same results (bit-exact
+ * topk_idx and topk_w), with its scratch in a fixed static device array of the library
+ * (256 B of counters + 3 x 16384 floats, 196864 bytes, per device) instead of a caller
+ * buffer.  There is no counterpart in the method's sources: it is a convenience of this
+ * library for callers that have no workspace to pass and must not allocate, such as an
+ * engine that has already handed every free byte of the device to its KV cache, or a
+ * latency-critical loop in which the implicit device-wide synchronisation of
+ * cudaMalloc/cudaFree would stall the other streams.  This call allocates nothing; it
+ * makes no cudaMalloc, cudaFree or allocating library call.
+ * Limits: ceil(T / 16) <= 64 and T * n_experts <= 16384 (e.g. T <= 64 with 256
+ * experts); larger calls return MOE_ERR_WORKSPACE and launch nothing.  Other arguments
+ * and errors as moe_route.
+ * The first call on each device looks up the array's address (cudaGetSymbolAddress,
+ * which may load the module) and caches it; make that first call before any stream
+ * capture begins.
+ * The scratch is shared by every handle and stream of the device: calls that may
+ * overlap in time (other streams, other threads, other handles) race on it and must be
+ * serialised by the caller.  Its 64 tile counters must be zero when a call starts: they
+ * are zero at load and every complete call leaves them zero; after a device-side error
+ * (moe_get_device_status != MOE_OK) the counters may be left non-zero and this entry
+ * point must not be used again in the process. */
+int moe_route_static(const moe_layer *layer, const uint16_t *x, int T, const float *logits_in,
+                     float *logits_out, int32_t *topk_idx, float *topk_w, moe_stream_t stream);
+
 /* Step 3.  topk_idx [T][k] with values in [0, E) (out-of-range values set
  * MOE_ERR_DEVICE_BOUNDS and are dropped).  Outputs (int32): counts [E], offsets [E+1]
  * (exclusive prefix sum of counts), perm [T*k] (assignment ids a = t*k + j ordered by

@@ -76,6 +76,7 @@ def lib():
         L.moe_workspace_size.argtypes = [vp, c_int]
         L.moe_workspace_size.restype = c_size
         L.moe_route.argtypes = [vp, vp, c_int, vp, vp, vp, vp, vp, c_size, vp]
+        L.moe_route_static.argtypes = [vp, vp, c_int, vp, vp, vp, vp, vp]
         L.moe_group.argtypes = [vp, vp, c_int, vp, vp, vp, vp, vp, vp, c_size, vp]
         L.moe_expert_ffn.argtypes = [vp, vp, c_int, vp, vp, vp, vp, vp, c_size, vp]
         L.moe_combine.argtypes = [vp, vp, vp, vp, c_int, vp, vp]
@@ -84,7 +85,7 @@ def lib():
         L.moe_forward_timed.argtypes = [vp, vp, c_int, vp, vp, c_size, vp, ctypes.POINTER(vp)]
         L.moe_get_device_status.argtypes = [vp, ctypes.POINTER(c_int)]
         L.moe_debug_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
-        for f in ("moe_layer_create", "moe_layer_destroy", "moe_route", "moe_group",
+        for f in ("moe_layer_create", "moe_layer_destroy", "moe_route", "moe_route_static", "moe_group",
                   "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host", "moe_forward_timed",
                   "moe_get_device_status", "moe_debug_wait_timeout"):
             getattr(L, f).restype = c_int
@@ -126,6 +127,11 @@ def moe_workspace_size(layer: int, T: int) -> int:
 def moe_route(layer, x, T, logits_in, logits_out, topk_idx, topk_w, ws, ws_bytes, stream=0):
     _check(lib().moe_route(layer, x, T, logits_in, logits_out, topk_idx, topk_w, ws, ws_bytes,
                            stream), "moe_route")
+
+
+def moe_route_static(layer, x, T, logits_in, logits_out, topk_idx, topk_w, stream=0):
+    _check(lib().moe_route_static(layer, x, T, logits_in, logits_out, topk_idx, topk_w, stream),
+           "moe_route_static")
 
 
 def moe_group(layer, topk_idx, T, counts, offsets, perm, unique, n_unique, ws, ws_bytes, stream=0):

@@ -14,6 +14,7 @@
 namespace moe {
 cudaError_t launch_router(const RouterParams &p, cudaStream_t s);
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
+cudaError_t static_route_scratch(void **ptr);
 cudaError_t launch_combine(const CombineParams &p, cudaStream_t s);
 cudaError_t launch_ffn(const LayerMaps &maps, const FfnParams &p, bool gate_up, int ks, int grid, bool pdl,
                        cudaStream_t s);
@@ -419,6 +420,40 @@ int moe_route(const moe_layer *L, const uint16_t *x, int T, const float *logits_
     p.logits = logits_in ? logits_out : (logits_out ? logits_out : at<float>(ws, W.logits));
     p.topk_idx = topk_idx;
     p.topk_w = topk_w;
+    p.do_gemv = logits_in ? 0 : 1;
+    p.do_group = 0;
+    return cuda_status(launch_router(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_route_static(const moe_layer *L, const uint16_t *x, int T, const float *logits_in, float *logits_out,
+                     int32_t *topk_idx, float *topk_w, moe_stream_t stream)
+{
+    if (!L || T < 0 || T > L->desc.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if ((!x && !logits_in) || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (x && !aligned16(x)) return MOE_ERR_INVALID_ARG;
+    const int E = L->desc.n_experts;
+    if ((T + kRouterTokTile - 1) / kRouterTokTile > kStaticRouteTiles || (size_t)T * E > (size_t)kStaticRouteElems)
+        return MOE_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    if (static_route_scratch(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+    RouterParams p = {};
+    p.x = x;
+    p.w = L->w.router_w;
+    p.bias = L->w.router_bias;
+    p.tile_counters = at<unsigned int>(scratch, 0);
+    p.score = at<float>(scratch, kStaticRouteScore);
+    p.sel = at<float>(scratch, kStaticRouteSel);
+    p.logits_in = logits_in;
+    p.logits = logits_in ? logits_out : (logits_out ? logits_out : at<float>(scratch, kStaticRouteLogits));
+    p.topk_idx = topk_idx;
+    p.topk_w = topk_w;
+    p.status = L->d_status;
+    p.T = T;
+    p.H = L->desc.hidden;
+    p.E = E;
+    p.k = L->desc.top_k;
+    p.scaling = L->desc.routed_scaling;
     p.do_gemv = logits_in ? 0 : 1;
     p.do_group = 0;
     return cuda_status(launch_router(p, reinterpret_cast<cudaStream_t>(stream)));

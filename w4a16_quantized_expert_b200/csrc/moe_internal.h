@@ -15,6 +15,15 @@ namespace moe {
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kRouterTokTile = 16;     // tokens per router CTA
+// scratch of the allocation-free routing entry point: 64 token-tile counters (256 B),
+// then score, selection score and logits for up to kStaticRouteElems (token, expert) pairs
+constexpr int kStaticRouteTiles = 64;
+constexpr int kStaticRouteElems = 16384;
+constexpr size_t kStaticRouteScore = 256;
+constexpr size_t kStaticRouteSel = kStaticRouteScore + (size_t)kStaticRouteElems * 4;
+constexpr size_t kStaticRouteLogits = kStaticRouteSel + (size_t)kStaticRouteElems * 4;
+constexpr size_t kStaticRouteBytes = kStaticRouteLogits + (size_t)kStaticRouteElems * 4;
+constexpr int kStaticRouteDevices = 64;   // device ordinals whose scratch address is cached
 constexpr int kRowTile = 16;           // output rows per expert work item (mma M)
 constexpr int kTokChunk = 32;          // tokens per expert work item (4 mma N-tiles)
 

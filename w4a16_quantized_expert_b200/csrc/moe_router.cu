@@ -20,6 +20,8 @@
 #include <cuda_fp16.h>
 #include <math.h>
 
+#include <mutex>
+
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -308,6 +310,30 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p)
     for (int j = 0; j < p.k; ++j)
         acc = fmaf(p.topk_w[(size_t)t * p.k + j], p.y_assign[((size_t)t * p.k + j) * p.H + m], acc);
     p.y[i] = __half_as_ushort(__float2half_rn(acc));
+}
+
+// ---------------------------------------------------------------------------- static scratch
+// Scratch of moe_route_static, which allocates nothing: the router's token-tile
+// counters, then score, selection score and logits for kStaticRouteElems (token,
+// expert) pairs.  Zero at module load; the counters are brought back to zero by every
+// complete call (atomicInc wraps), the float arrays are written before they are read.
+static __device__ __align__(256) unsigned char g_route_scratch[kStaticRouteBytes];
+
+cudaError_t static_route_scratch(void **ptr)
+{
+    static std::mutex mu;
+    static void *addr[kStaticRouteDevices] = {};
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kStaticRouteDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        e = cudaGetSymbolAddress(&addr[dev], g_route_scratch);
+        if (e != cudaSuccess) return e;
+    }
+    *ptr = addr[dev];
+    return cudaSuccess;
 }
 
 // ---------------------------------------------------------------------------- launchers

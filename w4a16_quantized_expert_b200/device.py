@@ -10,7 +10,7 @@ import torch
 
 from . import (MOE_FMT_INT4_ROWSCALE, MOE_FMT_NVFP4, moe_combine, moe_expert_ffn,
                moe_forward, moe_forward_host, moe_group, moe_layer_create, moe_layer_desc,
-               moe_layer_destroy, moe_route, moe_weights, moe_workspace_size)
+               moe_layer_destroy, moe_route, moe_route_static, moe_weights, moe_workspace_size)
 
 # host array key -> moe_weights field
 _FIELD = {
@@ -107,6 +107,18 @@ class DeviceLayer:
                   logits_in.data_ptr() if logits_in is not None else None,
                   lo.data_ptr() if lo is not None else None, idx.data_ptr(), w.data_ptr(),
                   ws.data_ptr(), ws.numel(), self._stream(stream))
+        return idx, w, lo
+
+    def route_static(self, x, T, logits_in=None, want_logits=False, stream=None):
+        """moe_route with the library's static scratch instead of a workspace."""
+        k, E = self.d["k"], self.d["E"]
+        idx = torch.empty((T, k), dtype=torch.int32, device=self.device)
+        w = torch.empty((T, k), dtype=torch.float32, device=self.device)
+        lo = torch.empty((T, E), dtype=torch.float32, device=self.device) if want_logits else None
+        moe_route_static(self.handle, x.data_ptr() if x is not None else None, T,
+                         logits_in.data_ptr() if logits_in is not None else None,
+                         lo.data_ptr() if lo is not None else None, idx.data_ptr(), w.data_ptr(),
+                         self._stream(stream))
         return idx, w, lo
 
     def group(self, topk_idx, T, ws, stream=None):
