@@ -13,9 +13,11 @@
 
 namespace moe {
 cudaError_t launch_router(const RouterParams &p, cudaStream_t s);
+cudaError_t router_prepare();
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
 cudaError_t static_route_scratch(void **ptr);
-cudaError_t launch_combine(const CombineParams &p, cudaStream_t s);
+cudaError_t launch_combine(const CombineParams &p, bool pdl, cudaStream_t s);
+cudaError_t launch_x_limbs(const uint16_t *x, int T, int H, unsigned char *limbs, float *scale, cudaStream_t s);
 cudaError_t launch_ffn(const LayerMaps &maps, const FfnParams &p, bool gate_up, int ks, int grid, bool pdl,
                        cudaStream_t s);
 cudaError_t ffn_prepare(int fmt, int E, int occ[2][2][2]);
@@ -30,10 +32,17 @@ size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
 // The counter block sits first and depends only on the handle, so counters keep their
 // place (and their zero value) whatever T successive calls use.
 struct Ws {
-    size_t ctr_tiles, ctr_group, ctr_rows, zrow, ctr_end;
+    size_t ctr_tiles, ctr_group, ctr_chunks, zrow, ctr_end;
     size_t logits, score, sel, topk_idx, topk_w, counts, offsets, perm, unique, n_unique;
-    size_t x_perm, h, h_sh, y_assign, y_shared, x_stage, y_stage, total;
+    size_t x_perm, h, h_sh, y_assign, y_shared, x_stage, y_stage;
+    size_t x_limbs, x_limb_scale, h_limbs, h_limb_scale, hsh_limbs, hsh_limb_scale, total;
 };
+
+// bytes of one row of int8 limbs of a K-long operand (blocks of 256 values, 3 limbs)
+size_t limb_row_bytes(int K) { return (size_t)((K + kLimbBlockK - 1) / kLimbBlockK) * kLimbBlockBytes; }
+
+// the int4 expert kernels run on the int8 path for decode-sized batches (8-token items)
+bool use_limbs(const moe_layer_desc &d, int T) { return d.format == MOE_FMT_INT4_ROWSCALE && T <= 16; }
 
 Ws ws_layout(const moe_layer_desc &d, int T)
 {
@@ -42,7 +51,7 @@ Ws ws_layout(const moe_layer_desc &d, int T)
     const int max_tiles = (d.max_tokens + kRouterTokTile - 1) / kRouterTokTile;
     w.ctr_tiles = o; o += (size_t)max_tiles * 4;
     w.ctr_group = o; o += 4;
-    w.ctr_rows = o; o += (size_t)(d.hidden / kRowTile) * 4;
+    w.ctr_chunks = o; o += (size_t)d.max_tokens * (d.top_k + 1) * 4;
     o = up256(o);
     // a row of zeros read by padding token columns (never written)
     w.zrow = o; o = up256(o + (size_t)std::max(d.hidden, std::max(d.inter, d.inter_shared)) * 2);
@@ -65,6 +74,13 @@ Ws ws_layout(const moe_layer_desc &d, int T)
     w.y_shared = o; o = up256(o + (size_t)T * d.hidden * 4 * (d.n_shared ? 1 : 0));
     w.x_stage = o; o = up256(o + (size_t)T * d.hidden * 2);
     w.y_stage = o; o = up256(o + (size_t)T * d.hidden * 2);
+    const bool lb = use_limbs(d, T);
+    w.x_limbs = o; o = up256(o + (lb ? (size_t)T * limb_row_bytes(d.hidden) : 0));
+    w.x_limb_scale = o; o = up256(o + (lb ? (size_t)T * 4 : 0));
+    w.h_limbs = o; o = up256(o + (lb ? Tk * limb_row_bytes(d.inter) : 0));
+    w.h_limb_scale = o; o = up256(o + (lb ? Tk * 4 : 0));
+    w.hsh_limbs = o; o = up256(o + (lb && d.n_shared ? (size_t)T * limb_row_bytes(d.inter_shared) : 0));
+    w.hsh_limb_scale = o; o = up256(o + (lb && d.n_shared ? (size_t)T * 4 : 0));
     w.total = o;
     return w;
 }
@@ -219,8 +235,17 @@ FfnParams ffn_params(const moe_layer *L, const uint16_t *x, int T, void *ws)
     p.wt = layer_weights(L);
     p.h = at<__half>(ws, W.h);
     p.h_sh = at<__half>(ws, W.h_sh);
-    p.row_counters = at<unsigned int>(ws, W.ctr_rows);
     p.status = L->d_status;
+    if (use_limbs(L->desc, T)) {
+        p.limbs = 1;
+        p.x_limbs = at<unsigned char>(ws, W.x_limbs);
+        p.x_limb_scale = at<float>(ws, W.x_limb_scale);
+        p.h_limbs = at<unsigned char>(ws, W.h_limbs);
+        p.h_limb_scale = at<float>(ws, W.h_limb_scale);
+        p.hsh_limbs = at<unsigned char>(ws, W.hsh_limbs);
+        p.hsh_limb_scale = at<float>(ws, W.hsh_limb_scale);
+        p.chunk_counters = at<unsigned int>(ws, W.ctr_chunks);
+    }
     return p;
 }
 
@@ -249,6 +274,7 @@ Launch ffn_launch(const moe_layer *L, int T, bool gu)
         const long per_sm = (n + L->num_sms - 1) / L->num_sms;
         return (double)n / (double)(per_sm * L->num_sms);
     };
+    if (use_limbs(d, T)) return {1, L->num_sms * L->occ[0][gu][0]};   // the int8 path has KS = 1 only
     const long i1 = items(4), i4 = items(1);
 #ifdef MOE_FORCE_KS
     if (MOE_FORCE_KS == 4) return {4, L->num_sms * L->occ[wide][gu][1]};
@@ -279,7 +305,12 @@ int run_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void 
     rp.n_unique = at<int32_t>(ws, W.n_unique);
     rp.do_gemv = 1;
     rp.do_group = 1;
-    if (L->desc.format == MOE_FMT_INT4_ROWSCALE) rp.x_perm = at<uint16_t>(ws, W.x_perm);
+    if (use_limbs(L->desc, T)) {
+        rp.x_limbs = at<unsigned char>(ws, W.x_limbs);
+        rp.x_limb_scale = at<float>(ws, W.x_limb_scale);
+    } else if (L->desc.format == MOE_FMT_INT4_ROWSCALE) {
+        rp.x_perm = at<uint16_t>(ws, W.x_perm);
+    }
     cudaError_t e = launch_router(rp, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     rec(1);
@@ -297,12 +328,22 @@ int run_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void 
     fp.y_assign = at<float>(ws, W.y_assign);
     fp.y_shared = at<float>(ws, W.y_shared);
     fp.y = y;
-    fp.fuse_combine = 1;
     const Launch lg = ffn_launch(L, T, true), ld = ffn_launch(L, T, false);
     e = launch_ffn(L->maps, fp, true, lg.ks, lg.grid, pdl, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     rec(2);
     e = launch_ffn(L->maps, fp, false, ld.ks, ld.grid, pdl, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    CombineParams cp = {};
+    cp.y_assign = fp.y_assign;
+    cp.y_shared = fp.y_shared;
+    cp.topk_w = rp.topk_w;
+    cp.y = y;
+    cp.T = T;
+    cp.H = L->desc.hidden;
+    cp.k = L->desc.top_k;
+    cp.n_shared = L->desc.n_shared;
+    e = launch_combine(cp, pdl, s);
     rec(3);
     return cuda_status(e);
 }
@@ -370,7 +411,7 @@ int moe_layer_create(const moe_layer_desc *desc, const moe_weights *weights, moe
         delete L;
         return MOE_ERR_CUDA;
     }
-    bool occ_ok = ffn_prepare(d.format, d.n_experts, L->occ) == cudaSuccess;
+    bool occ_ok = router_prepare() == cudaSuccess && ffn_prepare(d.format, d.n_experts, L->occ) == cudaSuccess;
     for (int a = 0; a < 2; ++a)
         for (int b = 0; b < 2; ++b)
             for (int c = 0; c < 2; ++c) occ_ok = occ_ok && L->occ[a][b][c] >= 1;
@@ -497,8 +538,10 @@ int moe_expert_ffn(const moe_layer *L, const uint16_t *x, int T, const int32_t *
     fp.perm = perm;
     fp.y_assign = y_assign;
     fp.y_shared = y_shared;
-    fp.fuse_combine = 0;
     const Launch lg = ffn_launch(L, T, true), ld = ffn_launch(L, T, false);
+    if (fp.limbs && launch_x_limbs(x, T, L->desc.hidden, const_cast<unsigned char *>(fp.x_limbs),
+                                   const_cast<float *>(fp.x_limb_scale), s) != cudaSuccess)
+        return MOE_ERR_CUDA;
     cudaError_t e = launch_ffn(L->maps, fp, true, lg.ks, lg.grid, false, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     return cuda_status(launch_ffn(L->maps, fp, false, ld.ks, ld.grid, true, s));
@@ -519,7 +562,7 @@ int moe_combine(const moe_layer *L, const float *y_assign, const float *y_shared
     p.H = L->desc.hidden;
     p.k = L->desc.top_k;
     p.n_shared = L->desc.n_shared;
-    return cuda_status(launch_combine(p, reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_combine(p, false, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int moe_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void *ws, size_t ws_bytes,

@@ -116,6 +116,25 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
 // ------------------------------------------------------------------ PDL
 // Programmatic dependent launch: wait for the prerequisite grid (no-op without one)
 // and allow dependents to be scheduled.
+// Increment of a completion counter with acquire-release semantics at GPU scope (wraps
+// to 0 after `last`, as atomicInc); returns the old value.  Writers publish what they
+// (and, through a preceding barrier, their block) stored; the last arriver sees it all.
+__device__ __forceinline__ unsigned atom_inc_acq_rel(unsigned *ctr, unsigned last)
+{
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;" : "=r"(old) : "l"(ctr), "r"(last) : "memory");
+    return old;
+}
+
+// 1-D bulk copy global -> shared completing on an mbarrier (16-byte aligned, size % 16 == 0)
+__device__ __forceinline__ void bulk_copy(void *smem_dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(smem_dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;"); }
 
@@ -200,6 +219,104 @@ __device__ __forceinline__ uint32_t e4m3_to_half2(uint32_t byte)
     const uint16_t two = static_cast<uint16_t>(byte | (byte << 8));
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(two));
     return r;
+}
+
+// ------------------------------------------------------------------ int8 tensor path
+// mma m16n8k32, s8 x s8 -> s32, accumulating in place
+__device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// An int4 word (8 two's complement codes, element i in bits 4i..4i+3) as two words of
+// four s8 bytes each holding 16 x code: the odd elements are already in place in the
+// high half of each byte (a byte 0xq0 read as s8 is 16 q), the even ones move there with
+// a 4-bit left shift.  Byte j of `even` is element 2j, byte j of `odd` element 2j + 1.
+__device__ __forceinline__ void int4_word_to_s8x16(uint32_t w, uint32_t &even, uint32_t &odd)
+{
+    odd = w & 0xF0F0F0F0u;
+    even = (w << 4) & 0xF0F0F0F0u;
+}
+
+// Activation limbs.  A row of fp16 values v_k is written as X_k = round(v_k * 2^sh) with
+// one power-of-two exponent sh per row chosen so that max |X_k| lies in [2^21, 2^22), and
+// X_k = P0 + 256 P1 + 65536 P2 with s8 digits (|P2| <= 64).  Every v_k whose binary
+// exponent is at least 11 below the row maximum's is represented exactly; smaller ones
+// are rounded to a multiple of 2^-sh (error <= 2^-22 max |v|).  The limbs of a row are
+// stored per block of 256 K values as three 256-byte arrays (P0, P1, P2), each in the
+// order in which the int8 kernels load their B fragments: the 8 values starting at K
+// offset k8 (a multiple of 8 inside the block) go to the word at
+// 64 (k8 / 64) + 16 ((k8 / 8) % 4) + 4 ((k8 / 32) % 2) (even elements, bytes in order)
+// and to the word 8 bytes further (odd elements).
+constexpr int kLimbBlockK = 256;
+constexpr int kLimbBlockBytes = 3 * kLimbBlockK;
+
+__device__ __forceinline__ int limb_word_offset(int k8)
+{
+    return 64 * (k8 >> 6) + 16 * ((k8 >> 3) & 3) + 4 * ((k8 >> 5) & 1);
+}
+
+// exponent sh for a row whose largest magnitude is amax (finite); 0 for an all-zero row
+__device__ __forceinline__ int limb_shift(float amax)
+{
+    if (!(amax > 0.f)) return 0;
+    const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);  // amax in [2^(e-127), 2^(e-126))
+    return 148 - e;
+}
+
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }   // -126 <= e <= 127
+
+// the three limb digits of round(v * scale) (scale = 2^sh)
+__device__ __forceinline__ void limb_digits(float v, float scale, int &p0, int &p1, int &p2)
+{
+    const int X = __float2int_rn(v * scale);
+    p0 = static_cast<int>(static_cast<int8_t>(X & 0xFF));
+    const int X1 = (X - p0) / 256;     // exact: X - p0 is a multiple of 256
+    p1 = static_cast<int>(static_cast<int8_t>(X1 & 0xFF));
+    p2 = (X1 - p1) / 256;
+}
+
+// Encodes 8 consecutive fp16 values (k8 .. k8+7 of a block) into the block's limb arrays.
+__device__ __forceinline__ void limb_encode8(const uint4 v8, float scale, unsigned char *block, int k8)
+{
+    const __half2 *h = reinterpret_cast<const __half2 *>(&v8);
+    uint32_t ev[3] = {0u, 0u, 0u}, od[3] = {0u, 0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(h[j]);
+        int a0, a1, a2, b0, b1, b2;
+        limb_digits(f.x, scale, a0, a1, a2);
+        limb_digits(f.y, scale, b0, b1, b2);
+        ev[0] |= (uint32_t)(a0 & 0xFF) << (8 * j);
+        ev[1] |= (uint32_t)(a1 & 0xFF) << (8 * j);
+        ev[2] |= (uint32_t)(a2 & 0xFF) << (8 * j);
+        od[0] |= (uint32_t)(b0 & 0xFF) << (8 * j);
+        od[1] |= (uint32_t)(b1 & 0xFF) << (8 * j);
+        od[2] |= (uint32_t)(b2 & 0xFF) << (8 * j);
+    }
+    const int o = limb_word_offset(k8);
+#pragma unroll
+    for (int p = 0; p < 3; ++p) {
+        *reinterpret_cast<uint32_t *>(block + p * kLimbBlockK + o) = ev[p];
+        *reinterpret_cast<uint32_t *>(block + p * kLimbBlockK + o + 8) = od[p];
+    }
+}
+
+// largest |v| of 8 fp16 values
+__device__ __forceinline__ float amax8(const uint4 v8)
+{
+    const __half2 *h = reinterpret_cast<const __half2 *>(&v8);
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(h[j]);
+        m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+    return m;
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr)

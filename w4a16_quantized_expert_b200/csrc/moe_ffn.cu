@@ -28,8 +28,8 @@
 //
 // gate/up: h = SiLU(g * sg) * (u * su) rounded to fp16, stored per bucket position with
 //          every 8-column group in the down kernel's B-fragment order.
-// down:    y_assign[a] = (W_d h) * sd in fp32; with fuse_combine, the last of the items
-//          writing a 16-row tile forms y = shared + sum_j w_j y_assign there.
+// down:    y_assign[a] = (W_d h) * sd in fp32 (and the shared expert's y_shared); a
+//          separate combine kernel forms y = shared + sum_j w_j y_assign.
 //
 // Programmatic dependent launch: the gate/up kernel runs the shared expert (no routing
 // needed) before griddepcontrol.wait; the down kernel's producer streams weights before
@@ -65,14 +65,21 @@ struct FfnCfg {
     static constexpr int kStageK = KS * kBoxBytes;        // K bytes per stage
     static constexpr int kCodeBytes = kMats * kMatStage;
     static constexpr int kScaleBytes = kNv ? kMats * kConsumerWarps * kScaleBoxSmem : 0;
+    // int4 decode variant: the int8 tensor path (weights as s8 bytes, activations as
+    // three int8 limbs; items of at most 8 tokens, KS = 1)
+    static constexpr bool kLimbs = FMT == MOE_FMT_INT4_ROWSCALE && NNMAX == 1 && KS == 1;
     // decode variant: the producer also copies each stage's slice of the (up to 8) token
-    // rows of the B operand into the stage, one 16-byte-padded row per token
-    static constexpr bool kSmemB = NNMAX == 1 && KS == 1;
+    // rows of the B operand into shared memory, one row per token: fp16 values padded to
+    // 16 bytes, or one 768-byte limb block (the stage's 256 K values, three limbs)
+    // (the int8 path loads its limb B fragments from global memory through L1 instead:
+    // the four warps of a CTA read the same bytes, and shared memory is left to weights)
+    static constexpr bool kSmemB = NNMAX == 1 && KS == 1 && !kLimbs;
     static constexpr int kBRow = 4 * kStageK + 16;
-    static constexpr int kBOff = kCodeBytes + kScaleBytes;
-    static constexpr int kBBytes = kSmemB ? 8 * kBRow : 0;
-    static constexpr int kStageBytes = ((kCodeBytes + kScaleBytes + kBBytes) + 1023) / 1024 * 1024;
-    static constexpr int kStages = GU ? (kSmemB ? 3 : 4) : 5;   // 3 CTAs per SM where it matters
+    static constexpr int kBBytes = kSmemB ? 8 * kBRow : 0;      // per stage, after the ring
+    static constexpr int kStageBytes = ((kCodeBytes + kScaleBytes) + 1023) / 1024 * 1024;
+    // Weights in flight per SM decide the bandwidth (DRAM latency under full load is
+    // about 2.5 us): the int8 path keeps 96 KB of stages per CTA, 2 CTAs per SM.
+    static constexpr int kStages = kLimbs ? (GU ? 6 : 12) : (GU ? (kSmemB ? 3 : 4) : 5);
     static constexpr int kZeroRow = kSmemB ? kBRow : 0;   // zero row read by padding lanes
     static constexpr int kRedFloats = KS > 1 ? kConsumerWarps * kMats * kTokChunk * kRowTile : 0;
 };
@@ -82,18 +89,10 @@ template <int FMT, bool GU, int KS, int NNMAX>
 __host__ __device__ constexpr size_t ffn_smem(int E)
 {
     using C = FfnCfg<FMT, GU, KS, NNMAX>;
-    return 1024 + (size_t)C::kStages * C::kStageBytes + C::kZeroRow + (size_t)C::kRedFloats * 4 +
+    return 1024 + (size_t)C::kStages * (C::kStageBytes + C::kBBytes) + C::kZeroRow + (size_t)C::kRedFloats * 4 +
            (size_t)4 * 4 * (E + 2) + 64 + 8 + (2 * C::kStages + 2) * 8;
 }
 
-// 1-D bulk copy global -> shared completing on an mbarrier (16-byte aligned, size % 16 == 0)
-__device__ __forceinline__ void bulk_copy(void *smem_dst, const void *src, uint32_t bytes, uint64_t *bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_u32(smem_dst)),
-                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
-}
 
 struct SlotTable {
     int *e;      // expert id, -1 = shared expert
@@ -241,6 +240,36 @@ __device__ __forceinline__ const uint16_t *item_brow(const FfnParams &p, const I
               : reinterpret_cast<const uint16_t *>(p.h) + (size_t)(it.boff + bpos) * p.I;
 }
 
+// bytes of one limb row of a K-long operand
+__device__ __forceinline__ size_t limb_row_bytes(int K)
+{
+    return (size_t)((K + kLimbBlockK - 1) / kLimbBlockK) * kLimbBlockBytes;
+}
+
+// int8 path: limb row of bucket column `col` of an item (x limbs for gate/up, h limbs for
+// down); NULL for padding columns or a bad index
+template <bool GU>
+__device__ __forceinline__ const unsigned char *item_brow_limbs(const FfnParams &p, const Item &it, int col)
+{
+    if (col >= it.ntok) return nullptr;
+    const bool sh = it.e < 0;
+    const int bpos = it.tok0 + col;
+    if (GU) {
+        int t = bpos;
+        if (!sh) {
+            const int a = __ldg(p.perm + it.boff + bpos);
+            t = (a >= 0 && a < p.T * p.k) ? a / p.k : -1;
+            if (t < 0) {
+                record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
+                return nullptr;
+            }
+        }
+        return p.x_limbs + (size_t)t * limb_row_bytes(p.H);
+    }
+    return sh ? p.hsh_limbs + (size_t)bpos * limb_row_bytes(p.I_sh)
+              : p.h_limbs + (size_t)(it.boff + bpos) * limb_row_bytes(p.I);
+}
+
 // position of h column n inside its 8-column group, in the order the down kernel's
 // B fragments want it (int4: pairs (0,4)(1,5)(2,6)(3,7); NVFP4: natural order)
 template <int FMT>
@@ -344,6 +373,36 @@ __device__ __forceinline__ void chunk_pair(const unsigned char *st, uint32_t aba
     }
 }
 
+// int8 path, one chunk pair: 64 K values of each of the warp's 16 rows and of each
+// matrix.  The ldmatrix words become s8 bytes 16 x code: even elements feed one mma,
+// odd elements a second one, with the matching limb bytes of the B operand (the 16
+// bytes at 64 q of the limb block: even elements of chunks 2q and 2q+1, then odd ones).  NN = 1:
+// one n-tile whose columns are (limb, token) = (g / 2, g % 2); NN = 3: n-tile = limb,
+// column = token.  Both mma accumulate 16 x sum(code * limb) exactly in s32.
+template <bool GU, int NN>
+__device__ __forceinline__ void chunk_pair_limbs(uint32_t abase, const Lane &L, int q, const uint4 (&Bq)[NN],
+                                                 int (&acc)[GU ? 2 : 1][NN][4])
+{
+    constexpr int M = GU ? 2 : 1;
+    uint32_t ev[M][4], od[M][4];
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        uint32_t r[4];
+        ldmatrix_x4(r[0], r[1], r[2], r[3], abase + m * kMatStage + L.off[q]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) int4_word_to_s8x16(r[i], ev[m][i], od[m][i]);
+    }
+#pragma unroll
+    for (int n = 0; n < NN; ++n) {
+        const uint4 B = Bq[n];
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            mma_s8(acc[m][n], ev[m][0], ev[m][1], ev[m][2], ev[m][3], B.x, B.y);
+            mma_s8(acc[m][n], od[m][0], od[m][1], od[m][2], od[m][3], B.z, B.w);
+        }
+    }
+}
+
 // One warp's share of one work item: the stages of the item (for each stage the B
 // fragments of the warp's K range are fetched before its weights are waited for, since
 // they do not depend on them), then the epilogue.  NN: n-tiles of 8 tokens.  PERM: the
@@ -352,8 +411,8 @@ __device__ __forceinline__ void chunk_pair(const unsigned char *st, uint32_t aba
 // Returns false (every consumer warp alike) when a wait gave up.
 template <int FMT, bool GU, int KS, int NNMAX, int NN, bool PERM>
 __device__ __forceinline__ bool consume_item(const FfnParams &p, const SlotTable tb, const Item it,
-                                          unsigned char *ring, uint64_t *full, uint64_t *empty, int &stage,
-                                          uint32_t &phase, const Lane L, const BRows brow, uint32_t zsm,
+                                          unsigned char *ring, unsigned char *bring, uint64_t *full, uint64_t *empty,
+                                          int &stage, uint32_t &phase, const Lane L, const BRows brow, uint32_t zsm,
                                           float *red, volatile int *cfail, volatile int *abort_flag)
 {
     using C = FfnCfg<FMT, GU, KS, NNMAX>;
@@ -382,7 +441,8 @@ __device__ __forceinline__ bool consume_item(const FfnParams &p, const SlotTable
             if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
             const unsigned char *st = ring + (size_t)stage * C::kStageBytes;
             const uint32_t abase = smem_u32(st + L.bx * kBoxSmem);
-            const uint32_t bsm = (L.g < it.ntok ? smem_u32(st + C::kBOff + L.g * C::kBRow) : zsm) + 16 * L.tq;
+            const uint32_t bsm =
+                (L.g < it.ntok ? smem_u32(bring + (size_t)stage * C::kBBytes + L.g * C::kBRow) : zsm) + 16 * L.tq;
             if (kbox + kBoxBytes <= Kb) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
@@ -480,31 +540,6 @@ __device__ __forceinline__ bool consume_item(const FfnParams &p, const SlotTable
                     }
                 }
             }
-        if (!GU && p.fuse_combine) {
-            // the last of the items writing this warp's 16-row tile combines it
-            const int tile = (it.row0 + L.rw * kRowTile) / kRowTile;
-            __threadfence();
-            __syncwarp();
-            unsigned last = 0;
-            if (L.lane == 0) {
-                int target = 0;
-                for (int s2 = 0; s2 < tb.hdr[0]; ++s2) target += (tb.cnt[s2] + p.tok_chunk - 1) / p.tok_chunk;
-                const unsigned old = atomicInc(p.row_counters + tile, (unsigned)target - 1u);
-                last = (old == (unsigned)target - 1u);
-            }
-            last = __shfl_sync(0xffffffffu, last, 0);
-            if (last) {
-                __threadfence();
-                for (int o = L.lane; o < p.T * kRowTile; o += 32) {
-                    const int t = o / kRowTile, row = tile * kRowTile + o % kRowTile;
-                    float yv = p.n_shared ? __ldcg(p.y_shared + (size_t)t * p.H + row) : 0.f;
-                    for (int j = 0; j < p.k; ++j)
-                        yv = fmaf(__ldg(p.topk_w + (size_t)t * p.k + j),
-                                  __ldcg(p.y_assign + ((size_t)t * p.k + j) * p.H + row), yv);
-                    p.y[(size_t)t * p.H + row] = __half_as_ushort(__float2half_rn(yv));
-                }
-            }
-        }
     } else {
         // ------------------------------------------------ K-split epilogue (KS = 4)
         // partial sums of the four K-slices -> shared memory [warp][mat][col][row]
@@ -549,32 +584,246 @@ __device__ __forceinline__ bool consume_item(const FfnParams &p, const SlotTable
             }
         }
         consumer_sync();
-        if (!GU && p.fuse_combine) {
-            __shared__ int s_last;
-            const int tile = it.row0 / kRowTile;
-            if (tid == 0) {
-                int target = 0;
-                for (int s2 = 0; s2 < tb.hdr[0]; ++s2) target += (tb.cnt[s2] + p.tok_chunk - 1) / p.tok_chunk;
-                __threadfence();
-                const unsigned old = atomicInc(p.row_counters + tile, (unsigned)target - 1u);
-                s_last = (old == (unsigned)target - 1u);
-            }
-            consumer_sync();
-            if (s_last) {
-                __threadfence();
-                for (int o = tid; o < p.T * kRowTile; o += kConsumerWarps * 32) {
-                    const int t = o / kRowTile, row = it.row0 + o % kRowTile;
-                    float yv = p.n_shared ? __ldcg(p.y_shared + (size_t)t * p.H + row) : 0.f;
-                    for (int j = 0; j < p.k; ++j)
-                        yv = fmaf(__ldg(p.topk_w + (size_t)t * p.k + j),
-                                  __ldcg(p.y_assign + ((size_t)t * p.k + j) * p.H + row), yv);
-                    p.y[(size_t)t * p.H + row] = __half_as_ushort(__float2half_rn(yv));
-                }
-            }
-            consumer_sync();
-        }
     }
     (void)RW;
+    return true;
+}
+
+// int8 path, gate/up: the ntok h rows of a finished token chunk (fp16, natural order,
+// K values each) -> int8 limb rows and their scales.  The four consumer warps.
+__device__ __noinline__ void convert_h_rows(const __half *src0, size_t src_stride, unsigned char *dst0, float *scale0, int ntok,
+                               int K)
+{
+    __shared__ float s_red[kConsumerWarps][8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nb = (K + kLimbBlockK - 1) / kLimbBlockK;
+    const size_t row_bytes = (size_t)nb * kLimbBlockBytes;
+    float m[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        m[j] = 0.f;
+        if (j < ntok)
+            for (int k8 = 8 * tid; k8 < K; k8 += 8 * kConsumerWarps * 32)
+                m[j] = fmaxf(m[j], amax8(__ldcg(reinterpret_cast<const uint4 *>(src0 + j * src_stride + k8))));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], off));
+        if (lane == 0) s_red[warp][j] = m[j];
+    }
+    consumer_sync();
+    for (int j = 0; j < ntok; ++j) {
+        float mx = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, s_red[w][j]);
+        const int sh = limb_shift(mx);
+        const float scale = pow2f(sh);
+        const __half *src = src0 + j * src_stride;
+        unsigned char *dst = dst0 + j * row_bytes;
+        for (int k8 = 8 * tid; k8 < nb * kLimbBlockK; k8 += 8 * kConsumerWarps * 32) {
+            const uint4 v = k8 < K ? __ldcg(reinterpret_cast<const uint4 *>(src + k8)) : make_uint4(0u, 0u, 0u, 0u);
+            limb_encode8(v, scale, dst + (size_t)(k8 / kLimbBlockK) * kLimbBlockBytes, k8 % kLimbBlockK);
+        }
+        if (tid == 0) scale0[j] = pow2f(-sh);
+    }
+    consumer_sync();   // s_red is reused by the next conversion
+}
+
+// A completion counter increment whose result is looked at later: gate/up on the int8
+// path counts each finished row tile of a token chunk at the end of an item and settles
+// it after the next item's stages; the CTA that completes the chunk converts its h rows.
+struct Pending {
+    int kind;          // 0 none, 1 h chunk
+    unsigned old, target;
+    int sh, tok0, ntok, boff;
+};
+
+template <bool GU>
+__device__ __forceinline__ void settle(const FfnParams &p, Pending &pd)
+{
+    if (pd.kind == 1) {
+        __shared__ int s_conv;
+        if (threadIdx.x == 0) s_conv = pd.old == pd.target;
+        consumer_sync();
+        if (s_conv) {
+            if (pd.sh)
+                convert_h_rows(p.h_sh + (size_t)pd.tok0 * p.I_sh, p.I_sh, p.hsh_limbs + (size_t)pd.tok0 * limb_row_bytes(p.I_sh),
+                               p.hsh_limb_scale + pd.tok0, pd.ntok, p.I_sh);
+            else
+                convert_h_rows(p.h + (size_t)(pd.boff + pd.tok0) * p.I, p.I,
+                               p.h_limbs + (size_t)(pd.boff + pd.tok0) * limb_row_bytes(p.I),
+                               p.h_limb_scale + pd.boff + pd.tok0, pd.ntok, p.I);
+        }
+    }
+    pd.kind = 0;
+}
+
+// One warp's share of one work item on the int8 path (int4 weights, KS = 1, at most 8
+// tokens): the stages, then the epilogue.  NN = 1 for items of 1-2 tokens, 3 otherwise.
+// The accumulators hold 16 x sum(code * limb) per (limb, token); the epilogue forms
+// sum(code * X) = S0 + 256 S1 + 65536 S2 exactly in 64-bit integers and scales it by
+// 2^-sh and the row scale in fp64.  Gate/up then stores h in fp16 and the last item of
+// a token chunk converts the chunk's h rows to limbs for the down kernel.  Everything
+// the epilogue needs besides the accumulators is loaded before the stages.
+template <bool GU, int NN>
+__device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const SlotTable tb, const Item it,
+                                                   unsigned char *ring, uint64_t *full, uint64_t *empty, int &stage,
+                                                   uint32_t &phase, const Lane L, Pending &pd, volatile int *cfail,
+                                                   volatile int *abort_flag)
+{
+    using C = FfnCfg<MOE_FMT_INT4_ROWSCALE, GU, 1, 1>;
+    constexpr int S = C::kStages;
+    constexpr int M = C::kMats;
+    const bool sh = it.e < 0;
+    const int Kb = it.K / 2;
+    const int nst = (Kb + C::kStageK - 1) / C::kStageK;
+    // this lane's B column in n-tile 0: (limb, token) -> its limb row (NULL: padding)
+    const int lcol = NN == 1 ? (L.g >> 1) : 0;
+    const int tcol = NN == 1 ? (L.g & 1) : L.g;
+    const unsigned char *brow = lcol < 3 ? item_brow_limbs<GU>(p, it, tcol) : nullptr;
+    const uint4 *bsrc = brow ? reinterpret_cast<const uint4 *>(brow + lcol * kLimbBlockK + 16 * L.tq) : nullptr;
+
+    // epilogue operands: row scales of rows g and g + 8, and for the lane's two output
+    // tokens (u = c & 1) the assignment id (routed) and the activation scale
+    const int rows_all = slot_rows<GU>(p, sh);
+    const int ez = sh ? 0 : it.e;
+    const int rowA = it.row0 + L.rw * kRowTile + L.g;
+    const float *sc0 = GU ? (sh ? p.wt.sh_g_scale : p.wt.g_scale) : (sh ? p.wt.sh_d_scale : p.wt.d_scale);
+    const float *sc1 = sh ? p.wt.sh_u_scale : p.wt.u_scale;
+    float rs0[2], rs1[2] = {0.f, 0.f}, xsc[2] = {0.f, 0.f};
+    int asg[2];
+    bool uval[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        rs0[h] = __ldg(sc0 + (size_t)ez * rows_all + rowA + 8 * h);
+        if (GU) rs1[h] = __ldg(sc1 + (size_t)ez * rows_all + rowA + 8 * h);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int t = NN == 1 ? u : 2 * L.tq + u;
+        uval[u] = (NN == 1 ? L.tq == 0 : true) && t < it.ntok;
+        const int bpos = it.tok0 + t;
+        asg[u] = (uval[u] && !sh) ? __ldg(p.perm + it.boff + bpos) : bpos;
+        if (!GU && uval[u]) xsc[u] = __ldcg(sh ? p.hsh_limb_scale + bpos : p.h_limb_scale + it.boff + bpos);
+    }
+
+    int acc[M][NN][4];
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+#pragma unroll
+        for (int n = 0; n < NN; ++n)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[m][n][c] = 0;
+
+    bool ok = true;
+    for (int s = 0; s < nst; ++s) {
+        const int kbox = s * C::kStageK;
+        const int npairs = kbox + kBoxBytes <= Kb ? 4 : (Kb - kbox) / 32;   // K is a multiple of 64
+        // the stage's B fragments (limb block s) are fetched before its weights are waited for
+        uint4 B[4][NN];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int n = 0; n < NN; ++n)
+                B[q][n] = (bsrc && q < npairs) ? __ldg(bsrc + (s * kLimbBlockBytes + n * kLimbBlockK + 64 * q) / 16)
+                                               : make_uint4(0u, 0u, 0u, 0u);
+        if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
+        if (GU && s == 0) {
+            // the activation scales of the lane's tokens (their ids came with the perm loads)
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int a = asg[u];
+                const int tok = sh ? a : ((a >= 0 && a < p.T * p.k) ? a / p.k : -1);
+                if (uval[u] && tok >= 0) xsc[u] = __ldcg(p.x_limb_scale + tok);
+            }
+        }
+        const uint32_t abase = smem_u32(ring + (size_t)stage * C::kStageBytes + L.bx * kBoxSmem);
+        if (npairs == 4) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) chunk_pair_limbs<GU, NN>(abase, L, q, B[q], acc);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (q < npairs) chunk_pair_limbs<GU, NN>(abase, L, q, B[q], acc);
+        }
+        __syncwarp();
+        if (L.lane == 0) mbar_arrive(&empty[stage]);
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+    }
+    if (!ok) {
+        *cfail = 1;
+        *abort_flag = 1;
+    }
+    if (GU) {
+        // the previous item's completion check, now that its atomic has long returned
+        // (its h conversion is a CTA-wide step), then agreement on failure
+        settle<GU>(p, pd);
+        consumer_sync();
+        if (*cfail) return false;
+    } else {
+        // down: the warps own disjoint rows and meet at no barrier; a warp whose wait gave
+        // up leaves, and the others end at their own bounded waits (the producer stops)
+        if (!ok) return false;
+    }
+
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        long long Sv[M];
+        if constexpr (NN == 1) {
+            // lanes tq = 0, 1, 2 of a quad hold limbs 0, 1, 2 of tokens c & 1
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+                const int v0 = acc[m][0][c] >> 4;
+                const int v1 = __shfl_down_sync(0xffffffffu, v0, 1);
+                const int v2 = __shfl_down_sync(0xffffffffu, v0, 2);
+                Sv[m] = (long long)v0 + 256ll * v1 + 65536ll * v2;
+            }
+        } else {
+#pragma unroll
+            for (int m = 0; m < M; ++m)
+                Sv[m] = (long long)(acc[m][0][c] >> 4) + 256ll * (acc[m][1][c] >> 4) + 65536ll * (acc[m][2][c] >> 4);
+        }
+        const int u = c & 1, h = c >> 1;
+        if (!uval[u]) continue;
+        const int row = rowA + 8 * h;
+        const int bpos = it.tok0 + (NN == 1 ? u : 2 * L.tq + u);
+        if (GU) {
+            const double xs = (double)xsc[u];
+            const float gv = (float)((double)Sv[0] * xs * (double)rs0[h]);
+            const float uv = (float)((double)Sv[M - 1] * xs * (double)rs1[h]);
+            const float hv = gv / (1.f + expf(-gv)) * uv;
+            __half *dst = sh ? p.h_sh + (size_t)bpos * p.I_sh : p.h + (size_t)(it.boff + bpos) * p.I;
+            dst[row] = __float2half_rn(hv);
+        } else {
+            const float yv = (float)((double)Sv[0] * (double)xsc[u] * (double)rs0[h]);
+            if (sh) {
+                p.y_shared[(size_t)bpos * p.H + row] = yv;
+            } else {
+                const int a = asg[u];
+                if (a >= 0 && a < p.T * p.k) p.y_assign[(size_t)a * p.H + row] = yv;
+                else record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
+            }
+        }
+    }
+    if (GU) {
+        if (!sh) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int a = asg[u];
+                if (uval[u] && (a < 0 || a >= p.T * p.k)) record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
+            }
+        }
+        // count this row tile of the token chunk; the last one converts the chunk's h rows
+        consumer_sync();
+        pd.kind = 1;
+        pd.sh = sh;
+        pd.tok0 = it.tok0;
+        pd.ntok = it.ntok;
+        pd.boff = it.boff;
+        pd.target = (unsigned)(rows_all / (kRowTile * C::kRW)) - 1u;
+        if (threadIdx.x == 0) {
+            const int idx = sh ? p.T * p.k + it.tok0 : it.boff + it.tok0;
+            pd.old = atom_inc_acq_rel(p.chunk_counters + idx, pd.target);
+        }
+    }
     return true;
 }
 
@@ -588,7 +837,8 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *ring = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char *zrow_sm = ring + (size_t)S * C::kStageBytes;
+    unsigned char *bring = ring + (size_t)S * C::kStageBytes;            // per-stage B rows (decode variant)
+    unsigned char *zrow_sm = bring + (size_t)S * C::kBBytes;
     float *red = reinterpret_cast<float *>(zrow_sm + C::kZeroRow);
     int *tbl = reinterpret_cast<int *>(red + C::kRedFloats);
     const int E = p.E;
@@ -606,6 +856,8 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x;
+    // the combine kernel after the down kernel may start at once: it waits for this grid
+    if constexpr (!GU) pdl_trigger();
     // Only the gate/up kernel runs shared-expert items before the slot table exists (they
     // need no routing).  The down kernel builds its table at once (no wait involved) and
     // its fused combine reads the table, so every one of its items goes through it.
@@ -637,12 +889,17 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
         const uint64_t pol = l2_evict_first_policy();
         int stage = 0;
         uint32_t phase = 0;
-        bool ok = true, have_table = false, pdl_done = GU;
+        // gate/up needs nothing from the router for its shared-expert items, except on the
+        // int8 path, whose x limbs the router writes: their B copies wait like h's do
+        bool ok = true, have_table = false, pdl_done = GU && !C::kLimbs;
         int total = n_pre;
         uint32_t unconfirmed = 0, issued_phase = 0;   // bit s: stage s in flight / its parity
         for (int i = blockIdx.x; ok; i += G) {
             if (i >= n_pre && !have_table) {
-                if (GU) pdl_wait();
+                if (GU) {
+                    pdl_wait();
+                    pdl_done = true;
+                }
                 build_slot_table<GU, RW>(p, tb, E);
                 if (lane == 0) mbar_arrive(table_ready);
                 have_table = true;
@@ -657,23 +914,31 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
                 const int Kb = it.K / 2;
                 const int nst = (Kb + C::kStageK - 1) / C::kStageK;
                 // decode variant: token rows of the B operand, copied stage by stage
-                const uint16_t *brows[8];
+                const unsigned char *brows[8];
                 int nb = 0;
                 if constexpr (C::kSmemB) {
                     const bool perm_b = GU && FMT == MOE_FMT_INT4_ROWSCALE && (i < n_pre || !p.xb_perm);
                     nb = min(it.ntok, 8);
-                    for (int j = 0; j < 8; ++j) brows[j] = j < nb ? item_brow<GU>(p, it, j, perm_b) : nullptr;
+                    for (int j = 0; j < 8; ++j) {
+                        if (C::kLimbs) brows[j] = j < nb ? item_brow_limbs<GU>(p, it, j) : nullptr;
+                        else brows[j] = j < nb ? reinterpret_cast<const unsigned char *>(item_brow<GU>(p, it, j, perm_b)) : nullptr;
+                    }
                 }
+                // bytes of a B row that stage s needs, and where they start
+                auto b_src = [&](int s2) -> size_t { return C::kLimbs ? (size_t)s2 * kLimbBlockBytes : (size_t)4 * s2 * C::kStageK; };
+                auto b_len = [&](int s2) -> uint32_t {
+                    return C::kLimbs ? (uint32_t)kLimbBlockBytes : 4u * (uint32_t)min(C::kStageK, Kb - s2 * C::kStageK);
+                };
                 // The down kernel starts early (programmatic launch) and its B operand, h,
                 // comes from the gate/up kernel: its first stages get their weights at once
                 // and their h rows only after the grid dependency is resolved.
-                const int defer = (!GU && C::kSmemB && !pdl_done) ? min(nst, S) : 0;
+                const int defer = ((!GU || C::kLimbs) && C::kSmemB && !pdl_done) ? min(nst, S) : 0;
                 for (int s = 0; s < nst; ++s) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
                     unconfirmed &= ~(1u << stage);
                     const int kb0 = s * C::kStageK;
                     const int nks = min(KS, (Kb - kb0 + kBoxBytes - 1) / kBoxBytes);
-                    const uint32_t bbytes = 4u * (uint32_t)min(C::kStageK, Kb - kb0);
+                    const uint32_t bbytes = b_len(s);
                     uint32_t tx = (uint32_t)C::kMats * RW * nks * (kBoxSmem + (C::kNv ? kScaleBoxSmem : 0));
                     if constexpr (C::kSmemB) {
                         for (int j = 0; j < nb; ++j) tx += brows[j] ? bbytes : 0u;
@@ -698,20 +963,22 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
                     if constexpr (C::kSmemB) {
                         if (s >= defer) {
                             for (int j = 0; j < nb; ++j)
-                                if (brows[j]) bulk_copy(st + C::kBOff + j * C::kBRow, brows[j] + 2 * kb0, bbytes, &full[stage]);
+                                if (brows[j])
+                                    bulk_copy(bring + (size_t)stage * C::kBBytes + j * C::kBRow, brows[j] + b_src(s), bbytes,
+                                              &full[stage]);
                         }
                         if (defer && s == defer - 1) {
-                            // h is complete once the gate/up grid is: the deferred rows now
+                            // h (x limbs) is complete once the gate/up grid (router) is:
+                            // the deferred rows now
                             pdl_wait();
                             pdl_done = true;
                             int st2 = stage - (defer - 1);
                             if (st2 < 0) st2 += S;
                             for (int s2 = 0; s2 < defer; ++s2) {
-                                const int k2 = s2 * C::kStageK;
-                                const uint32_t b2 = 4u * (uint32_t)min(C::kStageK, Kb - k2);
-                                unsigned char *stg = ring + (size_t)st2 * C::kStageBytes;
                                 for (int j = 0; j < nb; ++j)
-                                    if (brows[j]) bulk_copy(stg + C::kBOff + j * C::kBRow, brows[j] + 2 * k2, b2, &full[st2]);
+                                    if (brows[j])
+                                        bulk_copy(bring + (size_t)st2 * C::kBBytes + j * C::kBRow, brows[j] + b_src(s2),
+                                                  b_len(s2), &full[st2]);
                                 if (++st2 == S) st2 = 0;
                             }
                         }
@@ -755,6 +1022,8 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
     uint32_t phase = 0;
     bool have_table = false;
     int total = n_pre;
+    Pending pend;
+    pend.kind = 0;
 
     // cfail is written only by consumer warps and read only after a consumer barrier,
     // so all four warps take the same exit decision and meet at the same barriers.
@@ -776,6 +1045,16 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
         if (i >= total) break;
         const Item it = (i < n_pre) ? make_item<GU, RW>(p, -1, p.T, 0, i) : decode_item<GU, RW>(p, tb, i);
         const bool sh = it.e < 0;
+        const uint32_t zsm = smem_u32(zrow_sm);
+        if constexpr (C::kLimbs) {
+            // x limbs come from the router, h limbs from the gate/up kernel
+            if (i == blockIdx.x) pdl_wait();
+            const bool ok = it.ntok <= 2
+                                ? consume_item_limbs<GU, 1>(p, tb, it, ring, full, empty, stage, phase, L, pend, cfail, abort_flag)
+                                : consume_item_limbs<GU, 3>(p, tb, it, ring, full, empty, stage, phase, L, pend, cfail, abort_flag);
+            if (!ok) break;
+            continue;
+        } else {
 
         // B-operand rows of this thread's tokens (one per n-tile: column 8n + g); padding
         // columns read a zero row, so no lane needs a select in the inner loop
@@ -802,14 +1081,13 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
             }
         }
         if (!GU && i == blockIdx.x) pdl_wait();   // h is produced by the gate/up kernel
-        const uint32_t zsm = smem_u32(zrow_sm);
 
         const int nN = (it.ntok + 7) >> 3;
         bool ok;
         constexpr bool kPerm = GU && FMT == MOE_FMT_INT4_ROWSCALE;
 #define MOE_CONSUME(NN, PERM)                                                                                   \
-    consume_item<FMT, GU, KS, NNMAX, NN, PERM>(p, tb, it, ring, full, empty, stage, phase, L, brow, zsm, red, cfail, \
-                                               abort_flag)
+    consume_item<FMT, GU, KS, NNMAX, NN, PERM>(p, tb, it, ring, bring, full, empty, stage, phase, L, brow, zsm, red, \
+                                               cfail, abort_flag)
         // NNMAX = 1: items of at most 8 tokens (decode), one n-tile, few registers.
         // NNMAX = 4: items of up to 32 tokens; 2 and 3 n-tiles run the 4-tile code
         // (padding columns read the zero row), which keeps the kernel small.
@@ -822,6 +1100,12 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
         }
 #undef MOE_CONSUME
         if (!ok) break;
+        }
+    }
+    if constexpr (C::kLimbs && GU) {
+        // the last item's completion check (all consumer warps arrive here together, so
+        // the barriers inside line up; a failed CTA has nothing pending to settle safely)
+        if (!*cfail) settle<GU>(p, pend);
     }
 }
 
@@ -863,6 +1147,10 @@ static cudaError_t prepare_t(int E, int *blocks_per_sm)
     cudaError_t e = cudaFuncSetAttribute(ffn_kernel<FMT, GU, KS, NNMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)ffn_smem<FMT, GU, KS, NNMAX>(kMaxExperts));
     if (e != cudaSuccess) return e;
+    // the largest shared-memory carveout, so that the occupancy below is reached and CTAs
+    // of the next kernel can start beside this one's
+    e = cudaFuncSetAttribute(ffn_kernel<FMT, GU, KS, NNMAX>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, ffn_kernel<FMT, GU, KS, NNMAX>, kFfnThreads,
                                                          smem);
 }
@@ -874,9 +1162,15 @@ static cudaError_t prepare_fmt(int E, int occ[2][2][2])
 {
     cudaError_t e;
     if ((e = prepare_t<FMT, true, 1, 1>(E, &occ[0][1][0])) != cudaSuccess) return e;
-    if ((e = prepare_t<FMT, true, 4, 1>(E, &occ[0][1][1])) != cudaSuccess) return e;
     if ((e = prepare_t<FMT, false, 1, 1>(E, &occ[0][0][0])) != cudaSuccess) return e;
-    if ((e = prepare_t<FMT, false, 4, 1>(E, &occ[0][0][1])) != cudaSuccess) return e;
+    if constexpr (FMT == MOE_FMT_INT4_ROWSCALE) {
+        // the int8 path (int4, items of <= 8 tokens) has no K-split variant
+        occ[0][1][1] = occ[0][1][0];
+        occ[0][0][1] = occ[0][0][0];
+    } else {
+        if ((e = prepare_t<FMT, true, 4, 1>(E, &occ[0][1][1])) != cudaSuccess) return e;
+        if ((e = prepare_t<FMT, false, 4, 1>(E, &occ[0][0][1])) != cudaSuccess) return e;
+    }
     if ((e = prepare_t<FMT, true, 1, 4>(E, &occ[1][1][0])) != cudaSuccess) return e;
     if ((e = prepare_t<FMT, true, 4, 4>(E, &occ[1][1][1])) != cudaSuccess) return e;
     if ((e = prepare_t<FMT, false, 1, 4>(E, &occ[1][0][0])) != cudaSuccess) return e;
@@ -893,12 +1187,14 @@ static cudaError_t launch_fmt(const LayerMaps &maps, const FfnParams &p, bool gu
                               cudaStream_t s)
 {
     const bool wide = p.tok_chunk > 8;
-    if (gu) {
-        if (ks == 1) return wide ? launch_t<FMT, true, 1, 4>(maps, p, grid, pdl, s) : launch_t<FMT, true, 1, 1>(maps, p, grid, pdl, s);
-        return wide ? launch_t<FMT, true, 4, 4>(maps, p, grid, pdl, s) : launch_t<FMT, true, 4, 1>(maps, p, grid, pdl, s);
+    if (!wide && (ks == 1 || FMT == MOE_FMT_INT4_ROWSCALE))
+        return gu ? launch_t<FMT, true, 1, 1>(maps, p, grid, pdl, s) : launch_t<FMT, false, 1, 1>(maps, p, grid, pdl, s);
+    if (!wide) {
+        if constexpr (FMT != MOE_FMT_INT4_ROWSCALE)
+            return gu ? launch_t<FMT, true, 4, 1>(maps, p, grid, pdl, s) : launch_t<FMT, false, 4, 1>(maps, p, grid, pdl, s);
     }
-    if (ks == 1) return wide ? launch_t<FMT, false, 1, 4>(maps, p, grid, pdl, s) : launch_t<FMT, false, 1, 1>(maps, p, grid, pdl, s);
-    return wide ? launch_t<FMT, false, 4, 4>(maps, p, grid, pdl, s) : launch_t<FMT, false, 4, 1>(maps, p, grid, pdl, s);
+    if (gu) return ks == 1 ? launch_t<FMT, true, 1, 4>(maps, p, grid, pdl, s) : launch_t<FMT, true, 4, 4>(maps, p, grid, pdl, s);
+    return ks == 1 ? launch_t<FMT, false, 1, 4>(maps, p, grid, pdl, s) : launch_t<FMT, false, 4, 4>(maps, p, grid, pdl, s);
 }
 
 // p.tok_chunk (8 or 32) selects the kernel variant: 8-token items for decode batches,

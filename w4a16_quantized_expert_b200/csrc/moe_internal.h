@@ -15,6 +15,7 @@ namespace moe {
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kRouterTokTile = 16;     // tokens per router CTA
+constexpr int kRouterMaxDynSmem = 160 * 1024;   // router x staging limit
 // scratch of the allocation-free routing entry point: 64 token-tile counters (256 B),
 // then score, selection score and logits for up to kStaticRouteElems (token, expert) pairs
 constexpr int kStaticRouteTiles = 64;
@@ -46,6 +47,8 @@ struct LayerMaps {
 struct RouterParams {
     const uint16_t *x;       // [T][H]
     uint16_t *x_perm;        // optional [T][H]: x with every 8-group in int4 B-fragment order
+    unsigned char *x_limbs;  // optional [T][ceil(H/256)][3][256]: x as int8 limbs (needs do_gemv)
+    float *x_limb_scale;     // [T] 2^-sh of each row of x_limbs
     const float *w;          // [E][H]
     const float *bias;       // [E]
     const float *logits_in;  // optional [T][E]
@@ -62,6 +65,7 @@ struct RouterParams {
     int T, H, E, k;
     float scaling;
     int do_gemv, do_group;
+    int x_rows, x_bufs;      // GEMV: token rows per shared-memory x buffer, buffers (1 or 2)
 };
 
 struct GroupParams {
@@ -92,9 +96,16 @@ struct FfnParams {
     float *y_assign;           // [T*k][H]
     float *y_shared;           // [T][H]
     uint16_t *y;               // [T][H] fp16 (fused combine)
-    unsigned int *row_counters;  // [H/16] (fused combine)
+    // int8 tensor path (int4 weights, items of <= 8 tokens): activations as int8 limbs
+    int limbs;                 // 1: the int4 decode kernels run on the int8 path
+    const unsigned char *x_limbs;   // [T][nblk(H)][3][256]
+    const float *x_limb_scale;      // [T]
+    unsigned char *h_limbs;         // [T*k][nblk(I)][3][256], rows in perm order
+    float *h_limb_scale;            // [T*k]
+    unsigned char *hsh_limbs;       // [T][nblk(I_sh)][3][256]
+    float *hsh_limb_scale;          // [T]
+    unsigned int *chunk_counters;   // [T*k + T] gate/up row tiles finished per token chunk
     int *status;
-    int fuse_combine;
 };
 
 struct CombineParams {

@@ -20,6 +20,7 @@
 #include <cuda_fp16.h>
 #include <math.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "moe_device.cuh"
@@ -27,8 +28,9 @@
 
 namespace moe {
 
-constexpr int kRouterThreads = 128;
-constexpr int kWPerThread = 16;          // float4 of a router row held per thread per pass
+constexpr int kRouterThreads = 256;
+constexpr int kWPerThread = 16;          // float4 of the router row per thread: H <= 16384
+constexpr int kRouterXRows = 4;          // token rows per shared-memory x buffer
 
 __device__ __forceinline__ float sigmoid_ref(float logit)
 {
@@ -46,7 +48,7 @@ __device__ __forceinline__ unsigned float_key(float v)
 // One warp per token: k rounds, each one warp-wide max of the selection keys and one
 // min of the expert indices holding that max (equal scores -> lower expert index).
 __device__ void topk_token(const float *sel_row, const float *score_row, int E, int k,
-                           float scaling, int32_t *idx_out, float *w_out)
+                           float scaling, int32_t *idx_out, float *w_out, int *idx_smem)
 {
     const int lane = threadIdx.x & 31;
     constexpr int kPer = kMaxExperts / 32;
@@ -81,6 +83,7 @@ __device__ void topk_token(const float *sel_row, const float *score_row, int E, 
     double sum = 0.0;
     for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, s_mine, j);
     if (lane < k) {
+        idx_smem[lane] = my_idx;
         idx_out[lane] = my_idx;
         w_out[lane] = static_cast<float>(static_cast<double>(scaling) * (s_mine / sum));
     }
@@ -88,7 +91,7 @@ __device__ void topk_token(const float *sel_row, const float *score_row, int E, 
 
 // ---------------------------------------------------------------------------- grouping
 // Single-warp stable counting sort of the T*k assignment ids by expert.
-__device__ void group_warp(const int32_t *topk_idx, int n, int E, int32_t *counts,
+__device__ void group_warp(const int32_t *topk_idx, bool src_smem, int n, int E, int32_t *counts,
                            int32_t *offsets, int32_t *perm, int32_t *unique, int32_t *n_unique,
                            int *sm_run, int *sm_off, int *status)
 {
@@ -98,7 +101,7 @@ __device__ void group_warp(const int32_t *topk_idx, int n, int E, int32_t *count
     // pass 1: counts
     for (int base = 0; base < n; base += 32) {
         const int a = base + lane;
-        int e = (a < n) ? __ldcg(topk_idx + a) : -1;
+        int e = (a < n) ? (src_smem ? topk_idx[a] : __ldcg(topk_idx + a)) : -1;
         if (a < n && (e < 0 || e >= E)) {
             record_error(status, MOE_ERR_DEVICE_BOUNDS);
             e = -1;
@@ -151,7 +154,7 @@ __device__ void group_warp(const int32_t *topk_idx, int n, int E, int32_t *count
     // pass 2: place every assignment, ascending a inside its expert
     for (int base = 0; base < n; base += 32) {
         const int a = base + lane;
-        int e = (a < n) ? __ldcg(topk_idx + a) : -1;
+        int e = (a < n) ? (src_smem ? topk_idx[a] : __ldcg(topk_idx + a)) : -1;
         if (e >= E) e = -1;
         const unsigned peers = __match_any_sync(0xffffffffu, e);
         if (e >= 0) {
@@ -167,10 +170,15 @@ __device__ void group_warp(const int32_t *topk_idx, int n, int E, int32_t *count
 // ---------------------------------------------------------------------------- kernels
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p)
 {
+    extern __shared__ __align__(16) unsigned char r_smem[];   // x rows: [x_bufs][x_rows][H] fp16
     __shared__ float red[kRouterThreads / 32][kRouterTokTile];
+    __shared__ float red_max[kRouterThreads / 32][kRouterXRows];
+    __shared__ float s_amax[kRouterTokTile];
     __shared__ int s_flag;
     __shared__ int sm_run[kMaxExperts];
     __shared__ int sm_off[kMaxExperts + 1];
+    __shared__ int s_idx[kRouterTokTile * kMaxTopK];
+    __shared__ __align__(8) uint64_t s_bar[2];
 
     pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -180,129 +188,179 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p)
 
     if (p.do_gemv) {
         // ------------------------------------------------ logits of expert e, this tile
+        // The expert's fp32 router row is held in registers; the tile's token rows pass
+        // through shared memory in groups of x_rows (bulk copies, double-buffered).
         const int e = blockIdx.x;
-        const float4 *wrow = reinterpret_cast<const float4 *>(p.w + (size_t)e * p.H);
         const int H4 = p.H >> 2;
-        float acc[kRouterTokTile];
-#pragma unroll
-        for (int t = 0; t < kRouterTokTile; ++t) acc[t] = 0.f;
-        for (int base = 0; base < H4; base += kRouterThreads * kWPerThread) {
-            float4 wv[kWPerThread];
-#pragma unroll
-            for (int j = 0; j < kWPerThread; ++j) {
-                const int h4 = base + j * kRouterThreads + tid;
-                wv[j] = (h4 < H4) ? __ldg(wrow + h4) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int t = 0; t < kRouterTokTile; ++t) {
-                if (t < nt) {
-                    const uint2 *xrow = reinterpret_cast<const uint2 *>(p.x + (size_t)(t0 + t) * p.H);
-                    float a = acc[t];
-#pragma unroll
-                    for (int j = 0; j < kWPerThread; ++j) {
-                        const int h4 = base + j * kRouterThreads + tid;
-                        if (h4 < H4) {
-                            const uint2 xr = __ldg(xrow + h4);
-                            const float2 xa = __half22float2(*reinterpret_cast<const __half2 *>(&xr.x));
-                            const float2 xb = __half22float2(*reinterpret_cast<const __half2 *>(&xr.y));
-                            a = fmaf(wv[j].x, xa.x, a);
-                            a = fmaf(wv[j].y, xa.y, a);
-                            a = fmaf(wv[j].z, xb.x, a);
-                            a = fmaf(wv[j].w, xb.y, a);
-                        }
-                    }
-                    acc[t] = a;
-                }
-            }
-        }
-        if (p.x_perm && e == 0) {
-            // x with every 8-group as (0,4)(1,5)(2,6)(3,7): the B-fragment order of the int4
-            // gate/up kernel, so that its inner loop needs no permutes
-            const int H8 = p.H >> 3;
-            for (int t = 0; t < nt; ++t) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)(t0 + t) * p.H);
-                uint4 *dst = reinterpret_cast<uint4 *>(p.x_perm + (size_t)(t0 + t) * p.H);
-                for (int i = tid; i < H8; i += kRouterThreads) {
-                    const uint4 v = __ldg(src + i);
-                    dst[i] = make_uint4(pack_lo(v.x, v.z), pack_hi(v.x, v.z), pack_lo(v.y, v.w), pack_hi(v.y, v.w));
-                }
-            }
-        }
-        // deterministic block reduction: butterfly inside warps, then warps in order
-#pragma unroll
-        for (int t = 0; t < kRouterTokTile; ++t) {
-            if (t < nt) {
-                float v = acc[t];
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                if (lane == 0) red[warp][t] = v;
-            }
+        const int R = p.x_rows, NB = p.x_bufs;
+        const int ngrp = (nt + R - 1) / R;
+        const uint32_t row_bytes = (uint32_t)p.H * 2u;
+        const uint16_t *xs = reinterpret_cast<const uint16_t *>(r_smem);
+        // CTAs e < ceil(H/256) also write 256-value blocks of x as int8 limbs
+        const int nblk = (p.H + kLimbBlockK - 1) / kLimbBlockK;
+        const bool conv = p.x_limbs != nullptr && e < nblk;
+        if (tid == 0) {
+            mbar_init(&s_bar[0], 1);
+            mbar_init(&s_bar[1], 1);
+            fence_mbar_init();
         }
         __syncthreads();
+        auto issue = [&](int g) {   // thread 0: token rows of group g into buffer g % NB
+            const int bf = g % NB, r0 = g * R, nr = min(R, nt - r0);
+            mbar_arrive_expect_tx(&s_bar[bf], (uint32_t)nr * row_bytes);
+            for (int r = 0; r < nr; ++r)
+                bulk_copy(r_smem + ((size_t)bf * R + r) * row_bytes, p.x + (size_t)(t0 + r0 + r) * p.H, row_bytes,
+                          &s_bar[bf]);
+        };
+        if (tid == 0)
+            for (int g = 0; g < min(NB, ngrp); ++g) issue(g);
+        float4 wv[kWPerThread];
+#pragma unroll
+        for (int j = 0; j < kWPerThread; ++j) {
+            const int h4 = j * kRouterThreads + tid;
+            wv[j] = (h4 < H4) ? __ldg(reinterpret_cast<const float4 *>(p.w + (size_t)e * p.H) + h4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        for (int g = 0; g < ngrp; ++g) {
+            const int bf = g % NB, r0 = g * R, nr = min(R, nt - r0);
+            // a wait that gives up records MOE_ERR_DEVICE_TIMEOUT; the CTA still finishes
+            mbar_wait(&s_bar[bf], (uint32_t)((g / NB) & 1), p.status);
+            float acc[kRouterXRows], amx[kRouterXRows];
+#pragma unroll
+            for (int r = 0; r < kRouterXRows; ++r) {
+                acc[r] = amx[r] = 0.f;
+                if (r < nr) {
+                    const uint16_t *xrow = xs + ((size_t)bf * R + r) * p.H;
+#pragma unroll
+                    for (int j = 0; j < kWPerThread; ++j) {
+                        const int h4 = j * kRouterThreads + tid;
+                        if (h4 < H4) {
+                            const uint2 xr = *reinterpret_cast<const uint2 *>(xrow + 4 * h4);
+                            const float2 xa = __half22float2(*reinterpret_cast<const __half2 *>(&xr.x));
+                            const float2 xb = __half22float2(*reinterpret_cast<const __half2 *>(&xr.y));
+                            acc[r] = fmaf(wv[j].x, xa.x, acc[r]);
+                            acc[r] = fmaf(wv[j].y, xa.y, acc[r]);
+                            acc[r] = fmaf(wv[j].z, xb.x, acc[r]);
+                            acc[r] = fmaf(wv[j].w, xb.y, acc[r]);
+                            if (conv)
+                                amx[r] = fmaxf(amx[r], fmaxf(fmaxf(fabsf(xa.x), fabsf(xa.y)),
+                                                             fmaxf(fabsf(xb.x), fabsf(xb.y))));
+                        }
+                    }
+                }
+            }
+            // deterministic block reduction: butterfly inside warps, then warps in order
+#pragma unroll
+            for (int r = 0; r < kRouterXRows; ++r) {
+                if (r < nr) {
+                    float v = acc[r], m = amx[r];
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) {
+                        v += __shfl_xor_sync(0xffffffffu, v, off);
+                        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+                    }
+                    if (lane == 0) {
+                        red[warp][r0 + r] = v;
+                        red_max[warp][r] = m;
+                    }
+                }
+            }
+            __syncthreads();
+            if (conv) {
+                // the group's rows are in shared memory: their limb blocks b = e (mod gridDim.x)
+                if (tid < nr) {
+                    float m = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kRouterThreads / 32; ++w) m = fmaxf(m, red_max[w][tid]);
+                    s_amax[r0 + tid] = m;
+                }
+                __syncthreads();
+                const size_t lrow = (size_t)nblk * kLimbBlockBytes;
+                for (int b = e; b < nblk; b += gridDim.x)
+                    for (int j = tid; j < nr * 32; j += kRouterThreads) {
+                        const int r = j >> 5, k8 = (j & 31) * 8, k = b * kLimbBlockK + k8;
+                        const uint4 v = k < p.H ? *reinterpret_cast<const uint4 *>(xs + ((size_t)bf * R + r) * p.H + k)
+                                                : make_uint4(0u, 0u, 0u, 0u);
+                        limb_encode8(v, pow2f(limb_shift(s_amax[r0 + r])),
+                                     p.x_limbs + (size_t)(t0 + r0 + r) * lrow + (size_t)b * kLimbBlockBytes, k8);
+                    }
+                if (e == 0 && tid < nr) p.x_limb_scale[t0 + r0 + tid] = pow2f(-limb_shift(s_amax[r0 + tid]));
+                __syncthreads();
+            }
+            if (p.x_perm && e == 0) {
+                // x with every 8-group as (0,4)(1,5)(2,6)(3,7): the B-fragment order of the
+                // int4 expert kernels for larger batches, so their inner loop needs no permutes
+                const int H8 = p.H >> 3;
+                for (int j = tid; j < nr * H8; j += kRouterThreads) {
+                    const int r = j / H8, i = j % H8;
+                    const uint4 v = *reinterpret_cast<const uint4 *>(xs + ((size_t)bf * R + r) * p.H + 8 * i);
+                    reinterpret_cast<uint4 *>(p.x_perm + (size_t)(t0 + r0 + r) * p.H)[i] =
+                        make_uint4(pack_lo(v.x, v.z), pack_hi(v.x, v.z), pack_lo(v.y, v.w), pack_hi(v.y, v.w));
+                }
+                __syncthreads();
+            }
+            if (tid == 0 && g + NB < ngrp) issue(g + NB);   // the buffer is free again
+        }
         if (tid < nt) {
             float v = 0.f;
 #pragma unroll
             for (int w = 0; w < kRouterThreads / 32; ++w) v += red[w][tid];
             const size_t o = (size_t)(t0 + tid) * p.E + e;
-            const float s = sigmoid_ref(v);
+            const float sc = sigmoid_ref(v);
             p.logits[o] = v;
-            p.score[o] = s;
-            p.sel[o] = s + p.bias[e];
+            p.score[o] = sc;
+            p.sel[o] = sc + p.bias[e];
         }
         // the last CTA of this token tile runs its top-k
-        __threadfence();
         __syncthreads();
-        if (tid == 0) {
-            const unsigned old = atomicInc(p.tile_counters + tt, gridDim.x - 1);
-            s_flag = (old == gridDim.x - 1);
-        }
+        if (tid == 0) s_flag = atom_inc_acq_rel(p.tile_counters + tt, gridDim.x - 1) == gridDim.x - 1;
         __syncthreads();
         if (!s_flag) return;
-        __threadfence();
     } else {
         // ------------------------------------------------ scores from given logits
         for (int i = tid; i < nt * p.E; i += kRouterThreads) {
             const size_t o = (size_t)t0 * p.E + i;
             const float l = p.logits_in[o];
-            const float s = sigmoid_ref(l);
+            const float sc = sigmoid_ref(l);
             if (p.logits) p.logits[o] = l;
-            p.score[o] = s;
-            p.sel[o] = s + p.bias[i % p.E];
+            p.score[o] = sc;
+            p.sel[o] = sc + p.bias[i % p.E];
         }
-        __threadfence();
         __syncthreads();
     }
 
     for (int t = warp; t < nt; t += kRouterThreads / 32)
-        topk_token(p.sel + (size_t)(t0 + t) * p.E, p.score + (size_t)(t0 + t) * p.E, p.E, p.k,
-                   p.scaling, p.topk_idx + (size_t)(t0 + t) * p.k, p.topk_w + (size_t)(t0 + t) * p.k);
+        topk_token(p.sel + (size_t)(t0 + t) * p.E, p.score + (size_t)(t0 + t) * p.E, p.E, p.k, p.scaling,
+                   p.topk_idx + (size_t)(t0 + t) * p.k, p.topk_w + (size_t)(t0 + t) * p.k, s_idx + t * p.k);
     if (!p.do_group) return;
-
-    // the last token tile runs the grouping
-    __threadfence();
     __syncthreads();
-    if (tid == 0) {
-        const unsigned old = atomicInc(p.group_counter, gridDim.y - 1);
-        s_flag = (old == gridDim.y - 1);
+    if (gridDim.y == 1) {
+        // one token tile: group straight from this CTA's top-k
+        if (warp == 0)
+            group_warp(s_idx, true, p.T * p.k, p.E, p.counts, p.offsets, p.perm, p.unique, p.n_unique, sm_run, sm_off,
+                       p.status);
+        return;
     }
+    // the last token tile runs the grouping
+    if (tid == 0) s_flag = atom_inc_acq_rel(p.group_counter, gridDim.y - 1) == gridDim.y - 1;
     __syncthreads();
     if (!s_flag) return;
-    __threadfence();
     if (warp == 0)
-        group_warp(p.topk_idx, p.T * p.k, p.E, p.counts, p.offsets, p.perm, p.unique,
-                   p.n_unique, sm_run, sm_off, p.status);
+        group_warp(p.topk_idx, false, p.T * p.k, p.E, p.counts, p.offsets, p.perm, p.unique, p.n_unique, sm_run,
+                   sm_off, p.status);
 }
 
 __global__ void __launch_bounds__(32) group_kernel(GroupParams p)
 {
     __shared__ int sm_run[kMaxExperts];
     __shared__ int sm_off[kMaxExperts + 1];
-    group_warp(p.topk_idx, p.T * p.k, p.E, p.counts, p.offsets, p.perm, p.unique, p.n_unique,
+    group_warp(p.topk_idx, false, p.T * p.k, p.E, p.counts, p.offsets, p.perm, p.unique, p.n_unique,
                sm_run, sm_off, p.status);
 }
 
 __global__ void __launch_bounds__(256) combine_kernel(CombineParams p)
 {
+    pdl_wait();   // y_assign and y_shared come from the down kernel (no-op without PDL)
     const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (size_t)p.T * p.H) return;
     const int t = static_cast<int>(i / p.H), m = static_cast<int>(i % p.H);
@@ -310,6 +368,41 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p)
     for (int j = 0; j < p.k; ++j)
         acc = fmaf(p.topk_w[(size_t)t * p.k + j], p.y_assign[((size_t)t * p.k + j) * p.H + m], acc);
     p.y[i] = __half_as_ushort(__float2half_rn(acc));
+}
+
+// x -> int8 limbs on its own (the staged expert entry point, which runs no router):
+// one CTA per token row
+__global__ void __launch_bounds__(kRouterThreads) x_limbs_kernel(const uint16_t *x, int H, unsigned char *limbs,
+                                                                 float *scale)
+{
+    __shared__ float red_max[kRouterThreads / 32];
+    const int t = blockIdx.x, tid = threadIdx.x;
+    const uint16_t *row = x + (size_t)t * H;
+    float m = 0.f;
+    for (int k8 = 8 * tid; k8 < H; k8 += 8 * kRouterThreads)
+        m = fmaxf(m, amax8(__ldg(reinterpret_cast<const uint4 *>(row + k8))));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((tid & 31) == 0) red_max[tid >> 5] = m;
+    __syncthreads();
+    m = 0.f;
+#pragma unroll
+    for (int w = 0; w < kRouterThreads / 32; ++w) m = fmaxf(m, red_max[w]);
+    const int sh = limb_shift(m);
+    const int nblk = (H + kLimbBlockK - 1) / kLimbBlockK;
+    unsigned char *dst = limbs + (size_t)t * nblk * kLimbBlockBytes;
+    for (int k8 = 8 * tid; k8 < nblk * kLimbBlockK; k8 += 8 * kRouterThreads) {
+        const uint4 v = k8 < H ? __ldg(reinterpret_cast<const uint4 *>(row + k8)) : make_uint4(0u, 0u, 0u, 0u);
+        limb_encode8(v, pow2f(sh), dst + (size_t)(k8 / kLimbBlockK) * kLimbBlockBytes, k8 % kLimbBlockK);
+    }
+    if (tid == 0) scale[t] = pow2f(-sh);
+}
+
+cudaError_t launch_x_limbs(const uint16_t *x, int T, int H, unsigned char *limbs, float *scale, cudaStream_t s)
+{
+    if (T <= 0) return cudaSuccess;
+    x_limbs_kernel<<<T, kRouterThreads, 0, s>>>(x, H, limbs, scale);
+    return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------- static scratch
@@ -337,11 +430,30 @@ cudaError_t static_route_scratch(void **ptr)
 }
 
 // ---------------------------------------------------------------------------- launchers
-cudaError_t launch_router(const RouterParams &p, cudaStream_t s)
+// Shared-memory limits and carveout of the small kernels (once per process and device:
+// the attributes belong to the kernels).  The carveout asks for the largest shared
+// memory split so that the expert kernels' CTAs can start beside the router's.
+cudaError_t router_prepare()
 {
+    cudaError_t e = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRouterMaxDynSmem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(router_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(x_limbs_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    return e;
+}
+
+cudaError_t launch_router(const RouterParams &p0, cudaStream_t s)
+{
+    RouterParams p = p0;
     const int gx = p.do_gemv ? p.E : 1;
     const int gy = (p.T + kRouterTokTile - 1) / kRouterTokTile;
-    router_kernel<<<dim3(gx, gy), kRouterThreads, 0, s>>>(p);
+    size_t smem = 0;
+    if (p.do_gemv) {
+        const size_t row = (size_t)p.H * 2;
+        p.x_rows = std::min(p.T, kRouterXRows);
+        p.x_bufs = (p.T > p.x_rows && 2 * p.x_rows * row <= (size_t)kRouterMaxDynSmem) ? 2 : 1;
+        smem = (size_t)p.x_bufs * p.x_rows * row;
+    }
+    router_kernel<<<dim3(gx, gy), kRouterThreads, smem, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -351,11 +463,19 @@ cudaError_t launch_group(const GroupParams &p, cudaStream_t s)
     return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const CombineParams &p, cudaStream_t s)
+cudaError_t launch_combine(const CombineParams &p, bool pdl, cudaStream_t s)
 {
     const size_t n = (size_t)p.T * p.H;
-    combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((n + 255) / 256));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, combine_kernel, p);
 }
 
 }  // namespace moe
