@@ -33,7 +33,7 @@ size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
 // place (and their zero value) whatever T successive calls use.
 struct Ws {
     size_t ctr_tiles, ctr_group, ctr_chunks, zrow, ctr_end;
-    size_t logits, score, sel, topk_idx, topk_w, counts, offsets, perm, unique, n_unique;
+    size_t logits, score, sel, topk_idx, topk_w, counts, offsets, perm, unique, n_unique, slots;
     size_t x_perm, h, h_sh, y_assign, y_shared, x_stage, y_stage;
     size_t x_limbs, x_limb_scale, h_limbs, h_limb_scale, hsh_limbs, hsh_limb_scale, total;
 };
@@ -67,6 +67,7 @@ Ws ws_layout(const moe_layer_desc &d, int T)
     w.perm = o; o = up256(o + Tk * 4);
     w.unique = o; o = up256(o + (size_t)d.n_experts * 4);
     w.n_unique = o; o = up256(o + 4);
+    w.slots = o; o = up256(o + (size_t)d.n_experts * 16);
     w.x_perm = o; o = up256(o + (size_t)T * d.hidden * 2);
     w.h = o; o = up256(o + Tk * d.inter * 2);
     w.h_sh = o; o = up256(o + (size_t)T * d.inter_shared * 2 * (d.n_shared ? 1 : 0));
@@ -104,13 +105,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 
 // bytes [experts][rows][row_bytes], box {box_inner bytes, 16 rows, 1 expert}
 bool make_map(CUtensorMap *m, const void *base, int row_bytes, int rows, int experts, int box_inner,
-              bool swizzle128)
+              bool swizzle128, int box_rows = kRowTile)
 {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)rows, (cuuint64_t)experts};
     cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)row_bytes * (cuuint64_t)rows};
-    cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)kRowTile, 1};
+    cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -303,6 +304,7 @@ int run_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void 
     rp.perm = at<int32_t>(ws, W.perm);
     rp.unique = at<int32_t>(ws, W.unique);
     rp.n_unique = at<int32_t>(ws, W.n_unique);
+    rp.slots = at<int4>(ws, W.slots);
     rp.do_gemv = 1;
     rp.do_group = 1;
     if (use_limbs(L->desc, T)) {
@@ -325,6 +327,7 @@ int run_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void 
         fp.xb_perm = 1;
     }
     fp.n_unique = rp.n_unique;
+    fp.slots = rp.slots;
     fp.y_assign = at<float>(ws, W.y_assign);
     fp.y_shared = at<float>(ws, W.y_shared);
     fp.y = y;
@@ -391,21 +394,26 @@ int moe_layer_create(const moe_layer_desc *desc, const moe_weights *weights, moe
     const moe_layer_desc &d = *desc;
     const moe_weights &w = *weights;
     const int H = d.hidden, I = d.inter, Is = d.inter_shared, E = d.n_experts;
-    bool ok = make_map(&L->maps.g, w.gate, H / 2, I, E, 128, true) &&
-              make_map(&L->maps.u, w.up, H / 2, I, E, 128, true) &&
-              make_map(&L->maps.d, w.down, I / 2, H, E, 128, true);
-    if (ok && d.n_shared)
-        ok = make_map(&L->maps.sh_g, w.shared_gate, H / 2, Is, 1, 128, true) &&
-             make_map(&L->maps.sh_u, w.shared_up, H / 2, Is, 1, 128, true) &&
-             make_map(&L->maps.sh_d, w.shared_down, Is / 2, H, 1, 128, true);
-    if (ok && d.format == MOE_FMT_NVFP4) {
-        ok = make_map(&L->maps.gb, w.gate_bscale, H / 16, I, E, 16, false) &&
-             make_map(&L->maps.ub, w.up_bscale, H / 16, I, E, 16, false) &&
-             make_map(&L->maps.db, w.down_bscale, I / 16, H, E, 16, false);
+    bool ok = true;
+    LayerMaps &M = L->maps;
+    for (int r4 = 0; r4 < 2 && ok; ++r4) {
+        const int br = r4 ? 4 * kRowTile : kRowTile;
+        ok = make_map(r4 ? &M.g4 : &M.g, w.gate, H / 2, I, E, 128, true, br) &&
+             make_map(r4 ? &M.u4 : &M.u, w.up, H / 2, I, E, 128, true, br) &&
+             make_map(r4 ? &M.d4 : &M.d, w.down, I / 2, H, E, 128, true, br);
         if (ok && d.n_shared)
-            ok = make_map(&L->maps.sh_gb, w.shared_gate_bscale, H / 16, Is, 1, 16, false) &&
-                 make_map(&L->maps.sh_ub, w.shared_up_bscale, H / 16, Is, 1, 16, false) &&
-                 make_map(&L->maps.sh_db, w.shared_down_bscale, Is / 16, H, 1, 16, false);
+            ok = make_map(r4 ? &M.sh_g4 : &M.sh_g, w.shared_gate, H / 2, Is, 1, 128, true, br) &&
+                 make_map(r4 ? &M.sh_u4 : &M.sh_u, w.shared_up, H / 2, Is, 1, 128, true, br) &&
+                 make_map(r4 ? &M.sh_d4 : &M.sh_d, w.shared_down, Is / 2, H, 1, 128, true, br);
+        if (ok && d.format == MOE_FMT_NVFP4) {
+            ok = make_map(r4 ? &M.gb4 : &M.gb, w.gate_bscale, H / 16, I, E, 16, false, br) &&
+                 make_map(r4 ? &M.ub4 : &M.ub, w.up_bscale, H / 16, I, E, 16, false, br) &&
+                 make_map(r4 ? &M.db4 : &M.db, w.down_bscale, I / 16, H, E, 16, false, br);
+            if (ok && d.n_shared)
+                ok = make_map(r4 ? &M.sh_gb4 : &M.sh_gb, w.shared_gate_bscale, H / 16, Is, 1, 16, false, br) &&
+                     make_map(r4 ? &M.sh_ub4 : &M.sh_ub, w.shared_up_bscale, H / 16, Is, 1, 16, false, br) &&
+                     make_map(r4 ? &M.sh_db4 : &M.sh_db, w.shared_down_bscale, Is / 16, H, 1, 16, false, br);
+        }
     }
     if (!ok) {
         delete L;

@@ -71,26 +71,29 @@ struct FfnCfg {
     // decode variant: the producer also copies each stage's slice of the (up to 8) token
     // rows of the B operand into shared memory, one row per token: fp16 values padded to
     // 16 bytes, or one 768-byte limb block (the stage's 256 K values, three limbs)
-    // (the int8 path loads its limb B fragments from global memory through L1 instead:
-    // the four warps of a CTA read the same bytes, and shared memory is left to weights)
-    static constexpr bool kSmemB = NNMAX == 1 && KS == 1 && !kLimbs;
-    static constexpr int kBRow = 4 * kStageK + 16;
-    static constexpr int kBBytes = kSmemB ? 8 * kBRow : 0;      // per stage, after the ring
+    static constexpr bool kSmemB = NNMAX == 1 && KS == 1;
+    static constexpr int kBRow = kLimbs ? kLimbBlockBytes : 4 * kStageK + 16;
+    static constexpr int kBBytes = kSmemB ? 8 * kBRow : 0;      // per stage, after the ring (at most)
     static constexpr int kStageBytes = ((kCodeBytes + kScaleBytes) + 1023) / 1024 * 1024;
-    // Weights in flight per SM decide the bandwidth (DRAM latency under full load is
-    // about 2.5 us): the int8 path keeps 96 KB of stages per CTA, 2 CTAs per SM.
-    static constexpr int kStages = kLimbs ? (GU ? 6 : 12) : (GU ? (kSmemB ? 3 : 4) : 5);
+    // Ring depth.  Weights in flight per SM decide the bandwidth (DRAM latency under full
+    // load is about 2.5 us); the int8 path sizes its ring at launch (up to kStagesMax
+    // stages, as many as fit beside a second CTA on the SM, given the B rows per stage).
+    static constexpr int kStages = GU ? (kSmemB ? 3 : 4) : 5;
+    static constexpr int kStagesCap = kLimbs ? (GU ? 6 : 12) : kStages;
     static constexpr int kZeroRow = kSmemB ? kBRow : 0;   // zero row read by padding lanes
     static constexpr int kRedFloats = KS > 1 ? kConsumerWarps * kMats * kTokChunk * kRowTile : 0;
 };
 
-// dynamic shared memory of one CTA: ring + zero row + reduction + slot table + header/barriers
+constexpr int kStagesMax = 16;   // ring stages any launch may use (mbarrier slots)
+
+// dynamic shared memory of one CTA: ring (weights, then B rows) + zero row + reduction +
+// slot table + header/barriers
 template <int FMT, bool GU, int KS, int NNMAX>
-__host__ __device__ constexpr size_t ffn_smem(int E)
+__host__ __device__ constexpr size_t ffn_smem(int E, int stages, int b_stage)
 {
     using C = FfnCfg<FMT, GU, KS, NNMAX>;
-    return 1024 + (size_t)C::kStages * (C::kStageBytes + C::kBBytes) + C::kZeroRow + (size_t)C::kRedFloats * 4 +
-           (size_t)4 * 4 * (E + 2) + 64 + 8 + (2 * C::kStages + 2) * 8;
+    return 1024 + (size_t)stages * (C::kStageBytes + b_stage) + C::kZeroRow + (size_t)C::kRedFloats * 4 +
+           (size_t)4 * 4 * (E + 2) + 64 + 8 + (2 * kStagesMax + 2) * 8;
 }
 
 
@@ -174,15 +177,25 @@ __device__ void build_slot_table(const FfnParams &p, const SlotTable &tb, int E)
         acc = shared_items<GU, RW>(p);
     }
     const int tiles = slot_rows<GU>(p, false) / (kRowTile * RW);
+    // with the router's slot list, its first 32 entries are read together with its length
+    int4 s0 = make_int4(-1, 0, 0, 0);
+    if (p.slots && lane < E) s0 = __ldcg(p.slots + lane);
     const int n_scan = p.unique ? min(__ldcg(p.n_unique), E) : E;
     for (int b = 0; b < n_scan; b += 32) {
         const int j = b + lane;
         int e = -1, cnt = 0, off = 0;
         if (j < n_scan) {
-            e = p.unique ? __ldcg(p.unique + j) : j;
-            if (e >= 0 && e < E) {
-                off = __ldcg(p.offsets + e);
-                cnt = __ldcg(p.offsets + e + 1) - off;
+            if (p.slots) {
+                const int4 sj = b == 0 ? s0 : __ldcg(p.slots + j);
+                e = sj.x;
+                cnt = sj.y;
+                off = sj.z;
+            } else {
+                e = p.unique ? __ldcg(p.unique + j) : j;
+                if (e >= 0 && e < E) {
+                    off = __ldcg(p.offsets + e);
+                    cnt = __ldcg(p.offsets + e + 1) - off;
+                }
             }
             if (e < 0 || e >= E || off < 0 || cnt < 0 || off + cnt > p.T * p.k) {
                 if (p.unique || cnt != 0) record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
@@ -378,10 +391,11 @@ __device__ __forceinline__ void chunk_pair(const unsigned char *st, uint32_t aba
 // odd elements a second one, with the matching limb bytes of the B operand (the 16
 // bytes at 64 q of the limb block: even elements of chunks 2q and 2q+1, then odd ones).  NN = 1:
 // one n-tile whose columns are (limb, token) = (g / 2, g % 2); NN = 3: n-tile = limb,
-// column = token.  Both mma accumulate 16 x sum(code * limb) exactly in s32.
+// column = token.  The two mma accumulate 16 x sum(code * limb) exactly in s32, in two
+// independent chains (even and odd elements) so that a stage's mma do not serialise.
 template <bool GU, int NN>
 __device__ __forceinline__ void chunk_pair_limbs(uint32_t abase, const Lane &L, int q, const uint4 (&Bq)[NN],
-                                                 int (&acc)[GU ? 2 : 1][NN][4])
+                                                 int (&acc)[2][GU ? 2 : 1][NN][4])
 {
     constexpr int M = GU ? 2 : 1;
     uint32_t ev[M][4], od[M][4];
@@ -397,8 +411,8 @@ __device__ __forceinline__ void chunk_pair_limbs(uint32_t abase, const Lane &L, 
         const uint4 B = Bq[n];
 #pragma unroll
         for (int m = 0; m < M; ++m) {
-            mma_s8(acc[m][n], ev[m][0], ev[m][1], ev[m][2], ev[m][3], B.x, B.y);
-            mma_s8(acc[m][n], od[m][0], od[m][1], od[m][2], od[m][3], B.z, B.w);
+            mma_s8(acc[0][m][n], ev[m][0], ev[m][1], ev[m][2], ev[m][3], B.x, B.y);
+            mma_s8(acc[1][m][n], od[m][0], od[m][1], od[m][2], od[m][3], B.z, B.w);
         }
     }
 }
@@ -416,7 +430,7 @@ __device__ __forceinline__ bool consume_item(const FfnParams &p, const SlotTable
                                           float *red, volatile int *cfail, volatile int *abort_flag)
 {
     using C = FfnCfg<FMT, GU, KS, NNMAX>;
-    constexpr int S = C::kStages;
+    const int S = p.stages;
     constexpr int RW = C::kRW;
     const bool sh = it.e < 0;
     const int Kb = it.K / 2;
@@ -442,7 +456,7 @@ __device__ __forceinline__ bool consume_item(const FfnParams &p, const SlotTable
             const unsigned char *st = ring + (size_t)stage * C::kStageBytes;
             const uint32_t abase = smem_u32(st + L.bx * kBoxSmem);
             const uint32_t bsm =
-                (L.g < it.ntok ? smem_u32(bring + (size_t)stage * C::kBBytes + L.g * C::kBRow) : zsm) + 16 * L.tq;
+                (L.g < it.ntok ? smem_u32(bring + (size_t)stage * p.b_stage + L.g * C::kBRow) : zsm) + 16 * L.tq;
             if (kbox + kBoxBytes <= Kb) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
@@ -665,21 +679,23 @@ __device__ __forceinline__ void settle(const FfnParams &p, Pending &pd)
 // the epilogue needs besides the accumulators is loaded before the stages.
 template <bool GU, int NN>
 __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const SlotTable tb, const Item it,
-                                                   unsigned char *ring, uint64_t *full, uint64_t *empty, int &stage,
-                                                   uint32_t &phase, const Lane L, Pending &pd, volatile int *cfail,
+                                                   unsigned char *ring, unsigned char *bring, uint64_t *full,
+                                                   uint64_t *empty, int &stage, uint32_t &phase, const Lane L,
+                                                   uint32_t zsm, Pending &pd, volatile int *cfail,
                                                    volatile int *abort_flag)
 {
     using C = FfnCfg<MOE_FMT_INT4_ROWSCALE, GU, 1, 1>;
-    constexpr int S = C::kStages;
+    const int S = p.stages;
     constexpr int M = C::kMats;
     const bool sh = it.e < 0;
     const int Kb = it.K / 2;
     const int nst = (Kb + C::kStageK - 1) / C::kStageK;
-    // this lane's B column in n-tile 0: (limb, token) -> its limb row (NULL: padding)
+    // this lane's B column in n-tile 0: (limb, token); its limb block of each stage sits in
+    // the stage's B rows (padding columns read the zero row)
     const int lcol = NN == 1 ? (L.g >> 1) : 0;
     const int tcol = NN == 1 ? (L.g & 1) : L.g;
-    const unsigned char *brow = lcol < 3 ? item_brow_limbs<GU>(p, it, tcol) : nullptr;
-    const uint4 *bsrc = brow ? reinterpret_cast<const uint4 *>(brow + lcol * kLimbBlockK + 16 * L.tq) : nullptr;
+    const bool bval = lcol < 3 && tcol < it.ntok;
+    const uint32_t boff = (uint32_t)(tcol * C::kBRow + lcol * kLimbBlockK + 16 * L.tq);
 
     // epilogue operands: row scales of rows g and g + 8, and for the lane's two output
     // tokens (u = c & 1) the assignment id (routed) and the activation scale
@@ -705,27 +721,27 @@ __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const Slo
         if (!GU && uval[u]) xsc[u] = __ldcg(sh ? p.hsh_limb_scale + bpos : p.h_limb_scale + it.boff + bpos);
     }
 
-    int acc[M][NN][4];
+    int acc2[2][M][NN][4];
 #pragma unroll
-    for (int m = 0; m < M; ++m)
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int n = 0; n < NN; ++n)
+        for (int m = 0; m < M; ++m)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) acc[m][n][c] = 0;
+            for (int n = 0; n < NN; ++n)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc2[h][m][n][c] = 0;
 
     bool ok = true;
     for (int s = 0; s < nst; ++s) {
         const int kbox = s * C::kStageK;
         const int npairs = kbox + kBoxBytes <= Kb ? 4 : (Kb - kbox) / 32;   // K is a multiple of 64
-        // the stage's B fragments (limb block s) are fetched before its weights are waited for
+        if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
+        const uint32_t bb = bval ? smem_u32(bring + (size_t)stage * p.b_stage) + boff : zsm + 16 * L.tq;
         uint4 B[4][NN];
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
-            for (int n = 0; n < NN; ++n)
-                B[q][n] = (bsrc && q < npairs) ? __ldg(bsrc + (s * kLimbBlockBytes + n * kLimbBlockK + 64 * q) / 16)
-                                               : make_uint4(0u, 0u, 0u, 0u);
-        if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
+            for (int n = 0; n < NN; ++n) B[q][n] = lds128(bb + n * kLimbBlockK + 64 * q);
         if (GU && s == 0) {
             // the activation scales of the lane's tokens (their ids came with the perm loads)
 #pragma unroll
@@ -738,11 +754,11 @@ __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const Slo
         const uint32_t abase = smem_u32(ring + (size_t)stage * C::kStageBytes + L.bx * kBoxSmem);
         if (npairs == 4) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) chunk_pair_limbs<GU, NN>(abase, L, q, B[q], acc);
+            for (int q = 0; q < 4; ++q) chunk_pair_limbs<GU, NN>(abase, L, q, B[q], acc2);
         } else {
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                if (q < npairs) chunk_pair_limbs<GU, NN>(abase, L, q, B[q], acc);
+                if (q < npairs) chunk_pair_limbs<GU, NN>(abase, L, q, B[q], acc2);
         }
         __syncwarp();
         if (L.lane == 0) mbar_arrive(&empty[stage]);
@@ -764,6 +780,13 @@ __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const Slo
         if (!ok) return false;
     }
 
+    int acc[M][NN][4];
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+#pragma unroll
+        for (int n = 0; n < NN; ++n)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[m][n][c] = acc2[0][m][n][c] + acc2[1][m][n][c];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         long long Sv[M];
@@ -833,12 +856,12 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
 {
     using C = FfnCfg<FMT, GU, KS, NNMAX>;
     constexpr int RW = C::kRW;
-    constexpr int S = C::kStages;
+    const int S = p.stages;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *ring = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     unsigned char *bring = ring + (size_t)S * C::kStageBytes;            // per-stage B rows (decode variant)
-    unsigned char *zrow_sm = bring + (size_t)S * C::kBBytes;
+    unsigned char *zrow_sm = bring + (size_t)S * p.b_stage;
     float *red = reinterpret_cast<float *>(zrow_sm + C::kZeroRow);
     int *tbl = reinterpret_cast<int *>(red + C::kRedFloats);
     const int E = p.E;
@@ -878,14 +901,16 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
 
     if (warp == kConsumerWarps) {
         // ======================================================== producer warp
-        const CUtensorMap *mA0 = GU ? &maps.g : &maps.d;
-        const CUtensorMap *mA1 = &maps.u;
-        const CUtensorMap *mS0 = GU ? &maps.sh_g : &maps.sh_d;
-        const CUtensorMap *mS1 = &maps.sh_u;
-        const CUtensorMap *bA0 = GU ? &maps.gb : &maps.db;
-        const CUtensorMap *bA1 = &maps.ub;
-        const CUtensorMap *bS0 = GU ? &maps.sh_gb : &maps.sh_db;
-        const CUtensorMap *bS1 = &maps.sh_ub;
+        // whole-K launches (KS = 1) fetch the four warps' 64 rows of a matrix in one box
+        constexpr bool kBox64 = KS == 1;
+        const CUtensorMap *mA0 = kBox64 ? (GU ? &maps.g4 : &maps.d4) : (GU ? &maps.g : &maps.d);
+        const CUtensorMap *mA1 = kBox64 ? &maps.u4 : &maps.u;
+        const CUtensorMap *mS0 = kBox64 ? (GU ? &maps.sh_g4 : &maps.sh_d4) : (GU ? &maps.sh_g : &maps.sh_d);
+        const CUtensorMap *mS1 = kBox64 ? &maps.sh_u4 : &maps.sh_u;
+        const CUtensorMap *bA0 = kBox64 ? (GU ? &maps.gb4 : &maps.db4) : (GU ? &maps.gb : &maps.db);
+        const CUtensorMap *bA1 = kBox64 ? &maps.ub4 : &maps.ub;
+        const CUtensorMap *bS0 = kBox64 ? (GU ? &maps.sh_gb4 : &maps.sh_db4) : (GU ? &maps.sh_gb : &maps.sh_db);
+        const CUtensorMap *bS1 = kBox64 ? &maps.sh_ub4 : &maps.sh_ub;
         const uint64_t pol = l2_evict_first_policy();
         int stage = 0;
         uint32_t phase = 0;
@@ -949,8 +974,9 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
                     for (int m = 0; m < C::kMats; ++m) {
                         const CUtensorMap *map = sh ? (m ? mS1 : mS0) : (m ? mA1 : mA0);
                         const CUtensorMap *bm = sh ? (m ? bS1 : bS0) : (m ? bA1 : bA0);
-                        for (int rw = 0; rw < RW; ++rw)
+                        for (int rw = 0; rw < (kBox64 ? 1 : RW); ++rw)
                             for (int ks = 0; ks < nks; ++ks) {
+                                // (a 64-row box lands as the four 16-row boxes, stacked)
                                 const int bx = rw * KS + ks;
                                 tma_load_3d(st + m * kMatStage + bx * kBoxSmem, map, &full[stage],
                                             kb0 + ks * kBoxBytes, it.row0 + rw * kRowTile, ez, pol);
@@ -964,7 +990,7 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
                         if (s >= defer) {
                             for (int j = 0; j < nb; ++j)
                                 if (brows[j])
-                                    bulk_copy(bring + (size_t)stage * C::kBBytes + j * C::kBRow, brows[j] + b_src(s), bbytes,
+                                    bulk_copy(bring + (size_t)stage * p.b_stage + j * C::kBRow, brows[j] + b_src(s), bbytes,
                                               &full[stage]);
                         }
                         if (defer && s == defer - 1) {
@@ -977,7 +1003,7 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
                             for (int s2 = 0; s2 < defer; ++s2) {
                                 for (int j = 0; j < nb; ++j)
                                     if (brows[j])
-                                        bulk_copy(bring + (size_t)st2 * C::kBBytes + j * C::kBRow, brows[j] + b_src(s2),
+                                        bulk_copy(bring + (size_t)st2 * p.b_stage + j * C::kBRow, brows[j] + b_src(s2),
                                                   b_len(s2), &full[st2]);
                                 if (++st2 == S) st2 = 0;
                             }
@@ -1049,9 +1075,10 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
         if constexpr (C::kLimbs) {
             // x limbs come from the router, h limbs from the gate/up kernel
             if (i == blockIdx.x) pdl_wait();
-            const bool ok = it.ntok <= 2
-                                ? consume_item_limbs<GU, 1>(p, tb, it, ring, full, empty, stage, phase, L, pend, cfail, abort_flag)
-                                : consume_item_limbs<GU, 3>(p, tb, it, ring, full, empty, stage, phase, L, pend, cfail, abort_flag);
+            const bool ok = it.ntok <= 2 ? consume_item_limbs<GU, 1>(p, tb, it, ring, bring, full, empty, stage, phase,
+                                                                     L, zsm, pend, cfail, abort_flag)
+                                         : consume_item_limbs<GU, 3>(p, tb, it, ring, bring, full, empty, stage, phase,
+                                                                     L, zsm, pend, cfail, abort_flag);
             if (!ok) break;
             continue;
         } else {
@@ -1122,13 +1149,36 @@ __global__ void wait_timeout_kernel(int *status, unsigned long long max_iters)
 }
 
 // ---------------------------------------------------------------------------- launchers
+// dynamic shared memory a CTA may use so that two fit on one SM (228 KB, 1 KB reserved
+// and up to 1 KB of static shared memory per CTA)
+constexpr size_t kSmemPerCta2 = 112 * 1024;
+
+// Ring geometry of a launch: the int8 path stages the B rows of min(T, 8) tokens per
+// stage and takes as many stages as fit beside a second CTA (at most its cap).
 template <int FMT, bool GU, int KS, int NNMAX>
-static cudaError_t launch_t(const LayerMaps &maps, const FfnParams &p, int grid, bool pdl, cudaStream_t s)
+static void ffn_geometry(int E, int T, int &stages, int &b_stage)
 {
+    using C = FfnCfg<FMT, GU, KS, NNMAX>;
+    if constexpr (C::kLimbs) {
+        b_stage = (T < 8 ? (T < 1 ? 1 : T) : 8) * C::kBRow;
+        const size_t fixed = ffn_smem<FMT, GU, KS, NNMAX>(E, 0, 0);
+        int n = fixed < kSmemPerCta2 ? (int)((kSmemPerCta2 - fixed) / (C::kStageBytes + b_stage)) : 0;
+        stages = n < 2 ? 2 : (n > C::kStagesCap ? C::kStagesCap : n);
+    } else {
+        stages = C::kStages;
+        b_stage = C::kBBytes;
+    }
+}
+
+template <int FMT, bool GU, int KS, int NNMAX>
+static cudaError_t launch_t(const LayerMaps &maps, const FfnParams &p0, int grid, bool pdl, cudaStream_t s)
+{
+    FfnParams p = p0;
+    ffn_geometry<FMT, GU, KS, NNMAX>(p.E, p.T, p.stages, p.b_stage);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kFfnThreads);
-    cfg.dynamicSmemBytes = ffn_smem<FMT, GU, KS, NNMAX>(p.E);
+    cfg.dynamicSmemBytes = ffn_smem<FMT, GU, KS, NNMAX>(p.E, p.stages, p.b_stage);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1141,11 +1191,24 @@ static cudaError_t launch_t(const LayerMaps &maps, const FfnParams &p, int grid,
 template <int FMT, bool GU, int KS, int NNMAX>
 static cudaError_t prepare_t(int E, int *blocks_per_sm)
 {
-    // the limit is a property of the kernel, shared by every handle: set it for the
-    // largest expert count; the occupancy is that of this handle's launches
-    const size_t smem = ffn_smem<FMT, GU, KS, NNMAX>(E);
-    cudaError_t e = cudaFuncSetAttribute(ffn_kernel<FMT, GU, KS, NNMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)ffn_smem<FMT, GU, KS, NNMAX>(kMaxExperts));
+    // the limit is a property of the kernel, shared by every handle: the device maximum;
+    // the occupancy is that of this handle's largest launch
+    size_t smem = 0;
+    for (int T = 1; T <= 8; ++T) {
+        int st, bs;
+        ffn_geometry<FMT, GU, KS, NNMAX>(E, T, st, bs);
+        const size_t v = ffn_smem<FMT, GU, KS, NNMAX>(E, st, bs);
+        smem = v > smem ? v : smem;
+    }
+    int dev = 0, optin = 0;
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, ffn_kernel<FMT, GU, KS, NNMAX>);
+    if (e != cudaSuccess) return e;
+    if (smem + fa.sharedSizeBytes > (size_t)optin) return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(ffn_kernel<FMT, GU, KS, NNMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             optin - (int)fa.sharedSizeBytes);
     if (e != cudaSuccess) return e;
     // the largest shared-memory carveout, so that the occupancy below is reached and CTAs
     // of the next kernel can start beside this one's

@@ -36,12 +36,16 @@ struct LayerWeights {
     const float *sh_g_scale, *sh_u_scale, *sh_d_scale;
 };
 
-// TMA descriptors over the quantised weights (3-D: K bytes, rows, experts).
+// TMA descriptors over the quantised weights (3-D: K bytes, rows, experts), with boxes of
+// 16 rows (one warp's rows: the K-split launches) and of 64 rows (the four warps' rows of
+// a whole-K launch, one copy per matrix and stage).
 struct LayerMaps {
     CUtensorMap g, u, d;           // routed codes
     CUtensorMap sh_g, sh_u, sh_d;  // shared codes (expert extent 1)
     CUtensorMap gb, ub, db;        // NVFP4 routed block scales
     CUtensorMap sh_gb, sh_ub, sh_db;
+    CUtensorMap g4, u4, d4, sh_g4, sh_u4, sh_d4;          // the same with 64-row boxes
+    CUtensorMap gb4, ub4, db4, sh_gb4, sh_ub4, sh_db4;
 };
 
 struct RouterParams {
@@ -59,6 +63,7 @@ struct RouterParams {
     float *topk_w;           // [T][k]
     // grouping outputs (only when do_group)
     int32_t *counts, *offsets, *perm, *unique, *n_unique;
+    int4 *slots;             // optional [E]: (expert, count, offset, 0) of the non-empty experts
     unsigned int *tile_counters;  // [ceil(T/16)] expert CTAs done per token tile
     unsigned int *group_counter;  // token tiles whose top-k is done
     int *status;
@@ -84,11 +89,13 @@ struct FfnParams {
     const uint16_t *zrow;      // max(H, I, I_sh) zero halves (padding token columns)
     int xb_perm;               // xb holds the permuted copy (else int4 gate/up permutes x)
     int tok_chunk;             // tokens per work item: 8 (decode variant) or 32
+    int stages, b_stage;       // ring stages and B-row bytes per stage of this launch (set by the launcher)
     const int32_t *offsets;    // [E+1]
     const int32_t *perm;       // [T*k]
     const float *topk_w;       // [T][k] (fused combine only)
     const int32_t *unique;     // optional compact list of non-empty experts (router output)
     const int32_t *n_unique;
+    const int4 *slots;         // optional: (expert, count, offset) per entry of that list
     LayerWeights wt;
     // intermediate / outputs
     __half *h;                 // [T*k][I], rows in perm order, columns in mma order
