@@ -32,7 +32,7 @@ size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
 // The counter block sits first and depends only on the handle, so counters keep their
 // place (and their zero value) whatever T successive calls use.
 struct Ws {
-    size_t ctr_tiles, ctr_group, ctr_chunks, zrow, ctr_end;
+    size_t ctr_tiles, ctr_group, ctr_chunks, h_amax, zrow, ctr_end;
     size_t logits, score, sel, topk_idx, topk_w, counts, offsets, perm, unique, n_unique, slots;
     size_t x_perm, h, h_sh, y_assign, y_shared, x_stage, y_stage;
     size_t x_limbs, x_limb_scale, h_limbs, h_limb_scale, hsh_limbs, hsh_limb_scale, total;
@@ -52,6 +52,7 @@ Ws ws_layout(const moe_layer_desc &d, int T)
     w.ctr_tiles = o; o += (size_t)max_tiles * 4;
     w.ctr_group = o; o += 4;
     w.ctr_chunks = o; o += (size_t)d.max_tokens * (d.top_k + 1) * 4;
+    w.h_amax = o; o += (size_t)d.max_tokens * (d.top_k + 1) * 4;
     o = up256(o);
     // a row of zeros read by padding token columns (never written)
     w.zrow = o; o = up256(o + (size_t)std::max(d.hidden, std::max(d.inter, d.inter_shared)) * 2);
@@ -246,6 +247,7 @@ FfnParams ffn_params(const moe_layer *L, const uint16_t *x, int T, void *ws)
         p.hsh_limbs = at<unsigned char>(ws, W.hsh_limbs);
         p.hsh_limb_scale = at<float>(ws, W.hsh_limb_scale);
         p.chunk_counters = at<unsigned int>(ws, W.ctr_chunks);
+        p.h_amax = at<unsigned int>(ws, W.h_amax);
     }
     return p;
 }

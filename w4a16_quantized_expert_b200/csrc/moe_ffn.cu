@@ -604,31 +604,23 @@ __device__ __forceinline__ bool consume_item(const FfnParams &p, const SlotTable
 }
 
 // int8 path, gate/up: the ntok h rows of a finished token chunk (fp16, natural order,
-// K values each) -> int8 limb rows and their scales.  The four consumer warps.
-__device__ __noinline__ void convert_h_rows(const __half *src0, size_t src_stride, unsigned char *dst0, float *scale0, int ntok,
-                               int K)
+// K values each) -> int8 limb rows and their scales.  The rows' largest magnitudes were
+// gathered by the items that wrote them (atomicMax on the float bits, reset here for the
+// next call).  The four consumer warps.
+__device__ __noinline__ void convert_h_rows(const __half *src0, size_t src_stride, unsigned char *dst0, float *scale0,
+                                            unsigned *amax0, int ntok, int K)
 {
-    __shared__ float s_red[kConsumerWarps][8];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nb = (K + kLimbBlockK - 1) / kLimbBlockK;
-    const size_t row_bytes = (size_t)nb * kLimbBlockBytes;
-    float m[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        m[j] = 0.f;
-        if (j < ntok)
-            for (int k8 = 8 * tid; k8 < K; k8 += 8 * kConsumerWarps * 32)
-                m[j] = fmaxf(m[j], amax8(__ldcg(reinterpret_cast<const uint4 *>(src0 + j * src_stride + k8))));
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], off));
-        if (lane == 0) s_red[warp][j] = m[j];
+    __shared__ float s_m[8];
+    const int tid = threadIdx.x;
+    if (tid < ntok) {
+        s_m[tid] = __uint_as_float(__ldcg(amax0 + tid));
+        amax0[tid] = 0u;
     }
     consumer_sync();
+    const int nb = (K + kLimbBlockK - 1) / kLimbBlockK;
+    const size_t row_bytes = (size_t)nb * kLimbBlockBytes;
     for (int j = 0; j < ntok; ++j) {
-        float mx = 0.f;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, s_red[w][j]);
-        const int sh = limb_shift(mx);
+        const int sh = limb_shift(s_m[j]);
         const float scale = pow2f(sh);
         const __half *src = src0 + j * src_stride;
         unsigned char *dst = dst0 + j * row_bytes;
@@ -638,7 +630,7 @@ __device__ __noinline__ void convert_h_rows(const __half *src0, size_t src_strid
         }
         if (tid == 0) scale0[j] = pow2f(-sh);
     }
-    consumer_sync();   // s_red is reused by the next conversion
+    consumer_sync();   // s_m is reused by the next conversion
 }
 
 // A completion counter increment whose result is looked at later: gate/up on the int8
@@ -660,11 +652,11 @@ __device__ __forceinline__ void settle(const FfnParams &p, Pending &pd)
         if (s_conv) {
             if (pd.sh)
                 convert_h_rows(p.h_sh + (size_t)pd.tok0 * p.I_sh, p.I_sh, p.hsh_limbs + (size_t)pd.tok0 * limb_row_bytes(p.I_sh),
-                               p.hsh_limb_scale + pd.tok0, pd.ntok, p.I_sh);
+                               p.hsh_limb_scale + pd.tok0, p.h_amax + p.T * p.k + pd.tok0, pd.ntok, p.I_sh);
             else
                 convert_h_rows(p.h + (size_t)(pd.boff + pd.tok0) * p.I, p.I,
                                p.h_limbs + (size_t)(pd.boff + pd.tok0) * limb_row_bytes(p.I),
-                               p.h_limb_scale + pd.boff + pd.tok0, pd.ntok, p.I);
+                               p.h_limb_scale + pd.boff + pd.tok0, p.h_amax + pd.boff + pd.tok0, pd.ntok, p.I);
         }
     }
     pd.kind = 0;
@@ -787,6 +779,7 @@ __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const Slo
         for (int n = 0; n < NN; ++n)
 #pragma unroll
             for (int c = 0; c < 4; ++c) acc[m][n][c] = acc2[0][m][n][c] + acc2[1][m][n][c];
+    float hmax[2] = {0.f, 0.f};   // gate/up: largest |h| (as stored) of the lane's tokens
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         long long Sv[M];
@@ -814,7 +807,9 @@ __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const Slo
             const float uv = (float)((double)Sv[M - 1] * xs * (double)rs1[h]);
             const float hv = gv / (1.f + expf(-gv)) * uv;
             __half *dst = sh ? p.h_sh + (size_t)bpos * p.I_sh : p.h + (size_t)(it.boff + bpos) * p.I;
-            dst[row] = __float2half_rn(hv);
+            const __half hh = __float2half_rn(hv);
+            dst[row] = hh;
+            hmax[u] = fmaxf(hmax[u], fabsf(__half2float(hh)));
         } else {
             const float yv = (float)((double)Sv[0] * (double)xsc[u] * (double)rs0[h]);
             if (sh) {
@@ -833,6 +828,21 @@ __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const Slo
                 const int a = asg[u];
                 if (uval[u] && (a < 0 || a >= p.T * p.k)) record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
             }
+        }
+        // the h rows' largest magnitudes (per token: lanes of a quad-column, then one atomic)
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            float m = hmax[u];
+            if constexpr (NN == 1) {
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            } else {
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            }
+            const int t = NN == 1 ? u : 2 * L.tq + u;
+            if (L.g == 0 && (NN == 1 ? L.tq == 0 : true) && t < it.ntok)
+                atomicMax(p.h_amax + (sh ? p.T * p.k : it.boff) + it.tok0 + t, __float_as_uint(m));
         }
         // count this row tile of the token chunk; the last one converts the chunk's h rows
         consumer_sync();

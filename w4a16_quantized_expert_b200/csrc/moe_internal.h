@@ -112,6 +112,7 @@ struct FfnParams {
     unsigned char *hsh_limbs;       // [T][nblk(I_sh)][3][256]
     float *hsh_limb_scale;          // [T]
     unsigned int *chunk_counters;   // [T*k + T] gate/up row tiles finished per token chunk
+    unsigned int *h_amax;           // [T*k + T] largest |h| of each h row (float bits; reset after use)
     int *status;
 };
 
