@@ -54,7 +54,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"
 
 # DRAM traffic per launch (bytes) of the dominant kernel from an ncu capture, keyed by
 # workload; valid only while the kernel source hashes to the recorded value.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/ffn_kernel_int4_decode1_e32_full.md: dram read 113,491,712 + write 3,476,992
+    # bytes per gate/up launch (a T=1 step reads the same 9 experts at E=32 as at E=256)
+    "decode1": {"kernel": "gate_up", "bytes": 116968704, "kernel_hash": "b0f251e08e167531"},
+}
 
 
 def describe(w) -> str:
@@ -195,13 +199,21 @@ def barrier(world):
 
 
 def max_over_ranks(world, value: float) -> float:
+    """The largest of the ranks' values (device timings are reported as the max)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tokens_per_s(world: int, steps: int, T: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank runs `steps` steps of T tokens (weak scaling);
+    the job takes the slowest rank's time."""
+    return world * steps * T / (ms_max / 1000.0)
 
 
 # ------------------------------------------------------------------ CPU baseline (oracle)
@@ -411,7 +423,7 @@ def run_ours(args, w):
     clocks.stop()
     ms_max = max_over_ranks(world, ms)
     ms_step = ms_max / K
-    tokens_per_s = world * K * w.T / (ms_max / 1000.0)
+    tokens_per_s = job_tokens_per_s(world, K, w.T, ms_max)
     st = moe.moe_get_device_status(base.handle)
     assert st == moe.MOE_OK, moe.status_string(st)
 
@@ -475,7 +487,7 @@ def run_ours(args, w):
         e1.record(stream)
     e1.synchronize()
     e2e_ms = max_over_ranks(world, e0.elapsed_time(e1))
-    e2e_value = world * K * w.T / (e2e_ms / 1000.0)
+    e2e_value = job_tokens_per_s(world, K, w.T, e2e_ms)
     st = moe.moe_get_device_status(base.handle)
     assert st == moe.MOE_OK, moe.status_string(st)
 
