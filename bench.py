@@ -457,7 +457,8 @@ def run_ours(args, w):
     dom_bytes = ab[names[dom]]
     achieved = dom_bytes / (k_ms[dom] * 1e-3) / 1e9
     tr = NCU_TRAFFIC.get(w.name)
-    traffic = tr["bytes"] if tr and tr.get("kernel_hash") == kernel_hash() else None
+    traffic = (tr["bytes"] if tr and tr.get("kernel") == names[dom] and tr.get("kernel_hash") == kernel_hash()
+               else None)
 
     # ---- end to end through the public API with host buffers
     xh = [torch.from_numpy(x.copy()).pin_memory() for x in xs_host]

@@ -12,7 +12,7 @@
 #include "moe_internal.h"
 
 namespace moe {
-cudaError_t launch_router(const RouterParams &p, cudaStream_t s);
+cudaError_t launch_router(const RouterParams &p, bool pdl, cudaStream_t s);
 cudaError_t router_prepare();
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
 cudaError_t static_route_scratch(void **ptr);
@@ -32,7 +32,7 @@ size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
 // The counter block sits first and depends only on the handle, so counters keep their
 // place (and their zero value) whatever T successive calls use.
 struct Ws {
-    size_t ctr_tiles, ctr_group, ctr_chunks, h_amax, zrow, ctr_end;
+    size_t ctr_tiles, ctr_group, ctr_work, ctr_chunks, h_amax, zrow, ctr_end;
     size_t logits, score, sel, topk_idx, topk_w, counts, offsets, perm, unique, n_unique, slots;
     size_t x_perm, h, h_sh, y_assign, y_shared, x_stage, y_stage;
     size_t x_limbs, x_limb_scale, h_limbs, h_limb_scale, hsh_limbs, hsh_limb_scale, total;
@@ -51,6 +51,7 @@ Ws ws_layout(const moe_layer_desc &d, int T)
     const int max_tiles = (d.max_tokens + kRouterTokTile - 1) / kRouterTokTile;
     w.ctr_tiles = o; o += (size_t)max_tiles * 4;
     w.ctr_group = o; o += 4;
+    w.ctr_work = o; o += 4 * 4;
     w.ctr_chunks = o; o += (size_t)d.max_tokens * (d.top_k + 1) * 4;
     w.h_amax = o; o += (size_t)d.max_tokens * (d.top_k + 1) * 4;
     o = up256(o);
@@ -238,6 +239,7 @@ FfnParams ffn_params(const moe_layer *L, const uint16_t *x, int T, void *ws)
     p.h = at<__half>(ws, W.h);
     p.h_sh = at<__half>(ws, W.h_sh);
     p.status = L->d_status;
+    p.work = at<unsigned int>(ws, W.ctr_work);
     if (use_limbs(L->desc, T)) {
         p.limbs = 1;
         p.x_limbs = at<unsigned char>(ws, W.x_limbs);
@@ -315,7 +317,7 @@ int run_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void 
     } else if (L->desc.format == MOE_FMT_INT4_ROWSCALE) {
         rp.x_perm = at<uint16_t>(ws, W.x_perm);
     }
-    cudaError_t e = launch_router(rp, s);
+    cudaError_t e = launch_router(rp, pdl, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     rec(1);
 
@@ -473,7 +475,7 @@ int moe_route(const moe_layer *L, const uint16_t *x, int T, const float *logits_
     p.topk_w = topk_w;
     p.do_gemv = logits_in ? 0 : 1;
     p.do_group = 0;
-    return cuda_status(launch_router(p, reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_router(p, false, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int moe_route_static(const moe_layer *L, const uint16_t *x, int T, const float *logits_in, float *logits_out,
@@ -507,7 +509,7 @@ int moe_route_static(const moe_layer *L, const uint16_t *x, int T, const float *
     p.scaling = L->desc.routed_scaling;
     p.do_gemv = logits_in ? 0 : 1;
     p.do_group = 0;
-    return cuda_status(launch_router(p, reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_router(p, false, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int moe_group(const moe_layer *L, const int32_t *topk_idx, int T, int32_t *counts, int32_t *offsets,

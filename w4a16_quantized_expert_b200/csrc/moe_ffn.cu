@@ -85,6 +85,7 @@ struct FfnCfg {
 };
 
 constexpr int kStagesMax = 16;   // ring stages any launch may use (mbarrier slots)
+constexpr int kItemQ = 4;        // work items the producer may announce ahead of the consumers
 
 // dynamic shared memory of one CTA: ring (weights, then B rows) + zero row + reduction +
 // slot table + header/barriers
@@ -93,7 +94,7 @@ __host__ __device__ constexpr size_t ffn_smem(int E, int stages, int b_stage)
 {
     using C = FfnCfg<FMT, GU, KS, NNMAX>;
     return 1024 + (size_t)stages * (C::kStageBytes + b_stage) + C::kZeroRow + (size_t)C::kRedFloats * 4 +
-           (size_t)4 * 4 * (E + 2) + 64 + 8 + (2 * kStagesMax + 2) * 8;
+           (size_t)4 * 4 * (E + 2) + 64 + 8 + (2 * kStagesMax + 1 + 2 * kItemQ) * 8;
 }
 
 
@@ -883,18 +884,22 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
     tb.hdr = tbl + 4 * (E + 2);
     volatile int *abort_flag = tb.hdr + 2;
     volatile int *cfail = tb.hdr + 3;
+    volatile int *q_item = tb.hdr + 4;   // [kItemQ] announced work items (-1: no more)
     uint64_t *bars = reinterpret_cast<uint64_t *>(
         (reinterpret_cast<uintptr_t>(tb.hdr + 16) + 7) & ~uintptr_t(7));
-    uint64_t *full = bars, *empty = bars + S, *table_ready = bars + 2 * S;
+    uint64_t *full = bars, *empty = bars + S, *table_ready = bars + 2 * kStagesMax;
+    uint64_t *q_full = table_ready + 1, *q_empty = q_full + kItemQ;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x;
     // the combine kernel after the down kernel may start at once: it waits for this grid
     if constexpr (!GU) pdl_trigger();
     // Only the gate/up kernel runs shared-expert items before the slot table exists (they
-    // need no routing).  The down kernel builds its table at once (no wait involved) and
-    // its fused combine reads the table, so every one of its items goes through it.
+    // need no routing).  The down kernel builds its table at once (no wait involved).
     const int n_pre = GU ? shared_items<GU, RW>(p) : 0;
+    // Work items are claimed from a global counter by each CTA's producer warp (items
+    // differ in cost with their token counts) and announced to the consumer warps through
+    // a small queue; the last CTA to finish resets the counters for the next launch.
 
     for (int i = tid; i < C::kZeroRow / 4; i += kFfnThreads) reinterpret_cast<uint32_t *>(zrow_sm)[i] = 0u;
     if (tid == 0) {
@@ -903,6 +908,10 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
             mbar_init(&empty[s], kConsumerWarps);
         }
         mbar_init(table_ready, 1);
+        for (int q = 0; q < kItemQ; ++q) {
+            mbar_init(&q_full[q], 1);
+            mbar_init(&q_empty[q], kConsumerWarps);
+        }
         tb.hdr[2] = 0;
         tb.hdr[3] = 0;
         fence_mbar_init();
@@ -929,8 +938,11 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
         bool ok = true, have_table = false, pdl_done = GU && !C::kLimbs;
         int total = n_pre;
         uint32_t unconfirmed = 0, issued_phase = 0;   // bit s: stage s in flight / its parity
-        for (int i = blockIdx.x; ok; i += G) {
-            if (i >= n_pre && !have_table) {
+        for (int n_item = 0;; ++n_item) {
+            // claimed only when this CTA can start it (its ring still holds the previous
+            // item's last stages, which cover the atomic's round trip)
+            const int i = (int)__shfl_sync(0xffffffffu, lane == 0 ? atomicAdd(p.work, 1u) : 0u, 0);
+            if (ok && i >= n_pre && !have_table) {
                 if (GU) {
                     pdl_wait();
                     pdl_done = true;
@@ -941,8 +953,16 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
                 total = tb.hdr[1];
                 if (GU) pdl_trigger();
             }
-            if (i >= total) break;
+            const bool done = !ok || i >= total;
             if (lane == 0) {
+                // announce item i (or the end) to the consumers
+                const int q = n_item % kItemQ;
+                if (!mbar_wait(&q_empty[q], (uint32_t)(((n_item / kItemQ) & 1) ^ 1), p.status)) ok = false;
+                q_item[q] = done ? -1 : i;
+                mbar_arrive(&q_full[q]);
+            }
+            if (done) break;
+            if (lane == 0 && ok) {
                 const Item it = (i < n_pre) ? make_item<GU, RW>(p, -1, p.T, 0, i) : decode_item<GU, RW>(p, tb, i);
                 const bool sh = it.e < 0;
                 const int ez = sh ? 0 : it.e;
@@ -1028,7 +1048,7 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (*abort_flag) ok = false;
         }
-        if (!have_table && lane == 0) mbar_arrive(table_ready);  // release the consumers
+        if (!have_table && lane == 0) mbar_arrive(table_ready);  // release the consumers (never waited for)
         if (lane == 0 && !ok) {
             // let copies still in flight land before the CTA may exit
             for (int s = 0; s < S; ++s)
@@ -1063,7 +1083,19 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
 
     // cfail is written only by consumer warps and read only after a consumer barrier,
     // so all four warps take the same exit decision and meet at the same barriers.
-    for (int i = blockIdx.x;; i += G) {
+    for (int n_item = 0;; ++n_item) {
+        const int q = n_item % kItemQ;
+        int i = -1;
+        if (mbar_wait(&q_full[q], (uint32_t)((n_item / kItemQ) & 1), p.status)) {
+            i = q_item[q];
+        } else {
+            *cfail = 1;
+            *abort_flag = 1;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_empty[q]);
+        consumer_sync();
+        if (*cfail || i < 0) break;
         if (i >= n_pre && !have_table) {
             if (!mbar_wait(table_ready, 0, p.status)) {
                 *cfail = 1;
@@ -1078,13 +1110,12 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
                 pdl_trigger();
             }
         }
-        if (i >= total) break;
         const Item it = (i < n_pre) ? make_item<GU, RW>(p, -1, p.T, 0, i) : decode_item<GU, RW>(p, tb, i);
         const bool sh = it.e < 0;
         const uint32_t zsm = smem_u32(zrow_sm);
         if constexpr (C::kLimbs) {
             // x limbs come from the router, h limbs from the gate/up kernel
-            if (i == blockIdx.x) pdl_wait();
+            if (n_item == 0) pdl_wait();
             const bool ok = it.ntok <= 2 ? consume_item_limbs<GU, 1>(p, tb, it, ring, bring, full, empty, stage, phase,
                                                                      L, zsm, pend, cfail, abort_flag)
                                          : consume_item_limbs<GU, 3>(p, tb, it, ring, bring, full, empty, stage, phase,
@@ -1117,7 +1148,7 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
                 }
             }
         }
-        if (!GU && i == blockIdx.x) pdl_wait();   // h is produced by the gate/up kernel
+        if (!GU && n_item == 0) pdl_wait();   // h is produced by the gate/up kernel
 
         const int nN = (it.ntok + 7) >> 3;
         bool ok;
@@ -1143,6 +1174,12 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
         // the last item's completion check (all consumer warps arrive here together, so
         // the barriers inside line up; a failed CTA has nothing pending to settle safely)
         if (!*cfail) settle<GU>(p, pend);
+    }
+    // the last CTA to finish resets the work counters (every producer has made its last
+    // claim before its consumers saw the end of the queue)
+    if (tid == 0 && !*cfail && atomicAdd(p.work + 1, 1u) == (unsigned)G - 1u) {
+        atomicExch(p.work, 0u);
+        atomicExch(p.work + 1, 0u);
     }
 }
 
@@ -1185,6 +1222,7 @@ static cudaError_t launch_t(const LayerMaps &maps, const FfnParams &p0, int grid
 {
     FfnParams p = p0;
     ffn_geometry<FMT, GU, KS, NNMAX>(p.E, p.T, p.stages, p.b_stage);
+    p.work = p0.work + (GU ? 0 : 2);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kFfnThreads);

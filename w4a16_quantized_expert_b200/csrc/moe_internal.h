@@ -90,6 +90,8 @@ struct FfnParams {
     int xb_perm;               // xb holds the permuted copy (else int4 gate/up permutes x)
     int tok_chunk;             // tokens per work item: 8 (decode variant) or 32
     int stages, b_stage;       // ring stages and B-row bytes per stage of this launch (set by the launcher)
+    unsigned int *work;        // work-item claim counter and finished-CTA counter of this launch
+                               // (the caller passes 4: gate/up uses [0..1], down [2..3])
     const int32_t *offsets;    // [E+1]
     const int32_t *perm;       // [T*k]
     const float *topk_w;       // [T][k] (fused combine only)

@@ -276,6 +276,16 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p)
     const int tt = blockIdx.y;
     const int t0 = tt * kRouterTokTile;
     const int nt = min(kRouterTokTile, p.T - t0);
+    if (p.do_gemv) {
+        // When launched behind the previous layer (programmatic dependent launch), the
+        // router row is pulled into L2 while that work drains (L2 stays coherent, so this
+        // is safe whatever the earlier work writes); every load and store of the kernel
+        // comes after the wait.
+        const char *row = reinterpret_cast<const char *>(p.w + (size_t)blockIdx.x * p.H);
+        for (int o = tid * 128; o < p.H * 4; o += kRouterThreads * 128)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(row + o));
+    }
+    pdl_wait();
 
     if (p.do_gemv) {
         // ------------------------------------------------ logits of expert e, this tile
@@ -454,7 +464,8 @@ __global__ void __launch_bounds__(32) group_kernel(GroupParams p)
 
 __global__ void __launch_bounds__(256) combine_kernel(CombineParams p)
 {
-    pdl_wait();   // y_assign and y_shared come from the down kernel (no-op without PDL)
+    pdl_trigger();   // a router launched behind this kernel may start (it waits for it)
+    pdl_wait();      // y_assign and y_shared come from the down kernel (no-op without PDL)
     const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (size_t)p.T * p.H) return;
     const int t = static_cast<int>(i / p.H), m = static_cast<int>(i % p.H);
@@ -535,7 +546,7 @@ cudaError_t router_prepare()
     return e;
 }
 
-cudaError_t launch_router(const RouterParams &p0, cudaStream_t s)
+cudaError_t launch_router(const RouterParams &p0, bool pdl, cudaStream_t s)
 {
     RouterParams p = p0;
     const int gx = p.do_gemv ? p.E : 1;
@@ -547,8 +558,17 @@ cudaError_t launch_router(const RouterParams &p0, cudaStream_t s)
         p.x_bufs = (p.T > p.x_rows && 2 * p.x_rows * row <= (size_t)kRouterMaxDynSmem) ? 2 : 1;
         smem = (size_t)p.x_bufs * p.x_rows * row;
     }
-    router_kernel<<<dim3(gx, gy), kRouterThreads, smem, s>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(gx, gy);
+    cfg.blockDim = dim3(kRouterThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, router_kernel, p);
 }
 
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s)
