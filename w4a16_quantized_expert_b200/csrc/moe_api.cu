@@ -21,6 +21,8 @@ cudaError_t launch_x_limbs(const uint16_t *x, int T, int H, unsigned char *limbs
 cudaError_t launch_ffn(const LayerMaps &maps, const FfnParams &p, bool gate_up, int ks, int grid, bool pdl,
                        cudaStream_t s);
 cudaError_t ffn_prepare(int fmt, int E, int occ[2][2][2]);
+cudaError_t tc_prepare(int E);
+cudaError_t launch_tc(const LayerMaps &maps, const FfnParams &p, bool gate_up, int grid, bool pdl, cudaStream_t s);
 cudaError_t launch_wait_timeout(int *status, unsigned long long max_iters, cudaStream_t s);
 
 namespace {
@@ -41,8 +43,20 @@ struct Ws {
 // bytes of one row of int8 limbs of a K-long operand (blocks of 256 values, 3 limbs)
 size_t limb_row_bytes(int K) { return (size_t)((K + kLimbBlockK - 1) / kLimbBlockK) * kLimbBlockBytes; }
 
-// the int4 expert kernels run on the int8 path for decode-sized batches (8-token items)
-bool use_limbs(const moe_layer_desc &d, int T) { return d.format == MOE_FMT_INT4_ROWSCALE && T <= 16; }
+// Larger int4 batches run the tensor-memory kernel (items of 128 rows and up to 40 tokens),
+// which needs row counts that are multiples of 128.
+bool use_tc(const moe_layer_desc &d, int T)
+{
+    return d.format == MOE_FMT_INT4_ROWSCALE && T > 16 && d.hidden % 128 == 0 && d.inter % 128 == 0 &&
+           (!d.n_shared || d.inter_shared % 128 == 0);
+}
+
+// the int4 expert kernels run on the int8 path (activations as limbs) for decode-sized
+// batches (8-token items) and on the tensor-memory kernel
+bool use_limbs(const moe_layer_desc &d, int T)
+{
+    return d.format == MOE_FMT_INT4_ROWSCALE && (T <= 16 || use_tc(d, T));
+}
 
 Ws ws_layout(const moe_layer_desc &d, int T)
 {
@@ -168,7 +182,7 @@ int validate_weights(const moe_layer_desc *d, const moe_weights *w)
 
 // tokens per expert work item: 8 for decode-sized batches (a one-n-tile kernel with few
 // registers; a bucket of more tokens becomes several items), 32 otherwise
-int tok_chunk(int T) { return T <= 16 ? 8 : kTokChunk; }
+int tok_chunk(int T) { return T <= 16 ? 8 : kTokChunk; }   // (the tensor-memory kernel sets its own)
 
 int check_ws(const moe_layer *L, int T, void *ws, size_t bytes)
 {
@@ -279,6 +293,7 @@ Launch ffn_launch(const moe_layer *L, int T, bool gu)
         const long per_sm = (n + L->num_sms - 1) / L->num_sms;
         return (double)n / (double)(per_sm * L->num_sms);
     };
+    if (use_tc(d, T)) return {1, L->num_sms};                         // one CTA per SM
     if (use_limbs(d, T)) return {1, L->num_sms * L->occ[0][gu][0]};   // the int8 path has KS = 1 only
     const long i1 = items(4), i4 = items(1);
 #ifdef MOE_FORCE_KS
@@ -336,10 +351,11 @@ int run_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void 
     fp.y_shared = at<float>(ws, W.y_shared);
     fp.y = y;
     const Launch lg = ffn_launch(L, T, true), ld = ffn_launch(L, T, false);
-    e = launch_ffn(L->maps, fp, true, lg.ks, lg.grid, pdl, s);
+    const bool tc = use_tc(L->desc, T);
+    e = tc ? launch_tc(L->maps, fp, true, lg.grid, pdl, s) : launch_ffn(L->maps, fp, true, lg.ks, lg.grid, pdl, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     rec(2);
-    e = launch_ffn(L->maps, fp, false, ld.ks, ld.grid, pdl, s);
+    e = tc ? launch_tc(L->maps, fp, false, ld.grid, pdl, s) : launch_ffn(L->maps, fp, false, ld.ks, ld.grid, pdl, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     CombineParams cp = {};
     cp.y_assign = fp.y_assign;
@@ -423,7 +439,8 @@ int moe_layer_create(const moe_layer_desc *desc, const moe_weights *weights, moe
         delete L;
         return MOE_ERR_CUDA;
     }
-    bool occ_ok = router_prepare() == cudaSuccess && ffn_prepare(d.format, d.n_experts, L->occ) == cudaSuccess;
+    bool occ_ok = router_prepare() == cudaSuccess && ffn_prepare(d.format, d.n_experts, L->occ) == cudaSuccess &&
+                  (d.format != MOE_FMT_INT4_ROWSCALE || tc_prepare(d.n_experts) == cudaSuccess);
     for (int a = 0; a < 2; ++a)
         for (int b = 0; b < 2; ++b)
             for (int c = 0; c < 2; ++c) occ_ok = occ_ok && L->occ[a][b][c] >= 1;
@@ -554,9 +571,11 @@ int moe_expert_ffn(const moe_layer *L, const uint16_t *x, int T, const int32_t *
     if (fp.limbs && launch_x_limbs(x, T, L->desc.hidden, const_cast<unsigned char *>(fp.x_limbs),
                                    const_cast<float *>(fp.x_limb_scale), s) != cudaSuccess)
         return MOE_ERR_CUDA;
-    cudaError_t e = launch_ffn(L->maps, fp, true, lg.ks, lg.grid, false, s);
+    const bool tc = use_tc(L->desc, T);
+    cudaError_t e = tc ? launch_tc(L->maps, fp, true, lg.grid, false, s) : launch_ffn(L->maps, fp, true, lg.ks, lg.grid, false, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    return cuda_status(launch_ffn(L->maps, fp, false, ld.ks, ld.grid, true, s));
+    return cuda_status(tc ? launch_tc(L->maps, fp, false, ld.grid, true, s)
+                          : launch_ffn(L->maps, fp, false, ld.ks, ld.grid, true, s));
 }
 
 int moe_combine(const moe_layer *L, const float *y_assign, const float *y_shared, const float *topk_w,

@@ -86,6 +86,7 @@ struct FfnCfg {
 
 constexpr int kStagesMax = 16;   // ring stages any launch may use (mbarrier slots)
 constexpr int kItemQ = 4;        // work items the producer may announce ahead of the consumers
+constexpr int kMaxConvRows = 64; // h rows one conversion handles (tokens of a work item)
 
 // dynamic shared memory of one CTA: ring (weights, then B rows) + zero row + reduction +
 // slot table + header/barriers
@@ -294,10 +295,12 @@ __device__ __forceinline__ int h_pos(int n)
     return (n & ~7) | ((m & 3) << 1) | (m >> 2);
 }
 
-// named barrier of the four consumer warps (the producer warp never joins it)
+// named barrier of the four consumer warps (the producer warp never joins it); NT: the
+// threads that meet there (the tensor-memory kernel's converter warps use it too)
+template <int NT = kConsumerWarps * 32>
 __device__ __forceinline__ void consumer_sync()
 {
-    asm volatile("bar.sync 1, %0;" ::"r"(kConsumerWarps * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"r"(NT) : "memory");
 }
 
 // int4: the fp32 scale of row `row`; NVFP4: the fp32 scale of the whole matrix
@@ -608,16 +611,16 @@ __device__ __forceinline__ bool consume_item(const FfnParams &p, const SlotTable
 // K values each) -> int8 limb rows and their scales.  The rows' largest magnitudes were
 // gathered by the items that wrote them (atomicMax on the float bits, reset here for the
 // next call).  The four consumer warps.
+template <int NT>
 __device__ __noinline__ void convert_h_rows(const __half *src0, size_t src_stride, unsigned char *dst0, float *scale0,
-                                            unsigned *amax0, int ntok, int K)
+                                            unsigned *amax0, int ntok, int K, int ltid)
 {
-    __shared__ float s_m[8];
-    const int tid = threadIdx.x;
-    if (tid < ntok) {
-        s_m[tid] = __uint_as_float(__ldcg(amax0 + tid));
-        amax0[tid] = 0u;
+    __shared__ float s_m[kMaxConvRows];
+    if (ltid < ntok) {
+        s_m[ltid] = __uint_as_float(__ldcg(amax0 + ltid));
+        amax0[ltid] = 0u;
     }
-    consumer_sync();
+    consumer_sync<NT>();
     const int nb = (K + kLimbBlockK - 1) / kLimbBlockK;
     const size_t row_bytes = (size_t)nb * kLimbBlockBytes;
     for (int j = 0; j < ntok; ++j) {
@@ -625,13 +628,13 @@ __device__ __noinline__ void convert_h_rows(const __half *src0, size_t src_strid
         const float scale = pow2f(sh);
         const __half *src = src0 + j * src_stride;
         unsigned char *dst = dst0 + j * row_bytes;
-        for (int k8 = 8 * tid; k8 < nb * kLimbBlockK; k8 += 8 * kConsumerWarps * 32) {
+        for (int k8 = 8 * ltid; k8 < nb * kLimbBlockK; k8 += 8 * NT) {
             const uint4 v = k8 < K ? __ldcg(reinterpret_cast<const uint4 *>(src + k8)) : make_uint4(0u, 0u, 0u, 0u);
             limb_encode8(v, scale, dst + (size_t)(k8 / kLimbBlockK) * kLimbBlockBytes, k8 % kLimbBlockK);
         }
-        if (tid == 0) scale0[j] = pow2f(-sh);
+        if (ltid == 0) scale0[j] = pow2f(-sh);
     }
-    consumer_sync();   // s_m is reused by the next conversion
+    consumer_sync<NT>();   // s_m is reused by the next conversion
 }
 
 // A completion counter increment whose result is looked at later: gate/up on the int8
@@ -643,21 +646,21 @@ struct Pending {
     int sh, tok0, ntok, boff;
 };
 
-template <bool GU>
-__device__ __forceinline__ void settle(const FfnParams &p, Pending &pd)
+template <bool GU, int NT = kConsumerWarps * 32>
+__device__ __forceinline__ void settle(const FfnParams &p, Pending &pd, int ltid)
 {
     if (pd.kind == 1) {
         __shared__ int s_conv;
-        if (threadIdx.x == 0) s_conv = pd.old == pd.target;
-        consumer_sync();
+        if (ltid == 0) s_conv = pd.old == pd.target;
+        consumer_sync<NT>();
         if (s_conv) {
             if (pd.sh)
-                convert_h_rows(p.h_sh + (size_t)pd.tok0 * p.I_sh, p.I_sh, p.hsh_limbs + (size_t)pd.tok0 * limb_row_bytes(p.I_sh),
-                               p.hsh_limb_scale + pd.tok0, p.h_amax + p.T * p.k + pd.tok0, pd.ntok, p.I_sh);
+                convert_h_rows<NT>(p.h_sh + (size_t)pd.tok0 * p.I_sh, p.I_sh, p.hsh_limbs + (size_t)pd.tok0 * limb_row_bytes(p.I_sh),
+                               p.hsh_limb_scale + pd.tok0, p.h_amax + p.T * p.k + pd.tok0, pd.ntok, p.I_sh, ltid);
             else
-                convert_h_rows(p.h + (size_t)(pd.boff + pd.tok0) * p.I, p.I,
+                convert_h_rows<NT>(p.h + (size_t)(pd.boff + pd.tok0) * p.I, p.I,
                                p.h_limbs + (size_t)(pd.boff + pd.tok0) * limb_row_bytes(p.I),
-                               p.h_limb_scale + pd.boff + pd.tok0, p.h_amax + pd.boff + pd.tok0, pd.ntok, p.I);
+                               p.h_limb_scale + pd.boff + pd.tok0, p.h_amax + pd.boff + pd.tok0, pd.ntok, p.I, ltid);
         }
     }
     pd.kind = 0;
@@ -764,7 +767,7 @@ __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const Slo
     if (GU) {
         // the previous item's completion check, now that its atomic has long returned
         // (its h conversion is a CTA-wide step), then agreement on failure
-        settle<GU>(p, pd);
+        settle<GU>(p, pd, threadIdx.x);
         consumer_sync();
         if (*cfail) return false;
     } else {
@@ -1173,13 +1176,496 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
     if constexpr (C::kLimbs && GU) {
         // the last item's completion check (all consumer warps arrive here together, so
         // the barriers inside line up; a failed CTA has nothing pending to settle safely)
-        if (!*cfail) settle<GU>(p, pend);
+        if (!*cfail) settle<GU>(p, pend, threadIdx.x);
     }
     // the last CTA to finish resets the work counters (every producer has made its last
     // claim before its consumers saw the end of the queue)
     if (tid == 0 && !*cfail && atomicAdd(p.work + 1, 1u) == (unsigned)G - 1u) {
         atomicExch(p.work, 0u);
         atomicExch(p.work + 1, 0u);
+    }
+}
+
+// ============================================================================ tcgen05 path
+// Expert GEMMs of larger batches (int4, T > 16): each work item is (expert, 128 output
+// rows, up to kTcTok tokens).  Arithmetic as on the decode path: weights as s8 bytes
+// 16 x code, activations as three exact int8 limbs, exact integer accumulation; here the
+// product runs on the 5th-generation tensor cores (tcgen05.mma kind::i8, M = 128,
+// N = 3 x tokens rounded up to 16, K = 32 per instruction, s32 accumulators in TMEM).
+//
+// Warps: 0 streams the packed codes with TMA into a ring of 256-K stages; 1 allocates
+// TMEM and issues the MMAs (one thread); 2..5 expand each 128-K half of a stage into the
+// 128-byte-swizzled K-major int8 layout the MMA reads (weights from the packed stage, the
+// tokens' limb rows from global memory), then, once an item's accumulators are complete,
+// read them from TMEM (warp w owns TMEM lanes 32 (w % 4) .., the two warps of a lane quarter
+// split the tokens) and run the epilogue.
+// Accumulators are double-buffered in TMEM, so the next item's MMAs overlap an epilogue.
+
+constexpr int kTcRows = 128;                    // output rows per item (MMA M)
+constexpr int kTcTok = 40;                      // tokens per item
+constexpr int kTcNMax = 128;                    // 3 x 40 rounded up to 16
+constexpr int kTcPack = 3;                      // packed stages (256 K each)
+constexpr int kTcSub = 2;                       // expanded sub-stages (128 K each)
+constexpr int kTcConv = 8;                      // converter / epilogue warps (two per TMEM lane quarter)
+constexpr int kTcConvT = kTcConv * 32;
+constexpr int kTcThreads = (2 + kTcConv) * 32;
+
+template <bool GU>
+struct TcCfg {
+    static constexpr int kMats = GU ? 2 : 1;
+    static constexpr int kPackBytes = kMats * kTcRows * kBoxBytes;   // one 256-K stage of codes
+    static constexpr int kABytes = kTcRows * 128;                    // one matrix, one 128-K sub-stage, s8
+    static constexpr int kBBytes = kTcNMax * 128;                    // limb rows of one sub-stage
+    static constexpr int kSubBytes = kMats * kABytes + kBBytes;
+    static constexpr int kAccCols = kMats * kTcNMax;                 // TMEM columns of one accumulator set
+    static constexpr int kTmemCols = 2 * kAccCols;                   // double-buffered (power of two)
+};
+
+template <bool GU>
+__host__ __device__ constexpr size_t tc_smem(int E)
+{
+    using C = TcCfg<GU>;
+    return 1024 + (size_t)kTcPack * C::kPackBytes + (size_t)kTcSub * C::kSubBytes + (size_t)4 * 4 * (E + 2) + 64 +
+           kTcTok * 16 + 8 + 8 + (2 * kTcPack + 2 * kTcSub + 4 + 2 * kItemQ + 1) * 8;
+}
+
+// UMMA shared-memory descriptor of a K-major tile of 8-row x 128-byte swizzle atoms
+__device__ __forceinline__ uint64_t umma_sdesc(uint32_t saddr)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// UMMA instruction descriptor: s8 x s8 -> s32, both K-major, M = 128
+__device__ __forceinline__ uint32_t umma_idesc_s8(int n)
+{
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kTcRows >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_s8(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+                 "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&v)[8])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                 : "r"(taddr));
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+template <bool GU>
+__global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_constant__ LayerMaps maps, const FfnParams p)
+{
+    using C = TcCfg<GU>;
+    constexpr int RW = kTcRows / kRowTile;   // 8: items of 128 rows
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *pack = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char *subs = pack + (size_t)kTcPack * C::kPackBytes;            // 1024-aligned (all sizes are)
+    int *tbl = reinterpret_cast<int *>(subs + (size_t)kTcSub * C::kSubBytes);
+    const int E = p.E;
+    SlotTable tb;
+    tb.e = tbl;
+    tb.cnt = tbl + (E + 2);
+    tb.off = tbl + 2 * (E + 2);
+    tb.base = tbl + 3 * (E + 2);
+    tb.hdr = tbl + 4 * (E + 2);
+    volatile int *abort_flag = tb.hdr + 2;
+    volatile int *cfail = tb.hdr + 3;
+    volatile int *q_item = tb.hdr + 4;
+    const unsigned char **s_brow = reinterpret_cast<const unsigned char **>(tb.hdr + 16);   // [kTcTok] limb rows
+    float *s_sc = reinterpret_cast<float *>(s_brow + kTcTok);   // [kTcTok] activation scale of each token
+    int *s_id = reinterpret_cast<int *>(s_sc + kTcTok);         // [kTcTok] token (gate/up) or assignment (down)
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(s_id + kTcTok);
+    uint64_t *bars = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(s_tmem + 2) + 7) & ~uintptr_t(7));
+    uint64_t *pk_full = bars, *pk_empty = pk_full + kTcPack;
+    uint64_t *sb_full = pk_empty + kTcPack, *sb_empty = sb_full + kTcSub;
+    uint64_t *acc_full = sb_empty + kTcSub, *acc_empty = acc_full + 2;
+    uint64_t *q_full = acc_empty + 2, *q_empty = q_full + kItemQ;
+    uint64_t *table_ready = q_empty + kItemQ;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = gridDim.x;
+    if constexpr (!GU) pdl_trigger();   // the combine kernel may start at once: it waits for this grid
+    const int n_pre = GU ? shared_items<GU, RW>(p) : 0;
+
+    if (tid == 0) {
+        for (int s = 0; s < kTcPack; ++s) {
+            mbar_init(&pk_full[s], 1);
+            mbar_init(&pk_empty[s], kTcConv);
+        }
+        for (int s = 0; s < kTcSub; ++s) {
+            mbar_init(&sb_full[s], kTcConv);
+            mbar_init(&sb_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&acc_full[s], 1);
+            mbar_init(&acc_empty[s], kTcConv);
+        }
+        for (int q = 0; q < kItemQ; ++q) {
+            mbar_init(&q_full[q], 1);
+            mbar_init(&q_empty[q], 1 + kTcConv);
+        }
+        mbar_init(table_ready, 1);
+        tb.hdr[2] = 0;
+        tb.hdr[3] = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
+                     "r"(C::kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+
+    if (warp == 0) {
+        // ======================================================== producer: packed codes
+        const CUtensorMap *mA0 = GU ? &maps.g4 : &maps.d4, *mA1 = &maps.u4;
+        const CUtensorMap *mS0 = GU ? &maps.sh_g4 : &maps.sh_d4, *mS1 = &maps.sh_u4;
+        const uint64_t pol = l2_evict_first_policy();
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true, have_table = false;
+        int total = n_pre;
+        uint32_t unconfirmed = 0, issued_phase = 0;
+        for (int n_item = 0;; ++n_item) {
+            const int i = (int)__shfl_sync(0xffffffffu, lane == 0 ? atomicAdd(p.work, 1u) : 0u, 0);
+            if (ok && i >= n_pre && !have_table) {
+                if (GU) pdl_wait();   // routing is complete (the down kernel's table sources are older)
+                build_slot_table<GU, RW>(p, tb, E);
+                if (lane == 0) mbar_arrive(table_ready);
+                have_table = true;
+                total = tb.hdr[1];
+                if (GU) pdl_trigger();
+            }
+            const bool done = !ok || i >= total;
+            if (lane == 0) {
+                const int q = n_item % kItemQ;
+                if (!mbar_wait(&q_empty[q], (uint32_t)(((n_item / kItemQ) & 1) ^ 1), p.status)) ok = false;
+                q_item[q] = done ? -1 : i;
+                mbar_arrive(&q_full[q]);
+            }
+            if (done) break;
+            if (lane == 0 && ok) {
+                const Item it = (i < n_pre) ? make_item<GU, RW>(p, -1, p.T, 0, i) : decode_item<GU, RW>(p, tb, i);
+                const bool sh = it.e < 0;
+                const int ez = sh ? 0 : it.e;
+                const int nst = (it.K / 2 + kBoxBytes - 1) / kBoxBytes;
+                for (int s = 0; s < nst; ++s) {
+                    if (!mbar_wait(&pk_empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
+                    unconfirmed &= ~(1u << stage);
+                    mbar_arrive_expect_tx(&pk_full[stage], (uint32_t)C::kPackBytes);
+                    unsigned char *st = pack + (size_t)stage * C::kPackBytes;
+#pragma unroll
+                    for (int m = 0; m < C::kMats; ++m) {
+                        const CUtensorMap *map = sh ? (m ? mS1 : mS0) : (m ? mA1 : mA0);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)   // two 64-row boxes
+                            tma_load_3d(st + (m * kTcRows + 64 * h) * kBoxBytes, map, &pk_full[stage], s * kBoxBytes,
+                                        it.row0 + 64 * h, ez, pol);
+                    }
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    unconfirmed |= 1u << stage;
+                    if (++stage == kTcPack) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) *abort_flag = 1;
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (*abort_flag) ok = false;
+        }
+        if (!have_table && lane == 0) mbar_arrive(table_ready);
+        if (lane == 0 && !ok)
+            for (int s = 0; s < kTcPack; ++s)
+                if (unconfirmed >> s & 1u) mbar_wait(&pk_full[s], issued_phase >> s & 1u, p.status, 10000000ull);
+    } else if (warp == 1) {
+        // ======================================================== MMA issuer
+        int sub = 0;
+        uint32_t sphase = 0;
+        bool ok = true, have_table = false;
+        for (int n_item = 0; ok; ++n_item) {
+            const int q = n_item % kItemQ;
+            int i = -1;
+            if (mbar_wait(&q_full[q], (uint32_t)((n_item / kItemQ) & 1), p.status)) i = q_item[q];
+            else ok = false;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_empty[q]);
+            if (i < 0) break;
+            if (i >= n_pre && !have_table) {
+                if (!mbar_wait(table_ready, 0, p.status)) { ok = false; break; }
+                have_table = true;
+            }
+            const Item it = (i < n_pre) ? make_item<GU, RW>(p, -1, p.T, 0, i) : decode_item<GU, RW>(p, tb, i);
+            const int n = ((3 * it.ntok + 15) / 16) * 16;
+            const uint32_t idesc = umma_idesc_s8(n);
+            const int buf = n_item & 1;
+            // the epilogue of the item two back has released this accumulator set
+            if (!mbar_wait(&acc_empty[buf], (uint32_t)(((n_item >> 1) & 1) ^ 1), p.status)) { ok = false; break; }
+            tc_fence_after();
+            const int nsub = (it.K + 127) / 128;   // 128-K halves of the packed stages
+            for (int u = 0; u < nsub; ++u) {
+                if (!mbar_wait(&sb_full[sub], sphase, p.status)) { ok = false; break; }
+                tc_fence_after();
+                const int kvals = min(128, it.K - 128 * u);   // a multiple of 64
+                if (lane == 0) {
+                    const uint32_t sbase = smem_u32(subs + (size_t)sub * C::kSubBytes);
+                    for (int kk = 0; kk < kvals / 32; ++kk) {
+                        const uint64_t db = umma_sdesc(sbase + C::kMats * C::kABytes + 32 * kk);
+#pragma unroll
+                        for (int m = 0; m < C::kMats; ++m)
+                            umma_s8(tmem + buf * C::kAccCols + m * kTcNMax, umma_sdesc(sbase + m * C::kABytes + 32 * kk),
+                                    db, idesc, (u > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&sb_empty[sub]);   // the sub-stage is free once these MMAs have read it
+                    if (u == nsub - 1) umma_commit(&acc_full[buf]);
+                }
+                __syncwarp();
+                if (++sub == kTcSub) { sub = 0; sphase ^= 1u; }
+            }
+        }
+        if (!ok) *abort_flag = 1;
+    } else {
+        // ======================================================== converters + epilogue
+        const int ltid = tid - 64;             // 0 .. kTcConvT - 1
+        const int quarter = warp & 3;          // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;      // which of the quarter's two warps: token blocks
+        const int row_l = 32 * quarter + lane; // the output row (TMEM lane) of this thread
+        int pstage = 0, sub = 0;
+        uint32_t pphase = 0, sphase = 0;
+        bool have_table = false;
+        Pending pend;
+        pend.kind = 0;
+        for (int n_item = 0;; ++n_item) {
+            const int q = n_item % kItemQ;
+            int i = -1;
+            if (mbar_wait(&q_full[q], (uint32_t)((n_item / kItemQ) & 1), p.status)) {
+                i = q_item[q];
+            } else {
+                *cfail = 1;
+                *abort_flag = 1;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_empty[q]);
+            consumer_sync<kTcConvT>();
+            if (*cfail || i < 0) break;
+            if (i >= n_pre && !have_table) {
+                if (!mbar_wait(table_ready, 0, p.status)) {
+                    *cfail = 1;
+                    *abort_flag = 1;
+                }
+                consumer_sync<kTcConvT>();
+                if (*cfail) break;
+                have_table = true;
+            }
+            if (n_item == 0) pdl_wait();   // limb rows come from the router / the gate/up kernel
+            const Item it = (i < n_pre) ? make_item<GU, RW>(p, -1, p.T, 0, i) : decode_item<GU, RW>(p, tb, i);
+            const bool sh = it.e < 0;
+            const int nrow = 3 * it.ntok;
+            // the item's tokens: limb rows, activation scales, ids (all loads in parallel)
+            if (ltid < it.ntok) {
+                const int bpos = it.tok0 + ltid;
+                s_brow[ltid] = item_brow_limbs<GU>(p, it, ltid);
+                int id = bpos;     // shared expert: the token itself
+                if (!sh) {
+                    const int aid = __ldg(p.perm + it.boff + bpos);
+                    id = (aid >= 0 && aid < p.T * p.k) ? (GU ? aid / p.k : aid) : -1;
+                }
+                s_id[ltid] = id;
+                s_sc[ltid] = GU ? (id >= 0 ? __ldcg(p.x_limb_scale + id) : 0.f)
+                                : __ldcg(sh ? p.hsh_limb_scale + bpos : p.h_limb_scale + it.boff + bpos);
+            }
+            consumer_sync<kTcConvT>();
+            const int nst = (it.K / 2 + kBoxBytes - 1) / kBoxBytes;
+            const int n = ((nrow + 15) / 16) * 16;   // MMA N
+            // this thread's 16-byte pieces of the B rows of one sub-stage (<= 8), loaded
+            // one sub-stage ahead of their use
+            constexpr int kBPer = kTcNMax * 8 / kTcConvT;
+            uint4 bv[kBPer];
+            auto bload = [&](int s2, int u2) {
+#pragma unroll
+                for (int x = 0; x < kBPer; ++x) {
+                    const int c = ltid + x * kTcConvT, jr = c >> 3, ch = c & 7;
+                    bv[x] = make_uint4(0u, 0u, 0u, 0u);
+                    if (jr < nrow) {
+                        const unsigned char *br = s_brow[jr / 3];
+                        if (br)
+                            bv[x] = __ldg(reinterpret_cast<const uint4 *>(br + (size_t)s2 * kLimbBlockBytes +
+                                                                          (jr % 3) * kLimbBlockK + 128 * u2 + 16 * ch));
+                    }
+                }
+            };
+            bload(0, 0);
+            bool ok = true;
+            for (int s = 0; s < nst && ok; ++s) {
+                if (!mbar_wait(&pk_full[pstage], pphase, p.status)) { ok = false; break; }
+                const unsigned char *pk = pack + (size_t)pstage * C::kPackBytes;
+                for (int u = 0; u < 2; ++u) {
+                    const int k0 = 256 * s + 128 * u;   // first K value of this half
+                    if (k0 >= it.K) break;
+                    if (!mbar_wait(&sb_empty[sub], sphase ^ 1u, p.status)) { ok = false; break; }
+                    unsigned char *sb = subs + (size_t)sub * C::kSubBytes;
+                    // weights: packed row bytes [64u, 64u + 64) -> 128 s8 bytes in limb order;
+                    // a thread takes one 64-K group of one row (32 packed bytes -> 64 bytes)
+                    for (int w = ltid; w < C::kMats * kTcRows * 2; w += kTcConvT) {
+                        const int m = w / (kTcRows * 2), r = (w >> 1) % kTcRows, gq = w & 1;
+                        const unsigned char *prow = pk + (size_t)(m * kTcRows + r) * kBoxBytes;
+                        const int c0 = 4 * u + 2 * gq;   // 16-byte packed chunks c0 (words 0-3) and c0 + 1 (words 4-7)
+                        const uint4 lo = *reinterpret_cast<const uint4 *>(prow + ((c0 ^ (r & 7)) << 4));
+                        const uint4 hi = *reinterpret_cast<const uint4 *>(prow + (((c0 + 1) ^ (r & 7)) << 4));
+                        const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
+                        unsigned char *arow = sb + (size_t)m * C::kABytes + r * 128;
+#pragma unroll
+                        for (int tq = 0; tq < 4; ++tq) {   // words tq and tq + 4 of the group -> one 16-byte chunk
+                            uint32_t e0, o0, e1, o1;
+                            int4_word_to_s8x16(wl[tq], e0, o0);
+                            int4_word_to_s8x16(wh[tq], e1, o1);
+                            const int ch = 4 * gq + tq;
+                            *reinterpret_cast<uint4 *>(arow + ((ch ^ (r & 7)) << 4)) = make_uint4(e0, e1, o0, o1);
+                        }
+                    }
+                    // activations: limb l of token j -> row 3j + l (zeros up to the MMA's N)
+                    unsigned char *bsm = sb + (size_t)C::kMats * C::kABytes;
+#pragma unroll
+                    for (int x = 0; x < kBPer; ++x) {
+                        const int c = ltid + x * kTcConvT, jr = c >> 3, ch = c & 7;
+                        if (jr < n) *reinterpret_cast<uint4 *>(bsm + jr * 128 + ((ch ^ (jr & 7)) << 4)) = bv[x];
+                    }
+                    // the next sub-stage's pieces, in flight while this one is consumed
+                    {
+                        const int un = u ^ 1, sn = s + u;
+                        if (256 * sn + 128 * un < it.K) bload(sn, un);
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor cores
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sb_full[sub]);
+                    if (++sub == kTcSub) { sub = 0; sphase ^= 1u; }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&pk_empty[pstage]);
+                if (++pstage == kTcPack) { pstage = 0; pphase ^= 1u; }
+            }
+            if (!ok) {
+                *cfail = 1;
+                *abort_flag = 1;
+            }
+            if (GU) settle<GU, kTcConvT>(p, pend, ltid);   // the previous item's h conversion, if due
+            consumer_sync<kTcConvT>();
+            if (*cfail) break;
+
+            // ---------------------------------------------------------------- epilogue
+            const int buf = n_item & 1;
+            if (!mbar_wait(&acc_full[buf], (uint32_t)((n_item >> 1) & 1), p.status)) {
+                *cfail = 1;
+                *abort_flag = 1;
+            }
+            tc_fence_after();
+            const int rows_all = slot_rows<GU>(p, sh);
+            const int ez = sh ? 0 : it.e;
+            const int row = it.row0 + row_l;
+            const float *sc0 = GU ? (sh ? p.wt.sh_g_scale : p.wt.g_scale) : (sh ? p.wt.sh_d_scale : p.wt.d_scale);
+            const float *sc1 = sh ? p.wt.sh_u_scale : p.wt.u_scale;
+            const double rs0 = (double)__ldg(sc0 + (size_t)ez * rows_all + row);
+            const double rs1 = GU ? (double)__ldg(sc1 + (size_t)ez * rows_all + row) : 0.0;
+            const uint32_t tbase = tmem + ((uint32_t)(32 * quarter) << 16) + buf * C::kAccCols;
+            // 8 tokens = 24 accumulator columns per matrix at a time; the quarter's two warps
+            // take alternate blocks of 8 tokens
+            for (int j0 = 8 * half; j0 < it.ntok; j0 += 16) {
+                uint32_t a[C::kMats][24];
+#pragma unroll
+                for (int m = 0; m < C::kMats; ++m)
+#pragma unroll
+                    for (int c8 = 0; c8 < 3; ++c8) {
+                        uint32_t v[8];
+                        tmem_ld8(tbase + m * kTcNMax + 3 * j0 + 8 * c8, v);
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) a[m][8 * c8 + x] = v[x];
+                    }
+                tmem_wait_ld();
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const int j = j0 + jj;
+                    const bool valid = j < it.ntok;
+                    long long Sv[C::kMats];
+#pragma unroll
+                    for (int m = 0; m < C::kMats; ++m)
+                        Sv[m] = (long long)((int)a[m][3 * jj] >> 4) + 256ll * ((int)a[m][3 * jj + 1] >> 4) +
+                                65536ll * ((int)a[m][3 * jj + 2] >> 4);
+                    const int bpos = it.tok0 + j;
+                    float hm = 0.f;
+                    if (GU) {
+                        float hv = 0.f;
+                        if (valid) {
+                            const int tok = s_id[j];
+                            if (tok < 0) record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
+                            if (tok >= 0) {
+                                const double xs = (double)s_sc[j];
+                                const float gv = (float)((double)Sv[0] * xs * rs0);
+                                const float uv = (float)((double)Sv[C::kMats - 1] * xs * rs1);
+                                hv = gv / (1.f + expf(-gv)) * uv;
+                            }
+                            __half *dst = sh ? p.h_sh + (size_t)bpos * p.I_sh : p.h + (size_t)(it.boff + bpos) * p.I;
+                            const __half hh = __float2half_rn(hv);
+                            dst[row] = hh;
+                            hm = fabsf(__half2float(hh));
+                        }
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) hm = fmaxf(hm, __shfl_xor_sync(0xffffffffu, hm, o));
+                        if (valid && lane == 0)
+                            atomicMax(p.h_amax + (sh ? p.T * p.k : it.boff) + bpos, __float_as_uint(hm));
+                    } else if (valid) {
+                        const float yv = (float)((double)Sv[0] * (double)s_sc[j] * rs0);
+                        if (sh) {
+                            p.y_shared[(size_t)bpos * p.H + row] = yv;
+                        } else {
+                            const int aid = s_id[j];
+                            if (aid >= 0) p.y_assign[(size_t)aid * p.H + row] = yv;
+                            else record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if (GU) {
+                // count this row tile of the token group; the last one converts its h rows
+                consumer_sync<kTcConvT>();
+                pend.kind = 1;
+                pend.sh = sh;
+                pend.tok0 = it.tok0;
+                pend.ntok = it.ntok;
+                pend.boff = it.boff;
+                pend.target = (unsigned)(rows_all / kTcRows) - 1u;
+                if (ltid == 0)
+                    pend.old = atom_inc_acq_rel(p.chunk_counters + (sh ? p.T * p.k + it.tok0 : it.boff + it.tok0), pend.target);
+            }
+        }
+        if (GU && !*cfail) settle<GU, kTcConvT>(p, pend, ltid);
+        if (ltid == 0 && !*cfail && atomicAdd(p.work + 1, 1u) == (unsigned)G - 1u) {
+            atomicExch(p.work, 0u);
+            atomicExch(p.work + 1, 0u);
+        }
+    }
+    // every role is done: release the tensor memory
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols));
     }
 }
 
@@ -1286,6 +1772,47 @@ static cudaError_t prepare_fmt(int E, int occ[2][2][2])
     if ((e = prepare_t<FMT, true, 4, 4>(E, &occ[1][1][1])) != cudaSuccess) return e;
     if ((e = prepare_t<FMT, false, 1, 4>(E, &occ[1][0][0])) != cudaSuccess) return e;
     return prepare_t<FMT, false, 4, 4>(E, &occ[1][0][1]);
+}
+
+template <bool GU>
+static cudaError_t tc_prepare_t(int E)
+{
+    int dev = 0, optin = 0;
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, ffn_tc_kernel<GU>);
+    if (e != cudaSuccess) return e;
+    if (tc_smem<GU>(E) + fa.sharedSizeBytes > (size_t)optin) return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(ffn_tc_kernel<GU>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(ffn_tc_kernel<GU>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+}
+
+cudaError_t tc_prepare(int E)
+{
+    cudaError_t e = tc_prepare_t<true>(E);
+    return e != cudaSuccess ? e : tc_prepare_t<false>(E);
+}
+
+// One CTA per SM (the kernel takes most of the shared memory and all of the TMEM).
+cudaError_t launch_tc(const LayerMaps &maps, const FfnParams &p0, bool gate_up, int grid, bool pdl, cudaStream_t s)
+{
+    FfnParams p = p0;
+    p.tok_chunk = kTcTok;
+    p.work = p0.work + (gate_up ? 0 : 2);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = gate_up ? tc_smem<true>(p.E) : tc_smem<false>(p.E);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return gate_up ? cudaLaunchKernelEx(&cfg, ffn_tc_kernel<true>, maps, p)
+                   : cudaLaunchKernelEx(&cfg, ffn_tc_kernel<false>, maps, p);
 }
 
 cudaError_t ffn_prepare(int fmt, int E, int occ[2][2][2])

@@ -445,13 +445,22 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p)
                        p.status, p.slots);
         return;
     }
-    // the last token tile runs the grouping
+    // the last token tile runs the grouping, from a shared-memory copy of all tiles' top-k
+    // when it fits in this CTA's x buffers (one parallel pass instead of dependent loads)
     if (tid == 0) s_flag = atom_inc_acq_rel(p.group_counter, gridDim.y - 1) == gridDim.y - 1;
     __syncthreads();
     if (!s_flag) return;
+    const int n = p.T * p.k;
+    const size_t dyn = p.do_gemv ? (size_t)p.x_bufs * p.x_rows * p.H * 2 : 0;
+    const bool in_smem = (size_t)n * 4 <= dyn;
+    if (in_smem) {
+        int *s_all = reinterpret_cast<int *>(r_smem);
+        for (int a = tid; a < n; a += kRouterThreads) s_all[a] = __ldcg(p.topk_idx + a);
+        __syncthreads();
+    }
     if (warp == 0)
-        group_warp(p.topk_idx, false, p.T * p.k, p.E, p.counts, p.offsets, p.perm, p.unique, p.n_unique, sm_run,
-                   sm_off, p.status, p.slots);
+        group_warp(in_smem ? reinterpret_cast<const int32_t *>(r_smem) : p.topk_idx, in_smem, n, p.E, p.counts,
+                   p.offsets, p.perm, p.unique, p.n_unique, sm_run, sm_off, p.status, p.slots);
 }
 
 __global__ void __launch_bounds__(32) group_kernel(GroupParams p)
