@@ -297,10 +297,10 @@ __device__ __forceinline__ int h_pos(int n)
 
 // named barrier of the four consumer warps (the producer warp never joins it); NT: the
 // threads that meet there (the tensor-memory kernel's converter warps use it too)
-template <int NT = kConsumerWarps * 32>
+template <int NT = kConsumerWarps * 32, int ID = 1>
 __device__ __forceinline__ void consumer_sync()
 {
-    asm volatile("bar.sync 1, %0;" ::"r"(NT) : "memory");
+    asm volatile("bar.sync %0, %1;" ::"n"(ID), "r"(NT) : "memory");
 }
 
 // int4: the fp32 scale of row `row`; NVFP4: the fp32 scale of the whole matrix
@@ -611,7 +611,7 @@ __device__ __forceinline__ bool consume_item(const FfnParams &p, const SlotTable
 // K values each) -> int8 limb rows and their scales.  The rows' largest magnitudes were
 // gathered by the items that wrote them (atomicMax on the float bits, reset here for the
 // next call).  The four consumer warps.
-template <int NT>
+template <int NT, int BAR = 1>
 __device__ __noinline__ void convert_h_rows(const __half *src0, size_t src_stride, unsigned char *dst0, float *scale0,
                                             unsigned *amax0, int ntok, int K, int ltid)
 {
@@ -620,7 +620,7 @@ __device__ __noinline__ void convert_h_rows(const __half *src0, size_t src_strid
         s_m[ltid] = __uint_as_float(__ldcg(amax0 + ltid));
         amax0[ltid] = 0u;
     }
-    consumer_sync<NT>();
+    consumer_sync<NT, BAR>();
     const int nb = (K + kLimbBlockK - 1) / kLimbBlockK;
     const size_t row_bytes = (size_t)nb * kLimbBlockBytes;
     for (int j = 0; j < ntok; ++j) {
@@ -634,7 +634,7 @@ __device__ __noinline__ void convert_h_rows(const __half *src0, size_t src_strid
         }
         if (ltid == 0) scale0[j] = pow2f(-sh);
     }
-    consumer_sync<NT>();   // s_m is reused by the next conversion
+    consumer_sync<NT, BAR>();   // s_m is reused by the next conversion
 }
 
 // A completion counter increment whose result is looked at later: gate/up on the int8
@@ -646,19 +646,19 @@ struct Pending {
     int sh, tok0, ntok, boff;
 };
 
-template <bool GU, int NT = kConsumerWarps * 32>
+template <bool GU, int NT = kConsumerWarps * 32, int BAR = 1>
 __device__ __forceinline__ void settle(const FfnParams &p, Pending &pd, int ltid)
 {
     if (pd.kind == 1) {
         __shared__ int s_conv;
         if (ltid == 0) s_conv = pd.old == pd.target;
-        consumer_sync<NT>();
+        consumer_sync<NT, BAR>();
         if (s_conv) {
             if (pd.sh)
-                convert_h_rows<NT>(p.h_sh + (size_t)pd.tok0 * p.I_sh, p.I_sh, p.hsh_limbs + (size_t)pd.tok0 * limb_row_bytes(p.I_sh),
+                convert_h_rows<NT, BAR>(p.h_sh + (size_t)pd.tok0 * p.I_sh, p.I_sh, p.hsh_limbs + (size_t)pd.tok0 * limb_row_bytes(p.I_sh),
                                p.hsh_limb_scale + pd.tok0, p.h_amax + p.T * p.k + pd.tok0, pd.ntok, p.I_sh, ltid);
             else
-                convert_h_rows<NT>(p.h + (size_t)(pd.boff + pd.tok0) * p.I, p.I,
+                convert_h_rows<NT, BAR>(p.h + (size_t)(pd.boff + pd.tok0) * p.I, p.I,
                                p.h_limbs + (size_t)(pd.boff + pd.tok0) * limb_row_bytes(p.I),
                                p.h_limb_scale + pd.boff + pd.tok0, p.h_amax + pd.boff + pd.tok0, pd.ntok, p.I, ltid);
         }
@@ -1208,7 +1208,8 @@ constexpr int kTcPack = 3;                      // packed stages (256 K each)
 constexpr int kTcSub = 2;                       // expanded sub-stages (128 K each)
 constexpr int kTcConv = 8;                      // converter / epilogue warps (two per TMEM lane quarter)
 constexpr int kTcConvT = kTcConv * 32;
-constexpr int kTcThreads = (2 + kTcConv) * 32;
+constexpr int kTcEpi = 4;                       // epilogue warps (one per TMEM lane quarter)
+constexpr int kTcThreads = (2 + kTcConv + kTcEpi) * 32;
 
 template <bool GU>
 struct TcCfg {
@@ -1226,7 +1227,7 @@ __host__ __device__ constexpr size_t tc_smem(int E)
 {
     using C = TcCfg<GU>;
     return 1024 + (size_t)kTcPack * C::kPackBytes + (size_t)kTcSub * C::kSubBytes + (size_t)4 * 4 * (E + 2) + 64 +
-           kTcTok * 16 + 8 + 8 + (2 * kTcPack + 2 * kTcSub + 4 + 2 * kItemQ + 1) * 8;
+           2 * kTcTok * 16 + 8 + 8 + (2 * kTcPack + 2 * kTcSub + 4 + 2 * kItemQ + 1) * 8;
 }
 
 // UMMA shared-memory descriptor of a K-major tile of 8-row x 128-byte swizzle atoms
@@ -1285,10 +1286,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
     volatile int *abort_flag = tb.hdr + 2;
     volatile int *cfail = tb.hdr + 3;
     volatile int *q_item = tb.hdr + 4;
-    const unsigned char **s_brow = reinterpret_cast<const unsigned char **>(tb.hdr + 16);   // [kTcTok] limb rows
-    float *s_sc = reinterpret_cast<float *>(s_brow + kTcTok);   // [kTcTok] activation scale of each token
-    int *s_id = reinterpret_cast<int *>(s_sc + kTcTok);         // [kTcTok] token (gate/up) or assignment (down)
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(s_id + kTcTok);
+    const unsigned char **s_brow = reinterpret_cast<const unsigned char **>(tb.hdr + 16);   // [2][kTcTok] limb rows
+    float *s_sc = reinterpret_cast<float *>(s_brow + 2 * kTcTok);   // [2][kTcTok] activation scale of each token
+    int *s_id = reinterpret_cast<int *>(s_sc + 2 * kTcTok);         // [2][kTcTok] token (gate/up) or assignment (down)
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(s_id + 2 * kTcTok);
     uint64_t *bars = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(s_tmem + 2) + 7) & ~uintptr_t(7));
     uint64_t *pk_full = bars, *pk_empty = pk_full + kTcPack;
     uint64_t *sb_full = pk_empty + kTcPack, *sb_empty = sb_full + kTcSub;
@@ -1312,11 +1313,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&acc_full[s], 1);
-            mbar_init(&acc_empty[s], kTcConv);
+            mbar_init(&acc_empty[s], kTcEpi);
         }
         for (int q = 0; q < kItemQ; ++q) {
             mbar_init(&q_full[q], 1);
-            mbar_init(&q_empty[q], 1 + kTcConv);
+            mbar_init(&q_empty[q], 1 + kTcConv + kTcEpi);
         }
         mbar_init(table_ready, 1);
         tb.hdr[2] = 0;
@@ -1439,225 +1440,244 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
         }
         if (!ok) *abort_flag = 1;
     } else {
-        // ======================================================== converters + epilogue
-        const int ltid = tid - 64;             // 0 .. kTcConvT - 1
-        const int quarter = warp & 3;          // TMEM lane quarter this warp may access
-        const int half = (warp - 2) >> 2;      // which of the quarter's two warps: token blocks
-        const int row_l = 32 * quarter + lane; // the output row (TMEM lane) of this thread
-        int pstage = 0, sub = 0;
-        uint32_t pphase = 0, sphase = 0;
-        bool have_table = false;
-        Pending pend;
-        pend.kind = 0;
-        for (int n_item = 0;; ++n_item) {
+        // ======================================================== converters / epilogue
+        // the item sequence, as the producer announces it (every role reads it)
+        auto next_item = [&](int n_item, int &i) -> bool {
             const int q = n_item % kItemQ;
-            int i = -1;
-            if (mbar_wait(&q_full[q], (uint32_t)((n_item / kItemQ) & 1), p.status)) {
-                i = q_item[q];
-            } else {
-                *cfail = 1;
-                *abort_flag = 1;
-            }
+            i = -1;
+            const bool got = mbar_wait(&q_full[q], (uint32_t)((n_item / kItemQ) & 1), p.status);
+            if (got) i = q_item[q];
             __syncwarp();
             if (lane == 0) mbar_arrive(&q_empty[q]);
-            consumer_sync<kTcConvT>();
-            if (*cfail || i < 0) break;
-            if (i >= n_pre && !have_table) {
-                if (!mbar_wait(table_ready, 0, p.status)) {
+            return got;
+        };
+        if (warp < 2 + kTcConv) {
+            // -------------------------------------------------------- converters
+            const int ltid = tid - 64;   // 0 .. kTcConvT - 1
+            int pstage = 0, sub = 0;
+            uint32_t pphase = 0, sphase = 0;
+            bool have_table = false;
+            for (int n_item = 0;; ++n_item) {
+                int i;
+                if (!next_item(n_item, i)) {
                     *cfail = 1;
                     *abort_flag = 1;
                 }
-                consumer_sync<kTcConvT>();
-                if (*cfail) break;
-                have_table = true;
-            }
-            if (n_item == 0) pdl_wait();   // limb rows come from the router / the gate/up kernel
-            const Item it = (i < n_pre) ? make_item<GU, RW>(p, -1, p.T, 0, i) : decode_item<GU, RW>(p, tb, i);
-            const bool sh = it.e < 0;
-            const int nrow = 3 * it.ntok;
-            // the item's tokens: limb rows, activation scales, ids (all loads in parallel)
-            if (ltid < it.ntok) {
-                const int bpos = it.tok0 + ltid;
-                s_brow[ltid] = item_brow_limbs<GU>(p, it, ltid);
-                int id = bpos;     // shared expert: the token itself
-                if (!sh) {
-                    const int aid = __ldg(p.perm + it.boff + bpos);
-                    id = (aid >= 0 && aid < p.T * p.k) ? (GU ? aid / p.k : aid) : -1;
-                }
-                s_id[ltid] = id;
-                s_sc[ltid] = GU ? (id >= 0 ? __ldcg(p.x_limb_scale + id) : 0.f)
-                                : __ldcg(sh ? p.hsh_limb_scale + bpos : p.h_limb_scale + it.boff + bpos);
-            }
-            consumer_sync<kTcConvT>();
-            const int nst = (it.K / 2 + kBoxBytes - 1) / kBoxBytes;
-            const int n = ((nrow + 15) / 16) * 16;   // MMA N
-            // this thread's 16-byte pieces of the B rows of one sub-stage (<= 8), loaded
-            // one sub-stage ahead of their use
-            constexpr int kBPer = kTcNMax * 8 / kTcConvT;
-            uint4 bv[kBPer];
-            auto bload = [&](int s2, int u2) {
-#pragma unroll
-                for (int x = 0; x < kBPer; ++x) {
-                    const int c = ltid + x * kTcConvT, jr = c >> 3, ch = c & 7;
-                    bv[x] = make_uint4(0u, 0u, 0u, 0u);
-                    if (jr < nrow) {
-                        const unsigned char *br = s_brow[jr / 3];
-                        if (br)
-                            bv[x] = __ldg(reinterpret_cast<const uint4 *>(br + (size_t)s2 * kLimbBlockBytes +
-                                                                          (jr % 3) * kLimbBlockK + 128 * u2 + 16 * ch));
+                consumer_sync<kTcConvT, 1>();
+                if (*cfail || i < 0) break;
+                if (i >= n_pre && !have_table) {
+                    if (!mbar_wait(table_ready, 0, p.status)) {
+                        *cfail = 1;
+                        *abort_flag = 1;
                     }
+                    consumer_sync<kTcConvT, 1>();
+                    if (*cfail) break;
+                    have_table = true;
                 }
-            };
-            bload(0, 0);
-            bool ok = true;
-            for (int s = 0; s < nst && ok; ++s) {
-                if (!mbar_wait(&pk_full[pstage], pphase, p.status)) { ok = false; break; }
-                const unsigned char *pk = pack + (size_t)pstage * C::kPackBytes;
-                for (int u = 0; u < 2; ++u) {
-                    const int k0 = 256 * s + 128 * u;   // first K value of this half
-                    if (k0 >= it.K) break;
-                    if (!mbar_wait(&sb_empty[sub], sphase ^ 1u, p.status)) { ok = false; break; }
-                    unsigned char *sb = subs + (size_t)sub * C::kSubBytes;
-                    // weights: packed row bytes [64u, 64u + 64) -> 128 s8 bytes in limb order;
-                    // a thread takes one 64-K group of one row (32 packed bytes -> 64 bytes)
-                    for (int w = ltid; w < C::kMats * kTcRows * 2; w += kTcConvT) {
-                        const int m = w / (kTcRows * 2), r = (w >> 1) % kTcRows, gq = w & 1;
-                        const unsigned char *prow = pk + (size_t)(m * kTcRows + r) * kBoxBytes;
-                        const int c0 = 4 * u + 2 * gq;   // 16-byte packed chunks c0 (words 0-3) and c0 + 1 (words 4-7)
-                        const uint4 lo = *reinterpret_cast<const uint4 *>(prow + ((c0 ^ (r & 7)) << 4));
-                        const uint4 hi = *reinterpret_cast<const uint4 *>(prow + (((c0 + 1) ^ (r & 7)) << 4));
-                        const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
-                        unsigned char *arow = sb + (size_t)m * C::kABytes + r * 128;
+                if (n_item == 0) pdl_wait();   // limb rows come from the router / the gate/up kernel
+                const Item it = (i < n_pre) ? make_item<GU, RW>(p, -1, p.T, 0, i) : decode_item<GU, RW>(p, tb, i);
+                const int nrow = 3 * it.ntok;
+                // the item's limb rows (one per token)
+                if (ltid < it.ntok) s_brow[ltid] = item_brow_limbs<GU>(p, it, ltid);
+                consumer_sync<kTcConvT, 1>();
+                const int nst = (it.K / 2 + kBoxBytes - 1) / kBoxBytes;
+                // B: each thread stages half of one limb row (four 16-byte pieces), loaded one
+                // sub-stage ahead of its use; rows past 3 x tokens are never read by the epilogue
+                const int jr = ltid >> 1, bh = ltid & 1;
+                const unsigned char *brow = nullptr;
+                if (jr < nrow) {
+                    const unsigned char *br = s_brow[jr / 3];
+                    if (br) brow = br + (jr % 3) * kLimbBlockK + 64 * bh;
+                }
+                uint4 bv[4];
+                auto bload = [&](int s2, int u2) {
 #pragma unroll
-                        for (int tq = 0; tq < 4; ++tq) {   // words tq and tq + 4 of the group -> one 16-byte chunk
-                            uint32_t e0, o0, e1, o1;
-                            int4_word_to_s8x16(wl[tq], e0, o0);
-                            int4_word_to_s8x16(wh[tq], e1, o1);
-                            const int ch = 4 * gq + tq;
-                            *reinterpret_cast<uint4 *>(arow + ((ch ^ (r & 7)) << 4)) = make_uint4(e0, e1, o0, o1);
+                    for (int x = 0; x < 4; ++x)
+                        bv[x] = brow ? __ldg(reinterpret_cast<const uint4 *>(brow + (size_t)s2 * kLimbBlockBytes + 128 * u2 + 16 * x))
+                                     : make_uint4(0u, 0u, 0u, 0u);
+                };
+                bload(0, 0);
+                bool ok = true;
+                for (int s = 0; s < nst && ok; ++s) {
+                    if (!mbar_wait(&pk_full[pstage], pphase, p.status)) { ok = false; break; }
+                    const unsigned char *pk = pack + (size_t)pstage * C::kPackBytes;
+                    for (int u = 0; u < 2; ++u) {
+                        const int k0 = 256 * s + 128 * u;   // first K value of this half
+                        if (k0 >= it.K) break;
+                        if (!mbar_wait(&sb_empty[sub], sphase ^ 1u, p.status)) { ok = false; break; }
+                        unsigned char *sb = subs + (size_t)sub * C::kSubBytes;
+                        // weights: packed row bytes [64u, 64u + 64) -> 128 s8 bytes in limb order;
+                        // a thread takes one 64-K group of one row (32 packed bytes -> 64 bytes)
+                        for (int w = ltid; w < C::kMats * kTcRows * 2; w += kTcConvT) {
+                            const int m = w / (kTcRows * 2), r = (w >> 1) % kTcRows, gq = w & 1;
+                            const unsigned char *prow = pk + (size_t)(m * kTcRows + r) * kBoxBytes;
+                            const int c0 = 4 * u + 2 * gq;   // packed chunks c0 (words 0-3), c0 + 1 (words 4-7)
+                            const uint4 lo = *reinterpret_cast<const uint4 *>(prow + ((c0 ^ (r & 7)) << 4));
+                            const uint4 hi = *reinterpret_cast<const uint4 *>(prow + (((c0 + 1) ^ (r & 7)) << 4));
+                            const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
+                            unsigned char *arow = sb + (size_t)m * C::kABytes + r * 128;
+#pragma unroll
+                            for (int tq = 0; tq < 4; ++tq) {   // words tq and tq + 4 -> one 16-byte chunk
+                                uint32_t e0, o0, e1, o1;
+                                int4_word_to_s8x16(wl[tq], e0, o0);
+                                int4_word_to_s8x16(wh[tq], e1, o1);
+                                const int ch = 4 * gq + tq;
+                                *reinterpret_cast<uint4 *>(arow + ((ch ^ (r & 7)) << 4)) = make_uint4(e0, e1, o0, o1);
+                            }
+                        }
+                        // activations: limb l of token j -> row 3j + l
+                        if (jr < nrow) {
+                            unsigned char *brs = sb + (size_t)C::kMats * C::kABytes + jr * 128;
+#pragma unroll
+                            for (int x = 0; x < 4; ++x)
+                                *reinterpret_cast<uint4 *>(brs + (((4 * bh + x) ^ (jr & 7)) << 4)) = bv[x];
+                        }
+                        {   // the next sub-stage's pieces, in flight while this one is consumed
+                            const int un = u ^ 1, sn = s + u;
+                            if (256 * sn + 128 * un < it.K) bload(sn, un);
+                        }
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor cores
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sb_full[sub]);
+                        if (++sub == kTcSub) { sub = 0; sphase ^= 1u; }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pk_empty[pstage]);
+                    if (++pstage == kTcPack) { pstage = 0; pphase ^= 1u; }
+                }
+                if (!ok) {
+                    *cfail = 1;
+                    *abort_flag = 1;
+                }
+            }
+        } else {
+            // -------------------------------------------------------- epilogue
+            const int etid = tid - 64 - kTcConvT;   // 0..127
+            const int quarter = warp & 3;           // TMEM lane quarter this warp may access
+            const int row_l = 32 * quarter + lane;  // the output row (TMEM lane) of this thread
+            bool have_table = false, ok = true;
+            Pending pend;
+            pend.kind = 0;
+            for (int n_item = 0;; ++n_item) {
+                int i;
+                if (!next_item(n_item, i)) ok = false;
+                if (!ok || i < 0) break;
+                if (i >= n_pre && !have_table) {
+                    if (!mbar_wait(table_ready, 0, p.status)) { ok = false; break; }
+                    have_table = true;
+                }
+                if (n_item == 0) pdl_wait();
+                const Item it = (i < n_pre) ? make_item<GU, RW>(p, -1, p.T, 0, i) : decode_item<GU, RW>(p, tb, i);
+                const bool sh = it.e < 0;
+                // the item's tokens: activation scales and ids, loaded while the MMAs run
+                if (etid < it.ntok) {
+                    const int bpos = it.tok0 + etid;
+                    int id = bpos;     // shared expert: the token itself
+                    if (!sh) {
+                        const int aid = __ldg(p.perm + it.boff + bpos);
+                        id = (aid >= 0 && aid < p.T * p.k) ? (GU ? aid / p.k : aid) : -1;
+                    }
+                    s_id[etid] = id;
+                    s_sc[etid] = GU ? (id >= 0 ? __ldcg(p.x_limb_scale + id) : 0.f)
+                                    : __ldcg(sh ? p.hsh_limb_scale + bpos : p.h_limb_scale + it.boff + bpos);
+                }
+                consumer_sync<kTcConvT / 2, 2>();
+                const int buf = n_item & 1;
+                if (!mbar_wait(&acc_full[buf], (uint32_t)((n_item >> 1) & 1), p.status)) { ok = false; break; }
+                tc_fence_after();
+                const int rows_all = slot_rows<GU>(p, sh);
+                const int ez = sh ? 0 : it.e;
+                const int row = it.row0 + row_l;
+                const float *sc0 = GU ? (sh ? p.wt.sh_g_scale : p.wt.g_scale) : (sh ? p.wt.sh_d_scale : p.wt.d_scale);
+                const float *sc1 = sh ? p.wt.sh_u_scale : p.wt.u_scale;
+                const double rs0 = (double)__ldg(sc0 + (size_t)ez * rows_all + row);
+                const double rs1 = GU ? (double)__ldg(sc1 + (size_t)ez * rows_all + row) : 0.0;
+                const uint32_t tbase = tmem + ((uint32_t)(32 * quarter) << 16) + buf * C::kAccCols;
+                const float *msc = s_sc;
+                const int *mid = s_id;
+                for (int j0 = 0; j0 < it.ntok; j0 += 8) {   // 8 tokens = 24 accumulator columns per matrix
+                    uint32_t a[C::kMats][24];
+#pragma unroll
+                    for (int m = 0; m < C::kMats; ++m)
+#pragma unroll
+                        for (int c8 = 0; c8 < 3; ++c8) {
+                            uint32_t v[8];
+                            tmem_ld8(tbase + m * kTcNMax + 3 * j0 + 8 * c8, v);
+#pragma unroll
+                            for (int x = 0; x < 8; ++x) a[m][8 * c8 + x] = v[x];
+                        }
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {
+                        const int j = j0 + jj;
+                        const bool valid = j < it.ntok;
+                        long long Sv[C::kMats];
+#pragma unroll
+                        for (int m = 0; m < C::kMats; ++m)
+                            Sv[m] = (long long)((int)a[m][3 * jj] >> 4) + 256ll * ((int)a[m][3 * jj + 1] >> 4) +
+                                    65536ll * ((int)a[m][3 * jj + 2] >> 4);
+                        const int bpos = it.tok0 + j;
+                        if (GU) {
+                            float hm = 0.f;
+                            if (valid) {
+                                float hv = 0.f;
+                                const int tok = mid[j];
+                                if (tok < 0) record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
+                                else {
+                                    const double xs = (double)msc[j];
+                                    const float gv = (float)((double)Sv[0] * xs * rs0);
+                                    const float uv = (float)((double)Sv[C::kMats - 1] * xs * rs1);
+                                    hv = gv / (1.f + expf(-gv)) * uv;
+                                }
+                                __half *dst = sh ? p.h_sh + (size_t)bpos * p.I_sh : p.h + (size_t)(it.boff + bpos) * p.I;
+                                const __half hh = __float2half_rn(hv);
+                                dst[row] = hh;
+                                hm = fabsf(__half2float(hh));
+                            }
+#pragma unroll
+                            for (int o = 16; o > 0; o >>= 1) hm = fmaxf(hm, __shfl_xor_sync(0xffffffffu, hm, o));
+                            if (valid && lane == 0)
+                                atomicMax(p.h_amax + (sh ? p.T * p.k : it.boff) + bpos, __float_as_uint(hm));
+                        } else if (valid) {
+                            const float yv = (float)((double)Sv[0] * (double)msc[j] * rs0);
+                            if (sh) {
+                                p.y_shared[(size_t)bpos * p.H + row] = yv;
+                            } else {
+                                const int aid = mid[j];
+                                if (aid >= 0) p.y_assign[(size_t)aid * p.H + row] = yv;
+                                else record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
+                            }
                         }
                     }
-                    // activations: limb l of token j -> row 3j + l (zeros up to the MMA's N)
-                    unsigned char *bsm = sb + (size_t)C::kMats * C::kABytes;
-#pragma unroll
-                    for (int x = 0; x < kBPer; ++x) {
-                        const int c = ltid + x * kTcConvT, jr = c >> 3, ch = c & 7;
-                        if (jr < n) *reinterpret_cast<uint4 *>(bsm + jr * 128 + ((ch ^ (jr & 7)) << 4)) = bv[x];
-                    }
-                    // the next sub-stage's pieces, in flight while this one is consumed
-                    {
-                        const int un = u ^ 1, sn = s + u;
-                        if (256 * sn + 128 * un < it.K) bload(sn, un);
-                    }
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor cores
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sb_full[sub]);
-                    if (++sub == kTcSub) { sub = 0; sphase ^= 1u; }
                 }
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&pk_empty[pstage]);
-                if (++pstage == kTcPack) { pstage = 0; pphase ^= 1u; }
+                if (lane == 0) mbar_arrive(&acc_empty[buf]);
+                consumer_sync<kTcConvT / 2, 2>();   // s_sc / s_id are rewritten for the next item
+                if (GU) {
+                    // the previous item's h conversion (if it completed a token group), then
+                    // count this row tile of the group; the last one converts its h rows
+                    settle<GU, kTcConvT / 2, 2>(p, pend, etid);
+                    consumer_sync<kTcConvT / 2, 2>();
+                    pend.kind = 1;
+                    pend.sh = sh;
+                    pend.tok0 = it.tok0;
+                    pend.ntok = it.ntok;
+                    pend.boff = it.boff;
+                    pend.target = (unsigned)(rows_all / kTcRows) - 1u;
+                    if (etid == 0)
+                        pend.old = atom_inc_acq_rel(p.chunk_counters + (sh ? p.T * p.k + it.tok0 : it.boff + it.tok0), pend.target);
+                }
             }
             if (!ok) {
                 *cfail = 1;
                 *abort_flag = 1;
             }
-            if (GU) settle<GU, kTcConvT>(p, pend, ltid);   // the previous item's h conversion, if due
-            consumer_sync<kTcConvT>();
-            if (*cfail) break;
-
-            // ---------------------------------------------------------------- epilogue
-            const int buf = n_item & 1;
-            if (!mbar_wait(&acc_full[buf], (uint32_t)((n_item >> 1) & 1), p.status)) {
-                *cfail = 1;
-                *abort_flag = 1;
+            if (GU && ok) settle<GU, kTcConvT / 2, 2>(p, pend, etid);
+            if (etid == 0 && ok && atomicAdd(p.work + 1, 1u) == (unsigned)G - 1u) {
+                atomicExch(p.work, 0u);
+                atomicExch(p.work + 1, 0u);
             }
-            tc_fence_after();
-            const int rows_all = slot_rows<GU>(p, sh);
-            const int ez = sh ? 0 : it.e;
-            const int row = it.row0 + row_l;
-            const float *sc0 = GU ? (sh ? p.wt.sh_g_scale : p.wt.g_scale) : (sh ? p.wt.sh_d_scale : p.wt.d_scale);
-            const float *sc1 = sh ? p.wt.sh_u_scale : p.wt.u_scale;
-            const double rs0 = (double)__ldg(sc0 + (size_t)ez * rows_all + row);
-            const double rs1 = GU ? (double)__ldg(sc1 + (size_t)ez * rows_all + row) : 0.0;
-            const uint32_t tbase = tmem + ((uint32_t)(32 * quarter) << 16) + buf * C::kAccCols;
-            // 8 tokens = 24 accumulator columns per matrix at a time; the quarter's two warps
-            // take alternate blocks of 8 tokens
-            for (int j0 = 8 * half; j0 < it.ntok; j0 += 16) {
-                uint32_t a[C::kMats][24];
-#pragma unroll
-                for (int m = 0; m < C::kMats; ++m)
-#pragma unroll
-                    for (int c8 = 0; c8 < 3; ++c8) {
-                        uint32_t v[8];
-                        tmem_ld8(tbase + m * kTcNMax + 3 * j0 + 8 * c8, v);
-#pragma unroll
-                        for (int x = 0; x < 8; ++x) a[m][8 * c8 + x] = v[x];
-                    }
-                tmem_wait_ld();
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const int j = j0 + jj;
-                    const bool valid = j < it.ntok;
-                    long long Sv[C::kMats];
-#pragma unroll
-                    for (int m = 0; m < C::kMats; ++m)
-                        Sv[m] = (long long)((int)a[m][3 * jj] >> 4) + 256ll * ((int)a[m][3 * jj + 1] >> 4) +
-                                65536ll * ((int)a[m][3 * jj + 2] >> 4);
-                    const int bpos = it.tok0 + j;
-                    float hm = 0.f;
-                    if (GU) {
-                        float hv = 0.f;
-                        if (valid) {
-                            const int tok = s_id[j];
-                            if (tok < 0) record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
-                            if (tok >= 0) {
-                                const double xs = (double)s_sc[j];
-                                const float gv = (float)((double)Sv[0] * xs * rs0);
-                                const float uv = (float)((double)Sv[C::kMats - 1] * xs * rs1);
-                                hv = gv / (1.f + expf(-gv)) * uv;
-                            }
-                            __half *dst = sh ? p.h_sh + (size_t)bpos * p.I_sh : p.h + (size_t)(it.boff + bpos) * p.I;
-                            const __half hh = __float2half_rn(hv);
-                            dst[row] = hh;
-                            hm = fabsf(__half2float(hh));
-                        }
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) hm = fmaxf(hm, __shfl_xor_sync(0xffffffffu, hm, o));
-                        if (valid && lane == 0)
-                            atomicMax(p.h_amax + (sh ? p.T * p.k : it.boff) + bpos, __float_as_uint(hm));
-                    } else if (valid) {
-                        const float yv = (float)((double)Sv[0] * (double)s_sc[j] * rs0);
-                        if (sh) {
-                            p.y_shared[(size_t)bpos * p.H + row] = yv;
-                        } else {
-                            const int aid = s_id[j];
-                            if (aid >= 0) p.y_assign[(size_t)aid * p.H + row] = yv;
-                            else record_error(p.status, MOE_ERR_DEVICE_BOUNDS);
-                        }
-                    }
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);
-            if (GU) {
-                // count this row tile of the token group; the last one converts its h rows
-                consumer_sync<kTcConvT>();
-                pend.kind = 1;
-                pend.sh = sh;
-                pend.tok0 = it.tok0;
-                pend.ntok = it.ntok;
-                pend.boff = it.boff;
-                pend.target = (unsigned)(rows_all / kTcRows) - 1u;
-                if (ltid == 0)
-                    pend.old = atom_inc_acq_rel(p.chunk_counters + (sh ? p.T * p.k + it.tok0 : it.boff + it.tok0), pend.target);
-            }
-        }
-        if (GU && !*cfail) settle<GU, kTcConvT>(p, pend, ltid);
-        if (ltid == 0 && !*cfail && atomicAdd(p.work + 1, 1u) == (unsigned)G - 1u) {
-            atomicExch(p.work, 0u);
-            atomicExch(p.work + 1, 0u);
         }
     }
     // every role is done: release the tensor memory
