@@ -44,7 +44,7 @@ class Case:
             idx, _, sel, gap = oracle.default().route(logits, self.router[1], w.k, self.desc["scaling"])
             order = np.argsort(-sel, axis=1, kind="stable")[:, : w.k + 2]
             experts = np.unique(order)
-        else:
+        elif isinstance(experts, str):   # "all"
             experts = None
         self.host = {"Wr": self.router[0], "bias": self.router[1]}
         self.host.update(synth.make_experts(w, experts))

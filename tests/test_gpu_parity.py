@@ -54,6 +54,25 @@ def test_route_gemv_logits(tiny):
     assert np.array_equal(idx.cpu().numpy()[keep], ref["topk_idx"][keep])
 
 
+@pytest.mark.parametrize("name,T", [("tiny", 17), ("tiny", 37), ("tiny", 64), ("decode8", 40),
+                                    ("prefill512", 512)])
+def test_route_logits_batches(name, T):
+    """Batches of several token tiles (the GEMM-tiled router): logits within fp32
+    accumulation error of the FP64 oracle's, and top-k indices and weights identical to
+    the oracle's routing of the GPU's own logits."""
+    case = Case(W[name], T=T, experts=[0])
+    ws = case.dev.workspace(T)
+    idx, w, lo = case.dev.route(case.x_dev, T, ws, want_logits=True)
+    torch.cuda.synchronize()
+    o = oracle.default()
+    ref = o.router_logits(case.x, case.router[0])
+    lo = lo.cpu().numpy()
+    assert np.abs(lo - ref).max() <= 1e-5 * np.abs(ref).max() + 1e-6
+    r_idx, r_w, _, _ = o.route(lo, case.router[1], case.w.k, case.desc["scaling"])
+    assert np.array_equal(idx.cpu().numpy(), r_idx), "top-k of the GPU logits"
+    check_weights(w.cpu().numpy(), r_w.astype(np.float64))
+
+
 # ------------------------------------------------------------------ grouping
 @pytest.mark.parametrize("T,k,E,mode", [(4, 2, 16, "rand"), (1, 8, 256, "rand"), (16, 8, 256, "rand"),
                                         (512, 8, 256, "rand"), (40, 4, 16, "hot"), (9, 3, 1024, "rand")])
@@ -209,8 +228,9 @@ def test_forward_host_matches_forward(tiny):
 
 
 # ------------------------------------------------------------------ special shapes
-def _special(E, k, n_shared, scaling, fmt=0, bias_hot=None, T=6):
-    H, I = (256, 128) if fmt == 0 else (512, 256)
+def _special(E, k, n_shared, scaling, fmt=0, bias_hot=None, T=6, H=None, I=None):
+    H0, I0 = (256, 128) if fmt == 0 else (512, 256)
+    H, I = H or H0, I or I0
     w = synth.Workload("special", T, H, I, I, E, k, n_shared, scaling, fmt, "uniform", 99)
     host = synth.make_layer(w)
     if bias_hot is not None:
@@ -235,6 +255,19 @@ def _special(E, k, n_shared, scaling, fmt=0, bias_hot=None, T=6):
 ])
 def test_forward_special_shapes(E, k, n_shared, scaling, fmt, hot):
     case = _special(E, k, n_shared, scaling, fmt, hot)
+    y, _ = _forward(case)
+    ref = oracle.default().forward(case.desc, case.host, case.x)
+    check_y(y_to_f64(y), ref["y"], ref["gap"])
+
+
+@pytest.mark.parametrize("E,k,n_shared,fmt,T,H,I", [
+    (32, 8, 1, 1, 40, None, None),   # NVFP4, several token tiles
+    (5, 2, 1, 0, 50, None, None),    # one partial expert tile
+    (40, 4, 1, 0, 70, None, None),   # a full and a partial expert tile
+    (16, 2, 1, 0, 33, 320, 192),     # H with a partial K chunk; int4 rows not multiples of 128
+])
+def test_forward_special_batches(E, k, n_shared, fmt, T, H, I):
+    case = _special(E, k, n_shared, 2.5, fmt, None, T=T, H=H, I=I)
     y, _ = _forward(case)
     ref = oracle.default().forward(case.desc, case.host, case.x)
     check_y(y_to_f64(y), ref["y"], ref["gap"])

@@ -135,6 +135,19 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *src, uint3
                  : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared through L2 only (Ampere-style, per thread),
+// with commit groups and a wait for all but the newest N groups
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;"); }
 

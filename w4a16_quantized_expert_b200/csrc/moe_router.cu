@@ -463,12 +463,309 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p)
                    p.offsets, p.perm, p.unique, p.n_unique, sm_run, sm_off, p.status, p.slots);
 }
 
-__global__ void __launch_bounds__(32) group_kernel(GroupParams p)
+// ---------------------------------------------------------------------------- batches
+// Grouping of n assignments by the eight warps of a CTA (the larger batches): warp w
+// counts its contiguous segment of assignment ids per expert, one exclusive scan over
+// (expert, warp) gives every warp its first position inside each expert's bucket, and
+// each warp then places its segment in ascending a.  Same results as group_warp.
+// cnt: shared memory [8][E]; idx: the n top-k indices (shared or global memory).
+__device__ void group_warps8(const int32_t *idx, bool src_smem, int n, int E, int32_t *counts, int32_t *offsets,
+                             int32_t *perm, int32_t *unique, int32_t *n_unique, int4 *slots, int *cnt, int *status)
 {
-    __shared__ int sm_run[kMaxExperts];
-    __shared__ int sm_off[kMaxExperts + 1];
-    group_warp(p.topk_idx, false, p.T * p.k, p.E, p.counts, p.offsets, p.perm, p.unique, p.n_unique,
-               sm_run, sm_off, p.status);
+    constexpr int kW = kRouterThreads / 32;
+    __shared__ int s_wsum[kW], s_wnz[kW];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int i = tid; i < kW * E; i += kRouterThreads) cnt[i] = 0;
+    __syncthreads();
+    const int seg = (n + kW - 1) / kW;
+    const int a0 = min(n, warp * seg), a1 = min(n, a0 + seg);
+    int *my = cnt + warp * E;
+    for (int base = a0; base < a1; base += 32) {
+        const int a = base + lane;
+        int e = (a < a1) ? (src_smem ? idx[a] : __ldcg(idx + a)) : -1;
+        if (a < a1 && (e < 0 || e >= E)) {
+            record_error(status, MOE_ERR_DEVICE_BOUNDS);
+            e = -1;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    // exclusive scan over experts: thread t owns experts [t*P, t*P + P)
+    const int P = (E + kRouterThreads - 1) / kRouterThreads;
+    const int e0 = tid * P;
+    int local = 0, nz = 0;
+    for (int i = 0; i < P; ++i) {
+        const int e = e0 + i;
+        if (e < E) {
+            int c = 0;
+#pragma unroll
+            for (int w = 0; w < kW; ++w) c += cnt[w * E + e];
+            local += c;
+            nz += c > 0;
+        }
+    }
+    int incl = local, incl_nz = nz;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        const int u = __shfl_up_sync(0xffffffffu, incl_nz, off);
+        if (lane >= off) {
+            incl += v;
+            incl_nz += u;
+        }
+    }
+    if (lane == 31) {
+        s_wsum[warp] = incl;
+        s_wnz[warp] = incl_nz;
+    }
+    __syncthreads();
+    int pre = 0, pre_nz = 0;
+    for (int w = 0; w < warp; ++w) {
+        pre += s_wsum[w];
+        pre_nz += s_wnz[w];
+    }
+    int run = pre + incl - local, ur = pre_nz + incl_nz - nz;
+    for (int i = 0; i < P; ++i) {
+        const int e = e0 + i;
+        if (e < E) {
+            int c = 0;
+#pragma unroll
+            for (int w = 0; w < kW; ++w) {
+                const int cw = cnt[w * E + e];
+                cnt[w * E + e] = run + c;   // warp w's first position in bucket e
+                c += cw;
+            }
+            counts[e] = c;
+            offsets[e] = run;
+            if (c > 0) {
+                if (slots) slots[ur] = make_int4(e, c, run, 0);
+                unique[ur++] = e;
+            }
+            run += c;
+        }
+    }
+    if (tid == kRouterThreads - 1) {
+        offsets[E] = run;
+        *n_unique = ur;
+    }
+    __syncthreads();
+    for (int base = a0; base < a1; base += 32) {
+        const int a = base + lane;
+        int e = (a < a1) ? (src_smem ? idx[a] : __ldcg(idx + a)) : -1;
+        if (e < 0 || e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0) perm[my[e] + __popc(peers & ((1u << lane) - 1u))] = a;
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
+        __syncwarp();
+    }
+}
+
+// Router for batches of more than one token tile: CTA (expert tile, token tile) forms the
+// 16 x 32 block of logits as an fp32 GEMM tile.  K passes through a four-stage ring of
+// shared memory in chunks of 128, filled by every thread with 16-byte asynchronous copies
+// (coalesced rows; small rows make many bulk-copy requests, which the copy engine serves
+// too slowly here); rows are padded so that the lanes' loads meet no bank conflicts.
+// Warp w takes k in [16w, 16w + 16) of every chunk; lane (tg, eg) accumulates
+// tokens {tg, tg + 8} x experts
+// {eg + 4i}; the eight warps' partial sums are added in warp order (deterministic).
+// Scores, top-k and grouping then follow as in the GEMV router.  For the int8 expert
+// path every CTA also tracks the |x| maxima of its rows and, after the GEMM, writes its
+// share of x's limb blocks; for the int4 mma path the CTAs of expert tile 0 write x in
+// B-fragment order from the chunks they stage.
+constexpr int kRtE = 32;                        // experts per CTA
+constexpr int kRtK = 128;                       // K per stage
+constexpr int kRtWStride = kRtK + 4;            // fp32 router row stride in shared memory
+constexpr int kRtXStride = kRtK + 8;            // fp16 token row stride
+constexpr int kRtStageBytes = kRtE * kRtWStride * 4 + kRouterTokTile * kRtXStride * 2;
+constexpr int kRtStages = 4;
+constexpr int kRtSmem = kRtStages * kRtStageBytes;
+static_assert(kRouterTokTile <= 32, "one token row per lane of the issuing warp");
+static_assert(kRtSmem >= kRouterThreads / 32 * kRouterTokTile * (kRtE + 1) * 4, "partial sums alias the ring");
+
+__global__ void __launch_bounds__(kRouterThreads) router_tile_kernel(RouterParams p)
+{
+    extern __shared__ __align__(16) unsigned char r_smem[];
+    __shared__ float s_amax[kRouterTokTile];
+    __shared__ int s_flag;
+    __shared__ int s_idx[kRouterTokTile * kMaxTopK];
+
+    pdl_trigger();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tt = blockIdx.y, t0 = tt * kRouterTokTile, nt = min(kRouterTokTile, p.T - t0);
+    const int eb = blockIdx.x * kRtE, ne = min(kRtE, p.E - eb);
+    if (tt == 0) {
+        // the expert tile's router rows into L2 while earlier work drains
+        for (int r = 0; r < ne; ++r) {
+            const char *row = reinterpret_cast<const char *>(p.w + (size_t)(eb + r) * p.H);
+            for (int o = tid * 128; o < p.H * 4; o += kRouterThreads * 128)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(row + o));
+        }
+    }
+    pdl_wait();
+
+    const int nch = (p.H + kRtK - 1) / kRtK;
+    auto stage_w = [&](int s) { return reinterpret_cast<float *>(r_smem + (size_t)s * kRtStageBytes); };
+    auto stage_x = [&](int s) {
+        return reinterpret_cast<uint16_t *>(r_smem + (size_t)s * kRtStageBytes + kRtE * kRtWStride * 4);
+    };
+    auto issue = [&](int c) {   // all threads: chunk c into stage c % kRtStages (one commit group)
+        if (c < nch) {
+            const int s = c % kRtStages, k0 = c * kRtK, kc = min(kRtK, p.H - k0);
+            constexpr int kW16 = kRtK / 4, kX16 = kRtK / 8;   // 16-byte pieces of a row
+            for (int j = tid; j < kRtE * kW16; j += kRouterThreads) {
+                const int r = j / kW16, q = j % kW16;
+                if (r < ne && 4 * q < kc)
+                    cp_async16(stage_w(s) + r * kRtWStride + 4 * q, p.w + (size_t)(eb + r) * p.H + k0 + 4 * q);
+            }
+            for (int j = tid; j < kRouterTokTile * kX16; j += kRouterThreads) {
+                const int r = j / kX16, q = j % kX16;
+                if (r < nt && 8 * q < kc)
+                    cp_async16(stage_x(s) + r * kRtXStride + 8 * q, p.x + (size_t)(t0 + r) * p.H + k0 + 8 * q);
+            }
+        }
+        cp_async_commit();
+    };
+    for (int c = 0; c < kRtStages - 1; ++c) issue(c);
+
+    const bool conv = p.x_limbs != nullptr;
+    const bool perm = blockIdx.x == 0 && p.x_perm != nullptr;
+    const int nblk = (p.H + kLimbBlockK - 1) / kLimbBlockK;
+
+    const int tg = lane & 7, eg = lane >> 3;
+    float acc[2][8];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[a][i] = 0.f;
+    // |x| maxima of tokens tg and tg + 8 over this warp's k (for the limbs' row scales)
+    __half2 amx[2] = {__float2half2_rn(0.f), __float2half2_rn(0.f)};
+    for (int c = 0; c < nch; ++c) {
+        const int s = c % kRtStages, kc = min(kRtK, p.H - c * kRtK);
+        cp_async_wait<kRtStages - 2>();   // this thread's pieces of chunk c have landed
+        __syncthreads();                  // everyone's have; stage (c - 1) % S is free again
+        issue(c + kRtStages - 1);
+        const float *ws = stage_w(s);
+        const uint16_t *xs = stage_x(s);
+        if (perm) {
+            for (int j = tid; j < nt * (kRtK / 8); j += kRouterThreads) {
+                const int r = j / (kRtK / 8), k8 = (j % (kRtK / 8)) * 8;
+                if (k8 < kc) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(xs + r * kRtXStride + k8);
+                    *reinterpret_cast<uint4 *>(p.x_perm + (size_t)(t0 + r) * p.H + c * kRtK + k8) =
+                        make_uint4(pack_lo(v.x, v.z), pack_hi(v.x, v.z), pack_lo(v.y, v.w), pack_hi(v.y, v.w));
+                }
+            }
+        }
+        const int kw0 = warp * (kRtK / 8), kw1 = min(kc, kw0 + kRtK / 8);
+        for (int k = kw0; k < kw1; k += 4) {
+            float xf[2][4];
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+                const uint2 xr = *reinterpret_cast<const uint2 *>(xs + (tg + 8 * a) * kRtXStride + k);
+                if (conv)
+                    amx[a] = __hmax2(amx[a], __hmax2(__habs2(*reinterpret_cast<const __half2 *>(&xr.x)),
+                                                     __habs2(*reinterpret_cast<const __half2 *>(&xr.y))));
+                const float2 lo = __half22float2(*reinterpret_cast<const __half2 *>(&xr.x));
+                const float2 hi = __half22float2(*reinterpret_cast<const __half2 *>(&xr.y));
+                xf[a][0] = lo.x;
+                xf[a][1] = lo.y;
+                xf[a][2] = hi.x;
+                xf[a][3] = hi.y;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 wv = *reinterpret_cast<const float4 *>(ws + (eg + 4 * i) * kRtWStride + k);
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    acc[a][i] = fmaf(wv.x, xf[a][0], acc[a][i]);
+                    acc[a][i] = fmaf(wv.y, xf[a][1], acc[a][i]);
+                    acc[a][i] = fmaf(wv.z, xf[a][2], acc[a][i]);
+                    acc[a][i] = fmaf(wv.w, xf[a][3], acc[a][i]);
+                }
+            }
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    // partial sums [warp][token][expert] over the (now idle) ring, then summed in warp order
+    float *red = reinterpret_cast<float *>(r_smem);
+    float *amx_w = red + (kRouterThreads / 32) * kRouterTokTile * kRtE;   // [warp][token]
+#pragma unroll
+    for (int a = 0; a < 2; ++a) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) red[(warp * kRouterTokTile + tg + 8 * a) * kRtE + eg + 4 * i] = acc[a][i];
+        if (conv && eg == 0)
+            amx_w[warp * kRouterTokTile + tg + 8 * a] =
+                fmaxf(__low2float(amx[a]), __high2float(amx[a]));
+    }
+    __syncthreads();
+    if (conv) {
+        // x as int8 limbs: this CTA writes limb blocks b = blockIdx.x (mod expert tiles) of
+        // the tile's rows (x read again, from L2)
+        if (tid < nt) {
+            float m = 0.f;
+#pragma unroll
+            for (int w = 0; w < kRouterThreads / 32; ++w) m = fmaxf(m, amx_w[w * kRouterTokTile + tid]);
+            s_amax[tid] = m;
+            if (blockIdx.x == 0) p.x_limb_scale[t0 + tid] = pow2f(-limb_shift(m));
+        }
+        __syncthreads();
+        for (int b = blockIdx.x; b < nblk; b += gridDim.x)
+            for (int j = tid; j < nt * (kLimbBlockK / 8); j += kRouterThreads) {
+                const int r = j / (kLimbBlockK / 8), k8 = (j % (kLimbBlockK / 8)) * 8, k = b * kLimbBlockK + k8;
+                const uint4 v = k < p.H ? __ldcg(reinterpret_cast<const uint4 *>(p.x + (size_t)(t0 + r) * p.H + k))
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                limb_encode8(v, pow2f(limb_shift(s_amax[r])), p.x_limbs + ((size_t)(t0 + r) * nblk + b) * kLimbBlockBytes,
+                             k8);
+            }
+    }
+    for (int o = tid; o < kRouterTokTile * kRtE; o += kRouterThreads) {
+        const int t = o / kRtE, e = o % kRtE;
+        if (t < nt && e < ne) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kRouterThreads / 32; ++w) v += red[w * kRouterTokTile * kRtE + o];
+            const size_t g = (size_t)(t0 + t) * p.E + eb + e;
+            const float sc = sigmoid_ref(v);
+            p.logits[g] = v;
+            p.score[g] = sc;
+            p.sel[g] = sc + p.bias[eb + e];
+        }
+    }
+    // the last expert tile of this token tile runs its top-k
+    __syncthreads();
+    if (tid == 0) s_flag = atom_inc_acq_rel(p.tile_counters + tt, gridDim.x - 1) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_flag) return;
+    for (int t = warp; t < nt; t += kRouterThreads / 32)
+        topk_token(p.sel + (size_t)(t0 + t) * p.E, p.score + (size_t)(t0 + t) * p.E, p.E, p.k, p.scaling,
+                   p.topk_idx + (size_t)(t0 + t) * p.k, p.topk_w + (size_t)(t0 + t) * p.k, s_idx + t * p.k);
+    if (!p.do_group) return;
+    // the last token tile groups the whole batch
+    __syncthreads();
+    if (tid == 0) s_flag = atom_inc_acq_rel(p.group_counter, gridDim.y - 1) == gridDim.y - 1;
+    __syncthreads();
+    if (!s_flag) return;
+    const int n = p.T * p.k;
+    int *cnt = reinterpret_cast<int *>(r_smem);
+    int *s_all = cnt + (kRouterThreads / 32) * p.E;
+    const bool in_smem = (size_t)((kRouterThreads / 32) * p.E + n) * 4 <= (size_t)kRtSmem;
+    if (in_smem) {
+        for (int a = tid; a < n; a += kRouterThreads) s_all[a] = __ldcg(p.topk_idx + a);
+        __syncthreads();
+    }
+    group_warps8(in_smem ? s_all : p.topk_idx, in_smem, n, p.E, p.counts, p.offsets, p.perm, p.unique, p.n_unique,
+                 p.slots, cnt, p.status);
+}
+
+__global__ void __launch_bounds__(kRouterThreads) group_kernel(GroupParams p)
+{
+    extern __shared__ int g_cnt[];   // [8][E]
+    group_warps8(p.topk_idx, false, p.T * p.k, p.E, p.counts, p.offsets, p.perm, p.unique, p.n_unique, nullptr,
+                 g_cnt, p.status);
 }
 
 __global__ void __launch_bounds__(256) combine_kernel(CombineParams p)
@@ -552,16 +849,21 @@ cudaError_t router_prepare()
     cudaError_t e = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRouterMaxDynSmem);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(router_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(x_limbs_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(router_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRtSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(router_tile_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     return e;
 }
 
 cudaError_t launch_router(const RouterParams &p0, bool pdl, cudaStream_t s)
 {
     RouterParams p = p0;
-    const int gx = p.do_gemv ? p.E : 1;
+    // more than one token tile: the GEMM-tiled router
+    const bool tiled = p.do_gemv && p.T > kRouterTokTile;
+    const int gx = tiled ? (p.E + kRtE - 1) / kRtE : p.do_gemv ? p.E : 1;
     const int gy = (p.T + kRouterTokTile - 1) / kRouterTokTile;
-    size_t smem = 0;
-    if (p.do_gemv) {
+    size_t smem = tiled ? (size_t)kRtSmem : 0;
+    if (p.do_gemv && !tiled) {
         const size_t row = (size_t)p.H * 2;
         p.x_rows = std::min(p.T, kRouterXRows);
         p.x_bufs = (p.T > p.x_rows && 2 * p.x_rows * row <= (size_t)kRouterMaxDynSmem) ? 2 : 1;
@@ -577,12 +879,12 @@ cudaError_t launch_router(const RouterParams &p0, bool pdl, cudaStream_t s)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, router_kernel, p);
+    return tiled ? cudaLaunchKernelEx(&cfg, router_tile_kernel, p) : cudaLaunchKernelEx(&cfg, router_kernel, p);
 }
 
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s)
 {
-    group_kernel<<<1, 32, 0, s>>>(p);
+    group_kernel<<<1, kRouterThreads, (size_t)(kRouterThreads / 32) * p.E * sizeof(int), s>>>(p);
     return cudaGetLastError();
 }
 
