@@ -573,6 +573,7 @@ def main():
                     help="override E (smaller profiling-size layers; not a bench line)")
     ap.add_argument("--hidden", type=int, default=None, help="override H (profiling only)")
     ap.add_argument("--inter", type=int, default=None, help="override I and I_sh (profiling only)")
+    ap.add_argument("--tokens", type=int, default=None, help="override T (profiling only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
@@ -583,6 +584,8 @@ def main():
     if args.hidden or args.inter:
         w = w.with_(H=args.hidden or w.H, I=args.inter or w.I, I_sh=args.inter or w.I_sh,
                     name=f"{w.name}_h{args.hidden or w.H}_i{args.inter or w.I}")
+    if args.tokens:
+        w = w.with_(T=args.tokens, name=f"{w.name}_t{args.tokens}")
     if args.steps is None:
         args.steps = d[0]
     if args.warmup is None:

@@ -1194,40 +1194,61 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
 // N = 3 x tokens rounded up to 16, K = 32 per instruction, s32 accumulators in TMEM).
 //
 // Warps: 0 streams the packed codes with TMA into a ring of 256-K stages; 1 allocates
-// TMEM and issues the MMAs (one thread); 2..5 expand each 128-K half of a stage into the
-// 128-byte-swizzled K-major int8 layout the MMA reads (weights from the packed stage, the
-// tokens' limb rows from global memory), then, once an item's accumulators are complete,
-// read them from TMEM (warp w owns TMEM lanes 32 (w % 4) .., the two warps of a lane quarter
-// split the tokens) and run the epilogue.
+// TMEM and issues the MMAs (one thread); 2..9 expand each 128-K half of a stage to int8
+// and store it straight into tensor memory, where the MMA reads its A operand (row r =
+// TMEM lane r, four s8 per column), and copy the tokens' limb rows for that half into a
+// ring of shared-memory B slots (asynchronous 16-byte copies, in the 128-byte-swizzled
+// K-major layout, several halves ahead); 10..13 read an item's accumulators from TMEM
+// once they are complete (warp w owns TMEM lanes 32 (w % 4) ..) and run the epilogue.
+// Keeping the expanded weights out of shared memory leaves it two passes of a quarter
+// of the traffic (the TMA write and the read of the packed codes) plus the B slots.
 // Accumulators are double-buffered in TMEM, so the next item's MMAs overlap an epilogue.
 
 constexpr int kTcRows = 128;                    // output rows per item (MMA M)
-constexpr int kTcTok = 40;                      // tokens per item
-constexpr int kTcNMax = 128;                    // 3 x 40 rounded up to 16
-constexpr int kTcPack = 3;                      // packed stages (256 K each)
-constexpr int kTcSub = 2;                       // expanded sub-stages (128 K each)
-constexpr int kTcConv = 8;                      // converter / epilogue warps (two per TMEM lane quarter)
+constexpr int kTcTok = 32;                      // tokens per item
+constexpr int kTcNMax = 96;                     // 3 x 32 limb columns
+constexpr int kTcPackMax = 8;                   // packed stages (256 K each) at most
+constexpr int kTcASub = 2;                      // expanded 128-K halves held in TMEM
+constexpr int kTcBMax = 8;                      // B slots at most
+constexpr int kTcBSlot = kTcNMax * 128;         // one B slot: 96 limb rows of 128 K
+constexpr int kTcConv = 8;                      // converter warps (two per TMEM lane quarter)
 constexpr int kTcConvT = kTcConv * 32;
 constexpr int kTcEpi = 4;                       // epilogue warps (one per TMEM lane quarter)
 constexpr int kTcThreads = (2 + kTcConv + kTcEpi) * 32;
+// dynamic shared memory the kernel may take (the device's opt-in maximum less a margin
+// for static shared memory)
+constexpr size_t kTcSmemMax = 232448 - 1024;
+static_assert(kTcBSlot % 1024 == 0, "B slots keep the 1024-byte swizzle atoms aligned");
 
 template <bool GU>
 struct TcCfg {
     static constexpr int kMats = GU ? 2 : 1;
     static constexpr int kPackBytes = kMats * kTcRows * kBoxBytes;   // one 256-K stage of codes
-    static constexpr int kABytes = kTcRows * 128;                    // one matrix, one 128-K sub-stage, s8
-    static constexpr int kBBytes = kTcNMax * 128;                    // limb rows of one sub-stage
-    static constexpr int kSubBytes = kMats * kABytes + kBBytes;
     static constexpr int kAccCols = kMats * kTcNMax;                 // TMEM columns of one accumulator set
-    static constexpr int kTmemCols = 2 * kAccCols;                   // double-buffered (power of two)
+    static constexpr int kACols = kMats * 32;                        // TMEM columns of one expanded 128-K half
+    static constexpr int kACol0 = 2 * kAccCols;                      // first A column
+    static constexpr int kTmemCols = GU ? 512 : 256;                 // (a power of two)
+    static constexpr int kBSlots = GU ? 4 : 6;
+    static_assert(kACol0 + kTcASub * kACols <= kTmemCols, "TMEM budget");
 };
 
+// dynamic shared memory of a launch with np packed stages: stages, B slots, slot table,
+// item metadata, barriers
 template <bool GU>
-__host__ __device__ constexpr size_t tc_smem(int E)
+__host__ __device__ constexpr size_t tc_smem(int E, int np)
 {
     using C = TcCfg<GU>;
-    return 1024 + (size_t)kTcPack * C::kPackBytes + (size_t)kTcSub * C::kSubBytes + (size_t)4 * 4 * (E + 2) + 64 +
-           2 * kTcTok * 16 + 8 + 8 + (2 * kTcPack + 2 * kTcSub + 4 + 2 * kItemQ + 1) * 8;
+    return 1024 + (size_t)np * C::kPackBytes + (size_t)C::kBSlots * kTcBSlot + (size_t)4 * 4 * (E + 2) + 64 +
+           2 * kTcTok * 16 + 8 + 8 + (2 * kTcPackMax + 2 * kTcASub + kTcBMax + 4 + 2 * kItemQ + 1) * 8;
+}
+
+// packed stages of a launch: as many as fit (at most kTcPackMax)
+template <bool GU>
+static int tc_pack_stages(int E)
+{
+    const size_t base = tc_smem<GU>(E, 0);
+    const int n = base < kTcSmemMax ? (int)((kTcSmemMax - base) / TcCfg<GU>::kPackBytes) : 0;
+    return n > kTcPackMax ? kTcPackMax : n;
 }
 
 // UMMA shared-memory descriptor of a K-major tile of 8-row x 128-byte swizzle atoms
@@ -1249,6 +1270,26 @@ __device__ __forceinline__ void umma_s8(uint32_t tmem_d, uint64_t da, uint64_t d
                  "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
                  "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
 }
+
+// the same with the A operand in tensor memory
+__device__ __forceinline__ void umma_s8_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
+                                           uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+                 "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate));
+}
+
+// registers -> 16 consecutive TMEM columns of this thread's lane
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+                 ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+                 "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void umma_commit(uint64_t *bar)
 {
@@ -1274,8 +1315,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
     constexpr int RW = kTcRows / kRowTile;   // 8: items of 128 rows
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *pack = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char *subs = pack + (size_t)kTcPack * C::kPackBytes;            // 1024-aligned (all sizes are)
-    int *tbl = reinterpret_cast<int *>(subs + (size_t)kTcSub * C::kSubBytes);
+    const int NP = p.stages;                                                  // packed stages of this launch
+    unsigned char *bring = pack + (size_t)NP * C::kPackBytes;                 // B slots (1024-aligned: all sizes are)
+    constexpr int NB = C::kBSlots;
+    int *tbl = reinterpret_cast<int *>(bring + (size_t)NB * kTcBSlot);
     const int E = p.E;
     SlotTable tb;
     tb.e = tbl;
@@ -1291,9 +1334,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
     int *s_id = reinterpret_cast<int *>(s_sc + 2 * kTcTok);         // [2][kTcTok] token (gate/up) or assignment (down)
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(s_id + 2 * kTcTok);
     uint64_t *bars = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(s_tmem + 2) + 7) & ~uintptr_t(7));
-    uint64_t *pk_full = bars, *pk_empty = pk_full + kTcPack;
-    uint64_t *sb_full = pk_empty + kTcPack, *sb_empty = sb_full + kTcSub;
-    uint64_t *acc_full = sb_empty + kTcSub, *acc_empty = acc_full + 2;
+    uint64_t *pk_full = bars, *pk_empty = pk_full + kTcPackMax;
+    uint64_t *sb_full = pk_empty + kTcPackMax, *sb_empty = sb_full + kTcASub;   // expanded halves in TMEM
+    uint64_t *b_empty = sb_empty + kTcASub;                                     // B slots
+    uint64_t *acc_full = b_empty + kTcBMax, *acc_empty = acc_full + 2;
     uint64_t *q_full = acc_empty + 2, *q_empty = q_full + kItemQ;
     uint64_t *table_ready = q_empty + kItemQ;
 
@@ -1303,14 +1347,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
     const int n_pre = GU ? shared_items<GU, RW>(p) : 0;
 
     if (tid == 0) {
-        for (int s = 0; s < kTcPack; ++s) {
+        for (int s = 0; s < NP; ++s) {
             mbar_init(&pk_full[s], 1);
             mbar_init(&pk_empty[s], kTcConv);
         }
-        for (int s = 0; s < kTcSub; ++s) {
+        for (int s = 0; s < kTcASub; ++s) {
             mbar_init(&sb_full[s], kTcConv);
             mbar_init(&sb_empty[s], 1);
         }
+        for (int s = 0; s < NB; ++s) mbar_init(&b_empty[s], 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&acc_full[s], 1);
             mbar_init(&acc_empty[s], kTcEpi);
@@ -1382,7 +1427,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
                     }
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     unconfirmed |= 1u << stage;
-                    if (++stage == kTcPack) { stage = 0; phase ^= 1u; }
+                    if (++stage == NP) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) *abort_flag = 1;
             }
@@ -1391,11 +1436,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
         }
         if (!have_table && lane == 0) mbar_arrive(table_ready);
         if (lane == 0 && !ok)
-            for (int s = 0; s < kTcPack; ++s)
+            for (int s = 0; s < NP; ++s)
                 if (unconfirmed >> s & 1u) mbar_wait(&pk_full[s], issued_phase >> s & 1u, p.status, 10000000ull);
     } else if (warp == 1) {
         // ======================================================== MMA issuer
-        int sub = 0;
+        int sub = 0, gs = 0;   // expanded half (TMEM); halves so far (B slot gs % NB)
         uint32_t sphase = 0;
         bool ok = true, have_table = false;
         for (int n_item = 0; ok; ++n_item) {
@@ -1422,20 +1467,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
                 if (!mbar_wait(&sb_full[sub], sphase, p.status)) { ok = false; break; }
                 tc_fence_after();
                 const int kvals = min(128, it.K - 128 * u);   // a multiple of 64
+                const int bslot = gs % NB;
                 if (lane == 0) {
-                    const uint32_t sbase = smem_u32(subs + (size_t)sub * C::kSubBytes);
+                    const uint32_t bbase = smem_u32(bring + (size_t)bslot * kTcBSlot);
+                    const uint32_t abase = tmem + C::kACol0 + sub * C::kACols;
                     for (int kk = 0; kk < kvals / 32; ++kk) {
-                        const uint64_t db = umma_sdesc(sbase + C::kMats * C::kABytes + 32 * kk);
+                        const uint64_t db = umma_sdesc(bbase + 32 * kk);
 #pragma unroll
                         for (int m = 0; m < C::kMats; ++m)
-                            umma_s8(tmem + buf * C::kAccCols + m * kTcNMax, umma_sdesc(sbase + m * C::kABytes + 32 * kk),
-                                    db, idesc, (u > 0 || kk > 0) ? 1u : 0u);
+                            umma_s8_ta(tmem + buf * C::kAccCols + m * kTcNMax, abase + m * 32 + 8 * kk, db, idesc,
+                                       (u > 0 || kk > 0) ? 1u : 0u);
                     }
-                    umma_commit(&sb_empty[sub]);   // the sub-stage is free once these MMAs have read it
+                    umma_commit(&sb_empty[sub]);   // the half and the B slot are free once
+                    umma_commit(&b_empty[bslot]);  // these MMAs have read them
                     if (u == nsub - 1) umma_commit(&acc_full[buf]);
                 }
                 __syncwarp();
-                if (++sub == kTcSub) { sub = 0; sphase ^= 1u; }
+                ++gs;
+                if (++sub == kTcASub) { sub = 0; sphase ^= 1u; }
             }
         }
         if (!ok) *abort_flag = 1;
@@ -1454,7 +1503,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
         if (warp < 2 + kTcConv) {
             // -------------------------------------------------------- converters
             const int ltid = tid - 64;   // 0 .. kTcConvT - 1
-            int pstage = 0, sub = 0;
+            int pstage = 0, sub = 0, gsub = 0;   // gsub: halves of earlier items (B slots used)
             uint32_t pphase = 0, sphase = 0;
             bool have_table = false;
             for (int n_item = 0;; ++n_item) {
@@ -1481,70 +1530,90 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
                 if (ltid < it.ntok) s_brow[ltid] = item_brow_limbs<GU>(p, it, ltid);
                 consumer_sync<kTcConvT, 1>();
                 const int nst = (it.K / 2 + kBoxBytes - 1) / kBoxBytes;
-                // B: each thread stages half of one limb row (four 16-byte pieces), loaded one
-                // sub-stage ahead of its use; rows past 3 x tokens are never read by the epilogue
-                const int jr = ltid >> 1, bh = ltid & 1;
-                const unsigned char *brow = nullptr;
-                if (jr < nrow) {
-                    const unsigned char *br = s_brow[jr / 3];
-                    if (br) brow = br + (jr % 3) * kLimbBlockK + 64 * bh;
-                }
-                uint4 bv[4];
-                auto bload = [&](int s2, int u2) {
+                const int nsub = (it.K + 127) / 128;
+                // B: the 3 x tokens limb rows of every 128-K half, 16-byte pieces (8 per row),
+                // copied into B slot (gsub + half) % NB in the swizzled layout the MMA reads, up
+                // to NB - 2 halves ahead (a slot is refilled two halves after its last use, so the
+                // copies never wait for the MMAs just handed over).  Thread ltid owns pieces
+                // ltid, ltid + 256, ltid + 512 of each half.
+                const unsigned char *bsrc[3];
+                int bdst[3];
 #pragma unroll
-                    for (int x = 0; x < 4; ++x)
-                        bv[x] = brow ? __ldg(reinterpret_cast<const uint4 *>(brow + (size_t)s2 * kLimbBlockBytes + 128 * u2 + 16 * x))
-                                     : make_uint4(0u, 0u, 0u, 0u);
-                };
-                bload(0, 0);
+                for (int q = 0; q < 3; ++q) {
+                    const int pc = ltid + q * kTcConvT, jr = pc >> 3, x = pc & 7;
+                    bsrc[q] = nullptr;
+                    bdst[q] = -1;
+                    if (jr < nrow) {
+                        bdst[q] = jr * 128 + ((x ^ (jr & 7)) << 4);
+                        const unsigned char *br = s_brow[jr / 3];
+                        if (br) bsrc[q] = br + (jr % 3) * kLimbBlockK + 16 * x;
+                    }
+                }
+                const int ahead = min(NB - 2, nsub);
                 bool ok = true;
+                auto bissue = [&](int u2) {   // half u2 of this item into its slot (one commit group)
+                    const int g = gsub + u2, slot = g % NB;
+                    if (!mbar_wait(&b_empty[slot], (uint32_t)(((g / NB) & 1) ^ 1), p.status)) ok = false;
+                    if (ok) {
+                        unsigned char *sl = bring + (size_t)slot * kTcBSlot;
+                        const size_t so = (size_t)(u2 >> 1) * kLimbBlockBytes + 128 * (u2 & 1);
+#pragma unroll
+                        for (int q = 0; q < 3; ++q) {
+                            if (bdst[q] < 0) continue;
+                            if (bsrc[q]) cp_async16(sl + bdst[q], bsrc[q] + so);
+                            else *reinterpret_cast<uint4 *>(sl + bdst[q]) = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                    }
+                    cp_async_commit();
+                };
+                for (int u2 = 0; u2 < ahead; ++u2) bissue(u2);
+                // A: this thread expands row r of matrix m (gate/up), or one 64-K group of row r
+                // (down: the two warps of a lane quarter split each half), into TMEM lane r
+                const int cw = warp - 2, quarter = warp & 3, r = 32 * quarter + lane;
+                const int m = GU ? cw / 4 : 0, g0 = GU ? 0 : cw / 4, ng = GU ? 2 : 1;
+                const uint32_t tlane = tmem + ((uint32_t)(32 * quarter) << 16);
                 for (int s = 0; s < nst && ok; ++s) {
                     if (!mbar_wait(&pk_full[pstage], pphase, p.status)) { ok = false; break; }
-                    const unsigned char *pk = pack + (size_t)pstage * C::kPackBytes;
+                    const unsigned char *prow = pack + (size_t)pstage * C::kPackBytes + (size_t)(m * kTcRows + r) * kBoxBytes;
                     for (int u = 0; u < 2; ++u) {
                         const int k0 = 256 * s + 128 * u;   // first K value of this half
                         if (k0 >= it.K) break;
                         if (!mbar_wait(&sb_empty[sub], sphase ^ 1u, p.status)) { ok = false; break; }
-                        unsigned char *sb = subs + (size_t)sub * C::kSubBytes;
-                        // weights: packed row bytes [64u, 64u + 64) -> 128 s8 bytes in limb order;
-                        // a thread takes one 64-K group of one row (32 packed bytes -> 64 bytes)
-                        for (int w = ltid; w < C::kMats * kTcRows * 2; w += kTcConvT) {
-                            const int m = w / (kTcRows * 2), r = (w >> 1) % kTcRows, gq = w & 1;
-                            const unsigned char *prow = pk + (size_t)(m * kTcRows + r) * kBoxBytes;
+                        tc_fence_after();
+                        // packed row bytes [64u, 64u + 64) -> 128 s8 bytes in limb order: 64-K group
+                        // gq -> columns 16 gq .. 16 gq + 15 of the half (words tq, tq + 4 of the group
+                        // -> columns 4 tq .. 4 tq + 3: their even, then their odd elements)
+                        for (int gi = 0; gi < ng; ++gi) {
+                            const int gq = g0 + gi;
                             const int c0 = 4 * u + 2 * gq;   // packed chunks c0 (words 0-3), c0 + 1 (words 4-7)
                             const uint4 lo = *reinterpret_cast<const uint4 *>(prow + ((c0 ^ (r & 7)) << 4));
                             const uint4 hi = *reinterpret_cast<const uint4 *>(prow + (((c0 + 1) ^ (r & 7)) << 4));
                             const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
-                            unsigned char *arow = sb + (size_t)m * C::kABytes + r * 128;
+                            uint32_t v[16];
 #pragma unroll
-                            for (int tq = 0; tq < 4; ++tq) {   // words tq and tq + 4 -> one 16-byte chunk
-                                uint32_t e0, o0, e1, o1;
-                                int4_word_to_s8x16(wl[tq], e0, o0);
-                                int4_word_to_s8x16(wh[tq], e1, o1);
-                                const int ch = 4 * gq + tq;
-                                *reinterpret_cast<uint4 *>(arow + ((ch ^ (r & 7)) << 4)) = make_uint4(e0, e1, o0, o1);
+                            for (int tq = 0; tq < 4; ++tq) {
+                                int4_word_to_s8x16(wl[tq], v[4 * tq], v[4 * tq + 2]);
+                                int4_word_to_s8x16(wh[tq], v[4 * tq + 1], v[4 * tq + 3]);
                             }
+                            tmem_st16(tlane + C::kACol0 + sub * C::kACols + m * 32 + 16 * gq, v);
                         }
-                        // activations: limb l of token j -> row 3j + l
-                        if (jr < nrow) {
-                            unsigned char *brs = sb + (size_t)C::kMats * C::kABytes + jr * 128;
-#pragma unroll
-                            for (int x = 0; x < 4; ++x)
-                                *reinterpret_cast<uint4 *>(brs + (((4 * bh + x) ^ (jr & 7)) << 4)) = bv[x];
-                        }
-                        {   // the next sub-stage's pieces, in flight while this one is consumed
-                            const int un = u ^ 1, sn = s + u;
-                            if (256 * sn + 128 * un < it.K) bload(sn, un);
-                        }
-                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor cores
+                        // the B copies of a later half, then wait for this half's
+                        const int uu = 2 * s + u;
+                        if (uu + ahead < nsub) bissue(uu + ahead);
+                        else cp_async_commit();
+                        cp_async_wait_n(ahead);
+                        tmem_wait_st();
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // B visible to the tensor cores
+                        tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&sb_full[sub]);
-                        if (++sub == kTcSub) { sub = 0; sphase ^= 1u; }
+                        if (++sub == kTcASub) { sub = 0; sphase ^= 1u; }
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pk_empty[pstage]);
-                    if (++pstage == kTcPack) { pstage = 0; pphase ^= 1u; }
+                    if (++pstage == NP) { pstage = 0; pphase ^= 1u; }
                 }
+                gsub += nsub;
                 if (!ok) {
                     *cfail = 1;
                     *abort_flag = 1;
@@ -1681,6 +1750,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
         }
     }
     // every role is done: release the tensor memory
+    cp_async_wait<0>();   // no B copy may still be landing
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -1803,7 +1873,8 @@ static cudaError_t tc_prepare_t(int E)
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, ffn_tc_kernel<GU>);
     if (e != cudaSuccess) return e;
-    if (tc_smem<GU>(E) + fa.sharedSizeBytes > (size_t)optin) return cudaErrorInvalidValue;
+    if (tc_pack_stages<GU>(E) < 2 || tc_smem<GU>(E, tc_pack_stages<GU>(E)) + fa.sharedSizeBytes > (size_t)optin)
+        return cudaErrorInvalidValue;
     e = cudaFuncSetAttribute(ffn_tc_kernel<GU>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(ffn_tc_kernel<GU>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
@@ -1821,10 +1892,11 @@ cudaError_t launch_tc(const LayerMaps &maps, const FfnParams &p0, bool gate_up, 
     FfnParams p = p0;
     p.tok_chunk = kTcTok;
     p.work = p0.work + (gate_up ? 0 : 2);
+    p.stages = gate_up ? tc_pack_stages<true>(p.E) : tc_pack_stages<false>(p.E);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kTcThreads);
-    cfg.dynamicSmemBytes = gate_up ? tc_smem<true>(p.E) : tc_smem<false>(p.E);
+    cfg.dynamicSmemBytes = gate_up ? tc_smem<true>(p.E, p.stages) : tc_smem<false>(p.E, p.stages);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
