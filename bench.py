@@ -47,6 +47,7 @@ DEFAULTS = {
     "nvfp4_1": (40000, 400, 32),
     "nvfp4_16": (20000, 400, 16),
     "prefill512": (400, 20, 2),
+    "prefill2048": (100, 5, 1),
     "tiny": (20000, 200, 8),
 }
 

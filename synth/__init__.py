@@ -158,6 +158,9 @@ WORKLOADS = {
                          BASE_SEED + 3),
     "prefill512": Workload("prefill512", 512, 6144, 2048, 2048, 256, 8, 1, 2.5, FMT_INT4,
                            "uniform", BASE_SEED + 4),
+    # larger batch (about 64 tokens per expert): the tensor-memory kernel's compute-heavier regime
+    "prefill2048": Workload("prefill2048", 2048, 6144, 2048, 2048, 256, 8, 1, 2.5, FMT_INT4,
+                            "uniform", BASE_SEED + 5),
 }
 
 

@@ -181,6 +181,16 @@ def test_forward_prefill512_sampled():
     print(f"prefill512 sampled: excluded {excluded}/{len(tokens)}, rel err {err:.3g}")
 
 
+def test_forward_prefill2048_sampled():
+    """About 64 tokens per expert: several 32-token items per expert row tile."""
+    case = Case(W["prefill2048"])
+    y, _ = _forward(case)
+    tokens = [0, 1, 511, 512, 1024, 1535, 2046, 2047]
+    ref = case.oracle_forward(tokens=tokens)
+    excluded, err = check_y(y_to_f64(y)[tokens], ref["y"], ref["gap"])
+    print(f"prefill2048 sampled: excluded {excluded}/{len(tokens)}, rel err {err:.3g}")
+
+
 @pytest.mark.parametrize("T", [1, 2, 15, 16, 17, 33, 64])
 def test_forward_ragged_T(tiny, T):
     case = Case(W["tiny"], T=T, max_tokens=64, batch=T)
