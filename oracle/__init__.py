@@ -58,7 +58,8 @@ class OrcLayer(ctypes.Structure):
                 ("sh_g", vp), ("sh_u", vp), ("sh_d", vp),
                 ("sh_sg", vp), ("sh_su", vp), ("sh_sd", vp),
                 ("sh_bg", vp), ("sh_bu", vp), ("sh_bd", vp),
-                ("sh_tg", ctypes.c_float), ("sh_tu", ctypes.c_float), ("sh_td", ctypes.c_float)]
+                ("sh_tg", ctypes.c_float), ("sh_tu", ctypes.c_float), ("sh_td", ctypes.c_float),
+                ("top_p", ctypes.c_double)]
 
 
 class OrcResult(ctypes.Structure):
@@ -97,6 +98,8 @@ class Oracle:
         L.orc_router_logits.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, vp]
         L.orc_route.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                 vp, vp, vp, vp]
+        L.orc_route_p.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                  ctypes.c_double, vp, vp, vp, vp]
         L.orc_group.argtypes = [vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp]
         L.orc_expert_ffn.argtypes = [ctypes.POINTER(OrcMatrix)] * 3 + [vp, vp, vp]
         L.orc_routed_expert.argtypes = [ctypes.POINTER(OrcLayer), ctypes.c_int, vp, vp, vp]
@@ -105,7 +108,7 @@ class Oracle:
             getattr(L, f).argtypes = [ctypes.POINTER(OrcLayer), vp, ctypes.c_int, vp,
                                       ctypes.POINTER(OrcResult)]
         L.orc_forward_token.argtypes = [ctypes.POINTER(OrcLayer), vp, vp, vp, vp, vp, vp]
-        for f in ("orc_router_logits", "orc_route", "orc_group", "orc_expert_ffn",
+        for f in ("orc_router_logits", "orc_route", "orc_route_p", "orc_group", "orc_expert_ffn",
                   "orc_routed_expert", "orc_shared_expert", "orc_forward",
                   "orc_forward_per_token", "orc_forward_token"):
             getattr(L, f).restype = None
@@ -144,7 +147,9 @@ class Oracle:
         self.lib.orc_router_logits(_p(x), T, H, _p(Wr), E, _p(out))
         return out
 
-    def route(self, logits: np.ndarray, bias: np.ndarray, k: int, scaling: float):
+    def route(self, logits: np.ndarray, bias: np.ndarray, k: int, scaling: float, top_p: float = 0.0):
+        """Top-k routing (and adaptive top-p when 0 < top_p < 1: dropped entries are
+        index -1, weight 0).  Returns idx, w, sel, gap."""
         T, E = logits.shape
         logits = np.ascontiguousarray(logits, np.float32)
         bias = np.ascontiguousarray(bias, np.float32)
@@ -152,7 +157,11 @@ class Oracle:
         w = np.empty((T, k), np.float32)
         sel = np.empty((T, E), np.float32)
         gap = np.empty(T, np.float32)
-        self.lib.orc_route(_p(logits), _p(bias), T, E, k, scaling, _p(idx), _p(w), _p(sel), _p(gap))
+        if top_p:
+            self.lib.orc_route_p(_p(logits), _p(bias), T, E, k, scaling, float(top_p), _p(idx), _p(w),
+                                 _p(sel), _p(gap))
+        else:
+            self.lib.orc_route(_p(logits), _p(bias), T, E, k, scaling, _p(idx), _p(w), _p(sel), _p(gap))
         return idx, w, sel, gap
 
     def group(self, topk_idx: np.ndarray, E: int):
@@ -165,7 +174,8 @@ class Oracle:
         nu = ctypes.c_int32(0)
         self.lib.orc_group(_p(idx), T, k, E, _p(counts), _p(offsets), _p(perm), _p(unique),
                            ctypes.byref(nu))
-        return counts, offsets, perm, unique[: nu.value].copy()
+        # perm holds the offsets[E] grouped assignments (entries dropped by top-p are not)
+        return counts, offsets, perm[: offsets[E]].copy(), unique[: nu.value].copy()
 
     def expert_ffn(self, Wg: dict, Wu: dict, Wd: dict, x: np.ndarray):
         """One expert on one fp64 activation vector.  Each matrix is a dict with
@@ -212,7 +222,8 @@ class Oracle:
             return _p(a)
 
         L = OrcLayer(H=desc["H"], I=desc["I"], I_sh=desc["I_sh"], E=desc["E"], k=desc["k"],
-                     n_shared=desc["n_shared"], format=desc["fmt"], scaling=desc["scaling"])
+                     n_shared=desc["n_shared"], format=desc["fmt"], scaling=desc["scaling"],
+                     top_p=float(desc.get("top_p", 0.0)))
         for f in ("Wr", "bias", "g", "u", "d", "sg", "su", "sd", "bg", "bu", "bd", "tg", "tu",
                   "td", "sh_g", "sh_u", "sh_d", "sh_sg", "sh_su", "sh_sd", "sh_bg", "sh_bu",
                   "sh_bd"):
@@ -278,4 +289,4 @@ def default() -> Oracle:
 def desc_of(w) -> dict:
     """Layer description dict from a ``synth.Workload``."""
     return {"H": w.H, "I": w.I, "I_sh": w.I_sh, "E": w.E, "k": w.k, "n_shared": w.n_shared,
-            "scaling": w.scaling, "fmt": w.fmt}
+            "scaling": w.scaling, "fmt": w.fmt, "top_p": float(getattr(w, "top_p", 0.0))}

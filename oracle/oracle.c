@@ -42,6 +42,16 @@
  *    sums in ascending index order.
  *  - combine: y_t = shared(x_t) + sum_{j=0..k-1} w_tj * y_{e_tj}(x_t), the shared
  *    expert with weight 1.
+ *  - adaptive expert top-p (hakusoku page, section "実行・チューニングパラメータ":
+ *    the --topp option, which names the idea and its effect but not the rule).
+ *    Reading: after top-k, order the k chosen experts by their score s (descending,
+ *    equal scores -> lower expert index) and keep the shortest leading run whose
+ *    score sum reaches top_p times the sum over all k (at least one expert): expert
+ *    r of that order is kept iff the sum of the r before it is below top_p * S, all
+ *    sums in fp64 in the stated order, S summed in top-k order.  Kept experts keep
+ *    their top-k order and move to the front; their weights are scaling * s / S'
+ *    (S' the kept scores summed in top-k order); the rest are index -1, weight 0,
+ *    and take no part in grouping or combine.
  */
 #include <math.h>
 #include <stdint.h>
@@ -127,6 +137,64 @@ float orc_sigmoid_f32(float logit)
 void orc_route(const float *logits, const float *bias, int T, int E, int k, double scaling,
                int32_t *topk_idx, float *topk_w, float *sel_out, float *gap_out)
 {
+    orc_route_p(logits, bias, T, E, k, scaling, 0.0, topk_idx, topk_w, sel_out, gap_out);
+}
+
+/* Adaptive top-p on one token's k chosen experts (see the header comment).  Rewrites
+ * idx / w in place; returns the smallest distance of a cumulative share from top_p
+ * (how close the decision came to flipping), or +inf when nothing was decided. */
+static double top_p_token(const float *s, int k, double scaling, double top_p, int32_t *idx, float *w)
+{
+    double S = 0.0;
+    for (int j = 0; j < k; j++) S += (double)s[idx[j]];
+    /* order of the k experts by score: rank[j] = number of experts ahead of j */
+    int *rank = (int *)malloc(sizeof(int) * (size_t)k);
+    int *at = (int *)malloc(sizeof(int) * (size_t)k);
+    for (int j = 0; j < k; j++) {
+        int r = 0;
+        for (int i = 0; i < k; i++) {
+            float si = s[idx[i]], sj = s[idx[j]];
+            if (si > sj || (si == sj && idx[i] < idx[j])) r++;
+        }
+        rank[j] = r;
+        at[r] = j;
+    }
+    char *keep = (char *)calloc((size_t)k, 1);
+    double before = 0.0, margin = INFINITY;
+    for (int r = 0; r < k; r++) {                      /* walk the score order */
+        if (r > 0) {
+            double d = fabs(before / S - top_p);
+            if (d < margin) margin = d;
+        }
+        keep[at[r]] = before < top_p * S;
+        before += (double)s[idx[at[r]]];
+    }
+    double S2 = 0.0;
+    for (int j = 0; j < k; j++)
+        if (keep[j]) S2 += (double)s[idx[j]];
+    int32_t *old = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
+    memcpy(old, idx, sizeof(int32_t) * (size_t)k);
+    int m = 0;
+    for (int j = 0; j < k; j++)
+        if (keep[j]) {
+            idx[m] = old[j];
+            w[m] = (float)(scaling * ((double)s[old[j]] / S2));
+            m++;
+        }
+    for (; m < k; m++) {
+        idx[m] = -1;
+        w[m] = 0.0f;
+    }
+    free(rank);
+    free(at);
+    free(keep);
+    free(old);
+    return margin;
+}
+
+void orc_route_p(const float *logits, const float *bias, int T, int E, int k, double scaling,
+                 double top_p, int32_t *topk_idx, float *topk_w, float *sel_out, float *gap_out)
+{
     float *s = (float *)malloc(sizeof(float) * (size_t)E);
     float *sel = (float *)malloc(sizeof(float) * (size_t)E);
     char *taken = (char *)malloc((size_t)E);
@@ -151,13 +219,20 @@ void orc_route(const float *logits, const float *bias, int T, int E, int k, doub
         for (int j = 0; j < k; j++)
             topk_w[(size_t)t * k + j] =
                 (float)(scaling * ((double)s[topk_idx[(size_t)t * k + j]] / sum));
-        if (gap_out) {
+        float gap = INFINITY;
+        if (k < E) {
             /* margin between the k-th chosen and the best unchosen selection score */
             float next = -INFINITY;
             for (int e = 0; e < E; e++)
                 if (!taken[e] && sel[e] > next) next = sel[e];
-            gap_out[t] = (k < E) ? (float)((double)last - (double)next) : INFINITY;
+            gap = (float)((double)last - (double)next);
         }
+        if (top_p > 0.0 && top_p < 1.0) {
+            /* the top-p decision's own margin joins the gap (both decide integers) */
+            double m = top_p_token(s, k, scaling, top_p, topk_idx + (size_t)t * k, topk_w + (size_t)t * k);
+            if (m < (double)gap) gap = (float)m;
+        }
+        if (gap_out) gap_out[t] = gap;
     }
     free(s);
     free(sel);
@@ -171,13 +246,14 @@ void orc_group(const int32_t *topk_idx, int T, int k, int E, int32_t *counts, in
 {
     int n = T * k;
     for (int e = 0; e < E; e++) counts[e] = 0;
-    for (int a = 0; a < n; a++) counts[topk_idx[a]]++;
+    for (int a = 0; a < n; a++)
+        if (topk_idx[a] >= 0) counts[topk_idx[a]]++;   /* -1: dropped by top-p */
     offsets[0] = 0;
     for (int e = 0; e < E; e++) offsets[e + 1] = offsets[e] + counts[e];
     int32_t *fill = (int32_t *)calloc((size_t)E, sizeof(int32_t));
     for (int a = 0; a < n; a++) {                      /* ascending a: stable */
         int e = topk_idx[a];
-        perm[offsets[e] + fill[e]++] = a;
+        if (e >= 0) perm[offsets[e] + fill[e]++] = a;
     }
     free(fill);
     int u = 0;
@@ -278,19 +354,20 @@ static void route_all(const orc_layer *L, const uint16_t *x, int T, const float 
         memcpy(R->logits, logits_in, sizeof(float) * (size_t)T * L->E);
     else
         orc_router_logits(x, T, L->H, L->Wr, L->E, R->logits);
-    orc_route(R->logits, L->bias, T, L->E, L->k, L->scaling, R->topk_idx, R->topk_w, R->sel,
-              R->gap);
+    orc_route_p(R->logits, L->bias, T, L->E, L->k, L->scaling, L->top_p, R->topk_idx, R->topk_w,
+                R->sel, R->gap);
 }
 
 static void combine(const orc_layer *L, int T, const double *y_assign, const double *y_shared,
-                    const float *topk_w, double *y)
+                    const int32_t *topk_idx, const float *topk_w, double *y)
 {
     int H = L->H, k = L->k;
     for (int t = 0; t < T; t++)
         for (int m = 0; m < H; m++) {
             double acc = L->n_shared ? y_shared[(size_t)t * H + m] : 0.0;
             for (int j = 0; j < k; j++)
-                acc += (double)topk_w[(size_t)t * k + j] * y_assign[((size_t)t * k + j) * H + m];
+                if (topk_idx[(size_t)t * k + j] >= 0)
+                    acc += (double)topk_w[(size_t)t * k + j] * y_assign[((size_t)t * k + j) * H + m];
             y[(size_t)t * H + m] = acc;
         }
 }
@@ -319,7 +396,7 @@ void orc_forward(const orc_layer *L, const uint16_t *x, int T, const float *logi
             orc_shared_expert(L, xd + (size_t)t * H,
                               R->h_shared ? R->h_shared + (size_t)t * L->I_sh : NULL,
                               R->y_shared + (size_t)t * H);
-    combine(L, T, R->y_assign, R->y_shared, R->topk_w, R->y);
+    combine(L, T, R->y_assign, R->y_shared, R->topk_idx, R->topk_w, R->y);
     free(xd);
 }
 
@@ -335,6 +412,7 @@ void orc_forward_per_token(const orc_layer *L, const uint16_t *x, int T, const f
     for (int t = 0; t < T; t++) {
         for (int j = 0; j < k; j++) {
             int a = t * k + j;
+            if (R->topk_idx[a] < 0) continue;   /* dropped by top-p */
             orc_routed_expert(L, R->topk_idx[a], xd + (size_t)t * H,
                               R->h_assign ? R->h_assign + (size_t)a * L->I : NULL,
                               R->y_assign + (size_t)a * H);
@@ -344,7 +422,7 @@ void orc_forward_per_token(const orc_layer *L, const uint16_t *x, int T, const f
                               R->h_shared ? R->h_shared + (size_t)t * L->I_sh : NULL,
                               R->y_shared + (size_t)t * H);
     }
-    combine(L, T, R->y_assign, R->y_shared, R->topk_w, R->y);
+    combine(L, T, R->y_assign, R->y_shared, R->topk_idx, R->topk_w, R->y);
     free(xd);
 }
 
@@ -357,13 +435,14 @@ void orc_forward_token(const orc_layer *L, const uint16_t *x_t, const float *log
     float *logits = (float *)malloc(sizeof(float) * (size_t)E);
     if (logits_t) memcpy(logits, logits_t, sizeof(float) * (size_t)E);
     else orc_router_logits(x_t, 1, H, L->Wr, E, logits);
-    orc_route(logits, L->bias, 1, E, k, L->scaling, topk_idx, topk_w, NULL, gap);
+    orc_route_p(logits, L->bias, 1, E, k, L->scaling, L->top_p, topk_idx, topk_w, NULL, gap);
     double *xd = (double *)malloc(sizeof(double) * (size_t)H);
     double *ye = (double *)malloc(sizeof(double) * (size_t)H);
     decode_tokens(x_t, 1, H, xd);
     for (int m = 0; m < H; m++) y[m] = 0.0;
     if (L->n_shared) orc_shared_expert(L, xd, NULL, y);
     for (int j = 0; j < k; j++) {
+        if (topk_idx[j] < 0) continue;   /* dropped by top-p */
         orc_routed_expert(L, topk_idx[j], xd, NULL, ye);
         for (int m = 0; m < H; m++) y[m] += (double)topk_w[j] * ye[m];
     }

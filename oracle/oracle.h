@@ -40,6 +40,7 @@ typedef struct {
     const float *sh_sg, *sh_su, *sh_sd;
     const uint8_t *sh_bg, *sh_bu, *sh_bd;
     float sh_tg, sh_tu, sh_td;
+    double top_p;               /* adaptive expert top-p in (0, 1); otherwise off */
 } orc_layer;
 
 /* Caller-allocated outputs of a forward pass (h_assign / h_shared may be NULL). */
@@ -71,6 +72,12 @@ void orc_dequant_matrix(const orc_matrix *M, double *out);
 void orc_router_logits(const uint16_t *x, int T, int H, const float *Wr, int E, float *logits);
 void orc_route(const float *logits, const float *bias, int T, int E, int k, double scaling,
                int32_t *topk_idx, float *topk_w, float *sel_out, float *gap_out);
+/* The same with adaptive expert top-p: of the k chosen experts only the fewest with the
+ * largest scores whose score mass reaches top_p of the k's mass are kept (at least one),
+ * listed first in their top-k order and renormalised to the scaling factor; the other
+ * entries are index -1, weight 0.  top_p outside (0, 1) is plain top-k. */
+void orc_route_p(const float *logits, const float *bias, int T, int E, int k, double scaling,
+                 double top_p, int32_t *topk_idx, float *topk_w, float *sel_out, float *gap_out);
 void orc_group(const int32_t *topk_idx, int T, int k, int E, int32_t *counts, int32_t *offsets,
                int32_t *perm, int32_t *unique, int32_t *n_unique);
 void orc_expert_ffn(const orc_matrix *Wg, const orc_matrix *Wu, const orc_matrix *Wd,

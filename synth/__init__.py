@@ -139,6 +139,7 @@ class Workload:
     fmt: int
     bias: str            # "uniform" (U(-0.1, 0.1)) or "zipf" (Zipf(1.1) ranking into [-0.5, 0.5])
     seed: int
+    top_p: float = 0.0   # adaptive expert top-p (0: plain top-k)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)

@@ -305,9 +305,90 @@ def pin_route_weights(o):
     assert abs(float(gap[0]) - float(np.float32(0.7) - np.float32(0.5))) < 1e-7, gap
 
 
+# ---------------------------------------------------------------- adaptive top-p
+def _logit_of(p):
+    """A float32 logit whose fp32 sigmoid is close to p."""
+    return np.float32(np.log(p / (1.0 - p)))
+
+
+def pin_topp_hand(o):
+    """Hand example (scores about 0.9, 0.8, 0.3, 0.2 among k = 4 of E = 6, shares of
+    the k's mass after 1, 2, 3 experts about 0.41, 0.77, 0.91): p = 0.3 keeps one
+    expert, 0.5 two, 0.8 three, 0.95 all four.  A bias that puts the 0.8 expert first
+    in top-k order must not change which experts top-p keeps (scores decide), while
+    the kept ones stay in top-k order; dropped entries are -1 with weight 0."""
+    sv = [0.9, 0.8, 0.3, 0.2, 0.05, 0.04]
+    logits = np.array([[_logit_of(v) for v in sv]], np.float32)
+    bias = np.zeros(6, np.float32)
+    for p, n in ((0.3, 1), (0.5, 2), (0.8, 3), (0.95, 4)):
+        idx, w, sel, gap = o.route(logits, bias, 4, 2.5, top_p=p)
+        assert idx[0].tolist() == [0, 1, 2, 3][:n] + [-1] * (4 - n), (p, idx)
+        assert np.all(w[0, n:] == 0)
+        s = np.array([o.sigmoid_f32(float(v)) for v in logits[0, :n]], np.float64)
+        _close(w[0, :n], 2.5 * s / s.sum(), 1e-7, "renormalised weights")
+    bias = np.array([0.0, 0.2, 0.0, 0.0, 0.0, 0.0], np.float32)   # expert 1 first by selection
+    idx, w, sel, gap = o.route(logits, bias, 4, 2.5, top_p=0.3)
+    assert idx[0].tolist() == [0, -1, -1, -1], idx                 # the highest score is kept
+    idx, w, sel, gap = o.route(logits, bias, 4, 2.5, top_p=0.5)
+    assert idx[0].tolist() == [1, 0, -1, -1], idx                  # top-k order kept
+
+
+def pin_topp_boundary(o):
+    """Equal scores (logit 0: s = 1/2 exactly, S = 2 for k = 4).  Expert r is kept only
+    while the mass before it is below p * S, so when that mass equals p * S exactly the
+    expert is dropped: p = 1/4 keeps one expert, p just above 1/4 keeps two; equal
+    scores go in index order.  The gap reports the decision margin."""
+    logits = np.zeros((1, 6), np.float32)
+    bias = np.array([0.0, 0.0, 0.0, 0.0, -0.5, -0.5], np.float32)
+    idx, w, sel, gap = o.route(logits, bias, 4, 2.5, top_p=0.25)
+    assert idx[0].tolist() == [0, -1, -1, -1], idx
+    assert w[0, 0] == np.float32(2.5)
+    assert float(gap[0]) == 0.0, gap
+    idx, w, sel, gap = o.route(logits, bias, 4, 2.5, top_p=0.2500001)
+    assert idx[0].tolist() == [0, 1, -1, -1], idx
+    assert np.array_equal(w[0, :2], np.float32([1.25, 1.25]))
+    idx, w, sel, gap = o.route(logits, bias, 4, 2.5, top_p=0.6)
+    assert idx[0].tolist() == [0, 1, 2, -1], idx
+    assert abs(float(gap[0]) - 0.1) < 1e-6, gap                    # |0.5 - 0.6|
+
+
+def pin_topp_bruteforce(o):
+    """Over all subsets of the k chosen experts: top-p keeps the fewest experts whose
+    score mass reaches p times the k's mass, and among those the largest mass; the
+    weights sum to the scaling factor; p outside (0, 1) is plain top-k."""
+    rng = np.random.default_rng(9)
+    for E, k in ((6, 3), (8, 4), (7, 5), (9, 6)):
+        for tr in range(25):
+            T = 4
+            logits = (rng.standard_normal((T, E)) * 1.5).astype(np.float32)
+            bias = rng.uniform(-0.2, 0.2, E).astype(np.float32)
+            p = float(rng.uniform(0.05, 0.98))
+            idx0, w0, _, _ = o.route(logits, bias, k, 2.5)
+            idx, w, sel, gap = o.route(logits, bias, k, 2.5, top_p=p)
+            for off in (0.0, 1.0, 1.5):
+                i2, w2, _, _ = o.route(logits, bias, k, 2.5, top_p=off)
+                assert np.array_equal(i2, idx0) and np.array_equal(w2, w0), "top_p off != top-k"
+            s, _ = _sel_ref(o, logits, bias)
+            for t in range(T):
+                chosen = idx0[t].tolist()
+                S = sum(float(s[t, e]) for e in chosen)
+                kept = [e for e in idx[t].tolist() if e >= 0]
+                assert 1 <= len(kept) <= k
+                assert kept == [e for e in chosen if e in kept], "kept in top-k order"
+                assert all(e == -1 for e in idx[t, len(kept):]) and np.all(w[t, len(kept):] == 0)
+                assert abs(float(w[t, :len(kept)].astype(np.float64).sum()) - 2.5) <= len(kept) * 2 ** -22
+                if float(gap[t]) < 1e-6:
+                    continue   # the decision is within rounding of the threshold
+                best = {m: max(itertools.combinations(chosen, m), key=lambda c: sum(float(s[t, e]) for e in c))
+                        for m in range(1, k + 1)}
+                m_star = min(m for m in range(1, k + 1)
+                             if sum(float(s[t, e]) for e in best[m]) >= p * S)
+                assert sorted(kept) == sorted(best[m_star]), (p, kept, best[m_star])
+
+
 # ---------------------------------------------------------------- grouping
 def _group_brute(idx, E):
-    flat = idx.reshape(-1)
+    flat = idx.reshape(-1)   # -1 entries (dropped by top-p) belong to no expert
     counts = np.array([(flat == e).sum() for e in range(E)], np.int32)
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
     perm = np.array([a for e in range(E) for a in range(len(flat)) if flat[a] == e], np.int32)
@@ -323,6 +404,14 @@ def pin_group_bruteforce(o):
     for _ in range(20):
         T, k, E = int(rng.integers(1, 9)), int(rng.integers(1, 4)), 12
         cases.append(np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32))
+    for _ in range(10):   # with top-p drops: a tail of -1 per token
+        T, k, E = int(rng.integers(1, 9)), int(rng.integers(2, 5)), 12
+        rows = []
+        for _ in range(T):
+            r = rng.choice(E, k, replace=False).astype(np.int32)
+            r[int(rng.integers(1, k + 1)):] = -1
+            rows.append(r)
+        cases.append(np.stack(rows))
     for idx in cases:
         E = 12
         got = o.group(idx, E)
@@ -404,10 +493,32 @@ def pin_forward_token(o):
         assert a["gap"][t] == b["gap"]
 
 
+def pin_topp_layer(o):
+    """With adaptive top-p the batched driver (union of experts) still equals the
+    per-token driver bit for bit, the single-token driver equals both, and a layer
+    whose p keeps every expert equals the plain top-k layer."""
+    desc, L, x = small_layer(E=8, k=4, n_shared=1, fmt=0, scaling=2.5, seed=71)
+    desc = dict(desc, top_p=0.55)
+    a = o.forward(desc, L, x)
+    b = o.forward(desc, L, x, per_token=True)
+    assert np.array_equal(a["y"], b["y"]), "top-p: batched != per-token"
+    assert (a["topk_idx"] == -1).any(), "p = 0.55 drops some expert"
+    for t in range(x.shape[0]):
+        c = o.forward_token(desc, L, x[t])
+        assert np.array_equal(a["y"][t], c["y"]) and np.array_equal(a["topk_idx"][t], c["topk_idx"])
+    assert a["offsets"][-1] == (a["topk_idx"] >= 0).sum(), "only kept assignments are grouped"
+    full = o.forward(dict(desc, top_p=0.0), L, x)
+    keep_all = o.forward(dict(desc, top_p=0.999999), L, x)
+    same = (keep_all["topk_idx"] >= 0).all(axis=1)
+    assert np.array_equal(full["y"][same], keep_all["y"][same])
+
+
 PINS = [pin_half_exhaustive, pin_int4_hand, pin_e2m1_table, pin_e4m3_exhaustive,
         pin_nvfp4_hand, pin_sigmoid_closed_forms, pin_router_onehot, pin_router_matmul,
-        pin_topk_bruteforce, pin_route_weights, pin_group_bruteforce, pin_dense_equivalence,
-        pin_layer_composition, pin_union_identity, pin_expert_relabel, pin_forward_token]
+        pin_topk_bruteforce, pin_route_weights, pin_topp_hand, pin_topp_boundary,
+        pin_topp_bruteforce, pin_group_bruteforce, pin_dense_equivalence,
+        pin_layer_composition, pin_union_identity, pin_expert_relabel, pin_forward_token,
+        pin_topp_layer]
 
 
 def run_all(o) -> list[str]:

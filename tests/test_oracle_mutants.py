@@ -45,8 +45,8 @@ MUTANTS = {
     "weights_no_norm": ("((double)s[topk_idx[(size_t)t * k + j]] / sum));",
                         "((double)s[topk_idx[(size_t)t * k + j]] / 1.0));"),
     "group_unique_all": ("if (counts[e] > 0) unique[u++] = e;", "if (counts[e] >= 0) unique[u++] = e;"),
-    "group_count_dropped": ("for (int a = 0; a < n; a++) counts[topk_idx[a]]++;",
-                            "for (int a = 1; a < n; a++) counts[topk_idx[a]]++;"),
+    "group_count_dropped": ("for (int a = 0; a < n; a++)\n        if (topk_idx[a] >= 0) counts[topk_idx[a]]++;",
+                            "for (int a = 1; a < n; a++)\n        if (topk_idx[a] >= 0) counts[topk_idx[a]]++;"),
     "group_perm_reverse": ("for (int a = 0; a < n; a++) {                      /* ascending a: stable */",
                            "for (int a = n - 1; a >= 0; a--) {"),
     "silu_gate_up_swapped": ("h[n] = g / (1.0 + exp(-g)) * u;", "h[n] = u / (1.0 + exp(-u)) * g;"),
@@ -57,8 +57,19 @@ MUTANTS = {
     "combine_wrong_j": ("acc += (double)topk_w[(size_t)t * k + j] * y_assign",
                         "acc += (double)topk_w[(size_t)t * k + (k - 1 - j)] * y_assign"),
     "batched_token_index": ("int a = R->perm[p], t = a / k;", "int a = R->perm[p], t = a % T;"),
-    "gap_wrong": ("gap_out[t] = (k < E) ? (float)((double)last - (double)next) : INFINITY;",
-                  "gap_out[t] = (k < E) ? (float)((double)last) : INFINITY;"),
+    "gap_wrong": ("gap = (float)((double)last - (double)next);", "gap = (float)((double)last);"),
+    # adaptive expert top-p
+    "topp_le": ("keep[at[r]] = before < top_p * S;", "keep[at[r]] = before <= top_p * S;"),
+    "topp_rank_ascending": ("if (si > sj || (si == sj && idx[i] < idx[j])) r++;",
+                            "if (si < sj || (si == sj && idx[i] < idx[j])) r++;"),
+    "topp_tie_high": ("if (si > sj || (si == sj && idx[i] < idx[j])) r++;",
+                      "if (si > sj || (si == sj && idx[i] > idx[j])) r++;"),
+    "topp_no_renorm": ("w[m] = (float)(scaling * ((double)s[old[j]] / S2));",
+                       "w[m] = (float)(scaling * ((double)s[old[j]] / S));"),
+    "topp_score_order_out": ("idx[m] = old[j];", "idx[m] = old[at[m]];"),
+    "topp_margin_missing": ("if (m < (double)gap) gap = (float)m;", ";"),
+    "topp_kept_not_skipped": ("if (e >= 0) perm[offsets[e] + fill[e]++] = a;",
+                              "if (e >= 0) perm[offsets[e] + fill[e]++] = a; else perm[0] = a;"),
 }
 
 
