@@ -48,6 +48,7 @@ DEFAULTS = {
     "nvfp4_16": (20000, 400, 16),
     "prefill512": (400, 20, 2),
     "prefill2048": (100, 5, 1),
+    "decode1_topp": (40000, 400, 8),
     "tiny": (20000, 200, 8),
 }
 
@@ -65,8 +66,9 @@ NCU_TRAFFIC = {
 def describe(w) -> str:
     fmt = "int4 row-scale" if w.fmt == synth.FMT_INT4 else "NVFP4 (E2M1 + E4M3/16 + fp32)"
     bias = "Zipf(1.1) bias in [-0.5,0.5]" if w.bias == "zipf" else "bias U(-0.1,0.1)"
+    topp = f", adaptive expert top-p {w.top_p}" if getattr(w, "top_p", 0.0) else ""
     return (f"{w.name}: T={w.T}, H={w.H}, I={w.I}, E={w.E}, top-{w.k}, {w.n_shared} shared "
-            f"(I={w.I_sh}), {fmt}, {bias}, scaling {w.scaling}")
+            f"(I={w.I_sh}), {fmt}, {bias}, scaling {w.scaling}{topp}")
 
 
 # ------------------------------------------------------------------ byte accounting
@@ -95,8 +97,11 @@ def algorithmic_bytes(w, U: float) -> dict:
     return {"router": router, "gate_up": gate_up, "down": down, "total": total, "weights": weights}
 
 
-def flops(w) -> float:
-    return 6.0 * w.I * w.H * w.T * w.k + 6.0 * w.I_sh * w.H * w.T * w.n_shared + 2.0 * w.T * w.E * w.H
+def flops(w, assignments=None) -> float:
+    """Expert and router FLOPs of one layer call; ``assignments`` = (token, expert) pairs
+    that reach an expert (T*k, fewer with adaptive top-p)."""
+    a = w.T * w.k if assignments is None else assignments
+    return 6.0 * w.I * w.H * a + 6.0 * w.I_sh * w.H * w.T * w.n_shared + 2.0 * w.T * w.E * w.H
 
 
 def load_peaks() -> dict:
@@ -355,7 +360,7 @@ def run_ours(args, w):
     R = args.layers or DEFAULTS.get(w.name, (0, 0, 8))[2]
     K, Wm = args.steps, args.warmup
     desc = {"H": w.H, "I": w.I, "I_sh": w.I_sh, "E": w.E, "k": w.k, "n_shared": w.n_shared,
-            "scaling": w.scaling, "fmt": w.fmt}
+            "scaling": w.scaling, "fmt": w.fmt, "top_p": w.top_p}
 
     # ---- inputs resident in HBM
     host = synth.make_layer(w)
@@ -368,13 +373,15 @@ def run_ours(args, w):
     stream = torch.cuda.Stream(device=dev)
 
     # unique experts per batch (for the byte accounting), from the library's own grouping
-    U = []
+    U, A = [], []
     with torch.cuda.stream(stream):
         for x in xs:
             idx, _, _ = base.route(x, w.T, ws, stream=stream)
             _, _, _, _, nu = base.group(idx, w.T, ws, stream=stream)
             U.append(int(nu.item()))
+            A.append(int((idx >= 0).sum().item()))   # fewer than T*k with adaptive top-p
     U_mean = float(np.mean(U))
+    A_mean = float(np.mean(A))
     ab = algorithmic_bytes(w, U_mean)
 
     # ---- graphs of R consecutive layer calls
@@ -517,7 +524,7 @@ def run_ours(args, w):
         "data": "synthetic",
         "config": {
             "workload": describe(w),
-            "T": w.T, "H": w.H, "I": w.I, "E": w.E, "top_k": w.k, "n_shared": w.n_shared,
+            "T": w.T, "H": w.H, "I": w.I, "E": w.E, "top_k": w.k, "top_p": w.top_p, "n_shared": w.n_shared,
             "weights": "int4" if w.fmt == synth.FMT_INT4 else "nvfp4",
             "rotating_layers": R,
             "unique_experts_per_step": U_mean,
@@ -535,7 +542,7 @@ def run_ours(args, w):
             "frac_quantized_of_8tbs": weights_gbs / 8000.0,
             "peak_source": peaks["source"],
         },
-        "tflops": flops(w) / (ms_step * 1e-3) / 1e12,
+        "tflops": flops(w, A_mean) / (ms_step * 1e-3) / 1e12,
         "kernels_ms": {n: float(v) for n, v in zip(names, k_ms)},
         "roofline": {
             "kernel": names[dom],

@@ -89,6 +89,15 @@ typedef struct moe_layer_desc {
     float routed_scaling;  /* multiplies the normalised combine weights (e.g. 2.5) */
     int format;            /* MOE_FMT_* */
     int max_tokens;        /* largest T any call on this handle will pass, >= 1 */
+    float top_p;           /* adaptive expert top-p: in (0, 1), of each token's k chosen experts
+                              only the fewest with the highest scores s whose summed s reaches
+                              top_p of the k's sum are kept (at least one), listed first in
+                              top-k order with weights renormalised to routed_scaling; the
+                              other entries are index -1, weight 0 and reach no expert.
+                              0 or >= 1: plain top-k.  (The pages name the option, the
+                              "--topp" flag of the hakusoku page's section
+                              "実行・チューニングパラメータ", not its rule; this is the reading.)
+                              Negative or NaN: MOE_ERR_INVALID_ARG. */
 } moe_layer_desc;
 
 /* Device pointers to one layer's parameters (borrowed; see conventions).

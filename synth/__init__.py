@@ -159,6 +159,10 @@ WORKLOADS = {
                          BASE_SEED + 3),
     "prefill512": Workload("prefill512", 512, 6144, 2048, 2048, 256, 8, 1, 2.5, FMT_INT4,
                            "uniform", BASE_SEED + 4),
+    # decode1 with adaptive expert top-p 0.7 (the value of the --topp example on the hakusoku
+    # page, section "実行・チューニングパラメータ"); same weights and tokens as decode1
+    "decode1_topp": Workload("decode1_topp", 1, 6144, 2048, 2048, 256, 8, 1, 2.5, FMT_INT4,
+                             "uniform", BASE_SEED + 1, top_p=0.7),
     # larger batch (about 64 tokens per expert): the tensor-memory kernel's compute-heavier regime
     "prefill2048": Workload("prefill2048", 2048, 6144, 2048, 2048, 256, 8, 1, 2.5, FMT_INT4,
                             "uniform", BASE_SEED + 5),

@@ -26,6 +26,7 @@ W_RTOL = 1e-6
 def desc_of(w):
     d = oracle.desc_of(w)
     d["scaling"] = float(np.float32(w.scaling))   # the ABI carries an fp32 scaling factor
+    d["top_p"] = float(np.float32(d.get("top_p", 0.0)))   # and an fp32 top-p
     return d
 
 
@@ -73,6 +74,16 @@ def check_y(y_gpu: np.ndarray, y_ref: np.ndarray, gap: np.ndarray, tol: float = 
     err = np.abs(y_gpu[keep] - y_ref[keep]).max() / scale if keep.any() else 0.0
     assert err <= tol, f"max|gpu-oracle| = {err:.3g} * max|oracle| > {tol}"
     return int((~keep).sum()), float(err)
+
+
+def check_routing(idx_gpu, w_gpu, idx_ref, w_ref):
+    """Top-k (and top-p) routing: indices bit-exact (-1 = dropped by top-p), weights
+    within W_RTOL relative where kept and exactly zero where dropped."""
+    assert np.array_equal(idx_gpu, idx_ref), "topk_idx differs"
+    kept = idx_ref >= 0
+    assert np.all(w_gpu[~kept] == 0)
+    rel = np.abs(w_gpu[kept].astype(np.float64) - w_ref[kept]) / np.abs(w_ref[kept])
+    assert rel.max() <= W_RTOL, f"topk_w relative error {rel.max():.3g}"
 
 
 def check_weights(w_gpu: np.ndarray, w_ref: np.ndarray):

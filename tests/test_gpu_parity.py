@@ -7,7 +7,7 @@ import torch
 import oracle
 import synth
 import w4a16_quantized_expert_b200 as moe
-from gpu_cases import Case, check_weights, check_y, y_to_f64
+from gpu_cases import Case, check_routing, check_weights, check_y, y_to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -73,9 +73,40 @@ def test_route_logits_batches(name, T):
     check_weights(w.cpu().numpy(), r_w.astype(np.float64))
 
 
+# ------------------------------------------------------------------ adaptive top-p
+@pytest.mark.parametrize("name,T,p", [("tiny", 4, 0.5), ("tiny", 37, 0.5), ("decode8", 8, 0.7),
+                                      ("nvfp4_16", 16, 0.7)])
+def test_route_topp_bitexact_from_oracle_logits(name, T, p):
+    """Fed the oracle's fp32 logits, the GPU's top-p routing (kept experts, their order,
+    the -1 tail) is the oracle's, weights within 1e-6."""
+    w = W[name].with_(top_p=p)
+    case = Case(w, T=T, experts=[0])
+    ref = case.oracle_forward()
+    ws = case.dev.workspace(T)
+    li = torch.from_numpy(ref["logits"]).cuda()
+    idx, wt, _ = case.dev.route(None, T, ws, logits_in=li, want_logits=True)
+    torch.cuda.synchronize()
+    check_routing(idx.cpu().numpy(), wt.cpu().numpy(), ref["topk_idx"], ref["topk_w"].astype(np.float64))
+    assert (ref["topk_idx"] == -1).any(), "the case drops some experts"
+
+
+@pytest.mark.parametrize("name,T,p", [("tiny", 4, 0.5), ("tiny", 37, 0.5), ("decode1", 1, 0.7),
+                                      ("decode8", 8, 0.7), ("nvfp4_16", 16, 0.7)])
+def test_forward_topp(name, T, p):
+    """The whole layer with adaptive top-p against the oracle (tokens near a top-k or a
+    top-p decision excluded, as for plain top-k)."""
+    w = W[name].with_(top_p=p)
+    case = Case(w, T=T, experts="routed") if name != "tiny" else Case(w, T=T, max_tokens=64)
+    y, _ = _forward(case)
+    ref = case.oracle_forward()
+    excluded, err = check_y(y_to_f64(y), ref["y"], ref["gap"])
+    print(f"{name} top-p {p}: excluded {excluded}/{T}, kept {(ref['topk_idx'] >= 0).sum()}/{ref['topk_idx'].size}, rel err {err:.3g}")
+
+
 # ------------------------------------------------------------------ grouping
 @pytest.mark.parametrize("T,k,E,mode", [(4, 2, 16, "rand"), (1, 8, 256, "rand"), (16, 8, 256, "rand"),
-                                        (512, 8, 256, "rand"), (40, 4, 16, "hot"), (9, 3, 1024, "rand")])
+                                        (512, 8, 256, "rand"), (40, 4, 16, "hot"), (9, 3, 1024, "rand"),
+                                        (16, 8, 256, "drop"), (300, 8, 256, "drop")])
 def test_group_bitexact(T, k, E, mode):
     rng = np.random.default_rng(T * 1000 + E)
     if mode == "hot":
@@ -83,6 +114,9 @@ def test_group_bitexact(T, k, E, mode):
                         for _ in range(T)]).astype(np.int32)
     else:
         idx = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    if mode == "drop":   # top-p tails: entries past a random count per token are -1
+        for t in range(T):
+            idx[t, int(rng.integers(1, k + 1)):] = -1
     w = synth.WORKLOADS["tiny"].with_(E=E, k=k)
     host = {"Wr": np.zeros((E, 256), np.float32), "bias": np.zeros(E, np.float32)}
     host.update(synth.make_experts(w, experts=[]))
@@ -93,7 +127,7 @@ def test_group_bitexact(T, k, E, mode):
     c_ref, o_ref, p_ref, u_ref = oracle.default().group(idx, E)
     assert np.array_equal(counts.cpu().numpy(), c_ref)
     assert np.array_equal(offsets.cpu().numpy(), o_ref)
-    assert np.array_equal(perm.cpu().numpy()[: T * k], p_ref)
+    assert np.array_equal(perm.cpu().numpy()[: len(p_ref)], p_ref)
     n = int(nu.item())
     assert n == len(u_ref) and np.array_equal(unique.cpu().numpy()[:n], u_ref)
     assert moe.moe_get_device_status(dev.handle) == moe.MOE_OK

@@ -33,7 +33,8 @@ c_size = ctypes.c_size_t
 class moe_layer_desc(ctypes.Structure):
     _fields_ = [("hidden", c_int), ("inter", c_int), ("inter_shared", c_int),
                 ("n_experts", c_int), ("top_k", c_int), ("n_shared", c_int),
-                ("routed_scaling", ctypes.c_float), ("format", c_int), ("max_tokens", c_int)]
+                ("routed_scaling", ctypes.c_float), ("format", c_int), ("max_tokens", c_int),
+                ("top_p", ctypes.c_float)]
 
 
 WEIGHT_FIELDS = ["router_w", "router_bias", "gate", "up", "down",

@@ -150,6 +150,7 @@ int validate_desc(const moe_layer_desc *d)
     if (d->top_k < 1 || d->top_k > kMaxTopK || d->top_k > d->n_experts) return MOE_ERR_INVALID_ARG;
     if (d->max_tokens < 1 || d->max_tokens > 65536) return MOE_ERR_INVALID_ARG;
     if (!(d->routed_scaling == d->routed_scaling)) return MOE_ERR_INVALID_ARG;   // NaN
+    if (!(d->top_p >= 0.f)) return MOE_ERR_INVALID_ARG;                          // negative or NaN
     return MOE_OK;
 }
 
@@ -228,6 +229,7 @@ RouterParams router_params(const moe_layer *L, const uint16_t *x, int T, void *w
     p.E = L->desc.n_experts;
     p.k = L->desc.top_k;
     p.scaling = L->desc.routed_scaling;
+    p.top_p = (L->desc.top_p > 0.f && L->desc.top_p < 1.f) ? L->desc.top_p : 0.f;
     return p;
 }
 
@@ -524,6 +526,7 @@ int moe_route_static(const moe_layer *L, const uint16_t *x, int T, const float *
     p.E = E;
     p.k = L->desc.top_k;
     p.scaling = L->desc.routed_scaling;
+    p.top_p = (L->desc.top_p > 0.f && L->desc.top_p < 1.f) ? L->desc.top_p : 0.f;
     p.do_gemv = logits_in ? 0 : 1;
     p.do_group = 0;
     return cuda_status(launch_router(p, false, reinterpret_cast<cudaStream_t>(stream)));

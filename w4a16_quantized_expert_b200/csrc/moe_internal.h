@@ -69,6 +69,7 @@ struct RouterParams {
     int *status;
     int T, H, E, k;
     float scaling;
+    float top_p;             // adaptive expert top-p in (0, 1), 0 = off
     int do_gemv, do_group;
     int x_rows, x_bufs;      // GEMV: token rows per shared-memory x buffer, buffers (1 or 2)
 };

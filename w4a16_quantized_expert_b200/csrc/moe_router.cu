@@ -49,7 +49,7 @@ __device__ __forceinline__ unsigned float_key(float v)
 // min of the expert indices holding that max (equal scores -> lower expert index).
 template <int kPer>
 __device__ void topk_token_t(const float *sel_row, const float *score_row, int E, int k, float scaling,
-                             int32_t *idx_out, float *w_out, int *idx_smem)
+                             float top_p, int32_t *idx_out, float *w_out, int *idx_smem)
 {
     const int lane = threadIdx.x & 31;
     // selection keys and the unbiased scores, loaded together (one round trip)
@@ -92,6 +92,44 @@ __device__ void topk_token_t(const float *sel_row, const float *score_row, int E
     if (lane < k) s_mine = static_cast<double>(my_score);
     double sum = 0.0;
     for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, s_mine, j);
+    if (top_p > 0.f) {
+        // adaptive expert top-p: rank of this lane's expert among the k by score (equal
+        // scores: lower expert index first); the score mass ranked ahead of it, summed in
+        // rank order; kept while that mass is below top_p of the k's mass
+        int rank = 0;
+        for (int i = 0; i < k; ++i) {
+            const float si = __shfl_sync(0xffffffffu, my_score, i);
+            const int ei = __shfl_sync(0xffffffffu, my_idx, i);
+            if (lane < k && (si > my_score || (si == my_score && ei < my_idx))) ++rank;
+        }
+        double before = 0.0;
+        for (int r = 0; r < k; ++r) {
+            const unsigned who = __ballot_sync(0xffffffffu, lane < k && rank == r);
+            const double v = __shfl_sync(0xffffffffu, s_mine, __ffs(who) - 1);
+            if (r < rank) before += v;
+        }
+        const bool keep = lane < k && before < static_cast<double>(top_p) * sum;
+        const unsigned kept = __ballot_sync(0xffffffffu, keep);
+        // kept experts first, in top-k order, weights renormalised over them
+        double sum2 = 0.0;
+        for (int j = 0; j < k; ++j) {
+            const double v = __shfl_sync(0xffffffffu, s_mine, j);
+            if (kept >> j & 1u) sum2 += v;
+        }
+        const int pos = __popc(kept & ((1u << lane) - 1u)), m = __popc(kept);
+        if (keep) {
+            idx_smem[pos] = my_idx;
+            idx_out[pos] = my_idx;
+            w_out[pos] = static_cast<float>(static_cast<double>(scaling) * (s_mine / sum2));
+        }
+        __syncwarp();
+        if (lane < k && lane >= m) {
+            idx_smem[lane] = -1;
+            idx_out[lane] = -1;
+            w_out[lane] = 0.f;
+        }
+        return;
+    }
     if (lane < k) {
         idx_smem[lane] = my_idx;
         idx_out[lane] = my_idx;
@@ -100,10 +138,10 @@ __device__ void topk_token_t(const float *sel_row, const float *score_row, int E
 }
 
 __device__ void topk_token(const float *sel_row, const float *score_row, int E, int k, float scaling,
-                           int32_t *idx_out, float *w_out, int *idx_smem)
+                           float top_p, int32_t *idx_out, float *w_out, int *idx_smem)
 {
-    if (E <= 256) topk_token_t<8>(sel_row, score_row, E, k, scaling, idx_out, w_out, idx_smem);
-    else topk_token_t<kMaxExperts / 32>(sel_row, score_row, E, k, scaling, idx_out, w_out, idx_smem);
+    if (E <= 256) topk_token_t<8>(sel_row, score_row, E, k, scaling, top_p, idx_out, w_out, idx_smem);
+    else topk_token_t<kMaxExperts / 32>(sel_row, score_row, E, k, scaling, top_p, idx_out, w_out, idx_smem);
 }
 
 // ---------------------------------------------------------------------------- grouping
@@ -119,7 +157,7 @@ __device__ void group_warp(const int32_t *topk_idx, bool src_smem, int n, int E,
     for (int base = 0; base < n; base += 32) {
         const int a = base + lane;
         int e = (a < n) ? (src_smem ? topk_idx[a] : __ldcg(topk_idx + a)) : -1;
-        if (a < n && (e < 0 || e >= E)) {
+        if (a < n && (e < -1 || e >= E)) {   // -1: dropped by top-p, no expert
             record_error(status, MOE_ERR_DEVICE_BOUNDS);
             e = -1;
         }
@@ -202,17 +240,20 @@ __device__ void group_block(const int *s_idx, int n, int E, int32_t *counts, int
     __shared__ int s_nu;
     int rk[kPer], ee[kPer], lt[kPer], eq[kPer];
     bool fi[kPer];
+    int nk = 0;   // assignments that reach an expert (top-p drops are -1)
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
         const int a = tid + u * kRouterThreads;
         fi[u] = false;
-        if (a < n) {
+        if (u == 0)
+            for (int b = 0; b < n; ++b) nk += s_idx[b] >= 0;
+        if (a < n && s_idx[a] >= 0) {
             const int e = s_idx[a];
-            if (e < 0 || e >= E) record_error(status, MOE_ERR_DEVICE_BOUNDS);
+            if (e >= E) record_error(status, MOE_ERR_DEVICE_BOUNDS);
             int l = 0, q = 0, qb = 0;
             for (int b = 0; b < n; ++b) {
                 const int e2 = s_idx[b];
-                l += e2 < e;
+                l += (e2 >= 0) & (e2 < e);
                 q += e2 == e;
                 qb += (e2 == e) & (b < a);
             }
@@ -236,14 +277,14 @@ __device__ void group_block(const int *s_idx, int n, int E, int32_t *counts, int
             s_uniq[si] = ee[u];
             s_uoff[si] = lt[u];
             s_ucnt[si] = eq[u];
-            if (lt[u] + eq[u] == n) s_nu = si + 1;   // the last expert's slot
+            if (lt[u] + eq[u] == nk) s_nu = si + 1;   // the last expert's slot
         }
     }
     __syncthreads();
     const int nu = s_nu;
     if (tid == 0) {
         *n_unique = nu;
-        offsets[E] = n;
+        offsets[E] = nk;
     }
     for (int e = tid; e < E; e += kRouterThreads) {
         int lo = 0, hi = nu;   // first slot whose expert is >= e
@@ -254,7 +295,7 @@ __device__ void group_block(const int *s_idx, int n, int E, int32_t *counts, int
         }
         const bool has = lo < nu && s_uniq[lo] == e;
         counts[e] = has ? s_ucnt[lo] : 0;
-        offsets[e] = lo < nu ? s_uoff[lo] : n;
+        offsets[e] = lo < nu ? s_uoff[lo] : nk;
     }
 }
 
@@ -431,7 +472,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p)
     }
 
     for (int t = warp; t < nt; t += kRouterThreads / 32)
-        topk_token(p.sel + (size_t)(t0 + t) * p.E, p.score + (size_t)(t0 + t) * p.E, p.E, p.k, p.scaling,
+        topk_token(p.sel + (size_t)(t0 + t) * p.E, p.score + (size_t)(t0 + t) * p.E, p.E, p.k, p.scaling, p.top_p,
                    p.topk_idx + (size_t)(t0 + t) * p.k, p.topk_w + (size_t)(t0 + t) * p.k, s_idx + t * p.k);
     if (!p.do_group) return;
     __syncthreads();
@@ -483,7 +524,7 @@ __device__ void group_warps8(const int32_t *idx, bool src_smem, int n, int E, in
     for (int base = a0; base < a1; base += 32) {
         const int a = base + lane;
         int e = (a < a1) ? (src_smem ? idx[a] : __ldcg(idx + a)) : -1;
-        if (a < a1 && (e < 0 || e >= E)) {
+        if (a < a1 && (e < -1 || e >= E)) {   // -1: dropped by top-p, no expert
             record_error(status, MOE_ERR_DEVICE_BOUNDS);
             e = -1;
         }
@@ -741,7 +782,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_tile_kernel(RouterParam
     __syncthreads();
     if (!s_flag) return;
     for (int t = warp; t < nt; t += kRouterThreads / 32)
-        topk_token(p.sel + (size_t)(t0 + t) * p.E, p.score + (size_t)(t0 + t) * p.E, p.E, p.k, p.scaling,
+        topk_token(p.sel + (size_t)(t0 + t) * p.E, p.score + (size_t)(t0 + t) * p.E, p.E, p.k, p.scaling, p.top_p,
                    p.topk_idx + (size_t)(t0 + t) * p.k, p.topk_w + (size_t)(t0 + t) * p.k, s_idx + t * p.k);
     if (!p.do_group) return;
     // the last token tile groups the whole batch
@@ -776,8 +817,10 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p)
     if (i >= (size_t)p.T * p.H) return;
     const int t = static_cast<int>(i / p.H), m = static_cast<int>(i % p.H);
     float acc = p.n_shared ? p.y_shared[i] : 0.f;
-    for (int j = 0; j < p.k; ++j)
-        acc = fmaf(p.topk_w[(size_t)t * p.k + j], p.y_assign[((size_t)t * p.k + j) * p.H + m], acc);
+    for (int j = 0; j < p.k; ++j) {
+        const float w = p.topk_w[(size_t)t * p.k + j];
+        if (w != 0.f) acc = fmaf(w, p.y_assign[((size_t)t * p.k + j) * p.H + m], acc);   // 0: dropped by top-p
+    }
     p.y[i] = __half_as_ushort(__float2half_rn(acc));
 }
 

@@ -28,7 +28,7 @@ _FIELD = {
 def make_desc(d: dict, max_tokens: int) -> moe_layer_desc:
     return moe_layer_desc(hidden=d["H"], inter=d["I"], inter_shared=d["I_sh"], n_experts=d["E"],
                           top_k=d["k"], n_shared=d["n_shared"], routed_scaling=d["scaling"],
-                          format=d["fmt"], max_tokens=max_tokens)
+                          format=d["fmt"], max_tokens=max_tokens, top_p=float(d.get("top_p", 0.0)))
 
 
 def _to_device(a, device) -> torch.Tensor:
