@@ -57,9 +57,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"
 # DRAM traffic per launch (bytes) of the dominant kernel from an ncu capture, keyed by
 # workload; valid only while the kernel source hashes to the recorded value.
 NCU_TRAFFIC = {
-    # profiles/ffn_kernel_int4_decode1_e32_full.md: dram read 113,488,896 + write 3,098,368
+    # profiles/ffn_kernel_int4_decode1_e32_full.md: dram read 113,490,176 + write 3,437,824
     # bytes per gate/up launch (a T=1 step reads the same 9 experts at E=32 as at E=256)
-    "decode1": {"kernel": "gate_up", "bytes": 116587264, "kernel_hash": "7e57ff3a7fa57187"},
+    "decode1": {"kernel": "gate_up", "bytes": 116928000, "kernel_hash": "199024cc2aaa083e"},
 }
 
 
