@@ -72,7 +72,7 @@ def _create(desc, w):
     dict(n_experts=0), dict(n_experts=1025), dict(top_k=0), dict(top_k=33),
     dict(top_k=17), dict(n_shared=2), dict(inter_shared=50), dict(max_tokens=0),
     dict(max_tokens=70000), dict(format=7), dict(routed_scaling=float("nan")),
-    dict(format=1, hidden=320), dict(format=1, inter=128),
+    dict(format=1, hidden=320), dict(format=1, inter=128), dict(top_p=-0.1), dict(top_p=float("nan")),
 ])
 def test_create_rejects_bad_shapes(bad):
     rc, h = _create(_desc(**bad), _weights())
@@ -112,6 +112,32 @@ def test_null_handle_and_out_of_range_T():
     assert L.moe_layer_destroy(None) == moe.MOE_OK
     st = ctypes.c_int(0)
     assert L.moe_get_device_status(None, ctypes.byref(st)) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The ctypes mirrors of moe_layer_desc and moe_weights have the C header's sizes and
+    field offsets (compiled with the host C compiler)."""
+    import shutil
+    import subprocess
+    if not shutil.which("gcc"):
+        pytest.skip("no host C compiler")
+    fields = [f for f, _ in moe.moe_layer_desc._fields_]
+    wfields = [f for f, _ in moe.moe_weights._fields_]
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "moe.h"', "int main(void) {",
+             '  printf("%zu %zu\\n", sizeof(moe_layer_desc), sizeof(moe_weights));']
+    lines += [f'  printf("%zu\\n", offsetof(moe_layer_desc, {f}));' for f in fields]
+    lines += [f'  printf("%zu\\n", offsetof(moe_weights, {f}));' for f in wfields]
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    out = subprocess.check_output([str(exe)], text=True).split()
+    sizes, offs = [int(v) for v in out[:2]], [int(v) for v in out[2:]]
+    assert sizes == [ctypes.sizeof(moe.moe_layer_desc), ctypes.sizeof(moe.moe_weights)]
+    py = [getattr(moe.moe_layer_desc, f).offset for f in fields] + \
+         [getattr(moe.moe_weights, f).offset for f in wfields]
+    assert offs == py
 
 
 def test_product_path_has_no_oracle_or_fallback():
