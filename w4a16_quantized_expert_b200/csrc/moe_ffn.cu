@@ -1469,14 +1469,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
                 const int kvals = min(128, it.K - 128 * u);   // a multiple of 64
                 const int bslot = gs % NB;
                 if (lane == 0) {
-                    const uint32_t bbase = smem_u32(bring + (size_t)bslot * kTcBSlot);
+                    // The issuing thread's own instructions between MMAs add to every MMA's
+                    // cost (measured), so the operands are formed once per half: the B
+                    // descriptor advances 32 bytes (2 in its 16-byte address field) per step.
+                    const uint64_t db0 = umma_sdesc(smem_u32(bring + (size_t)bslot * kTcBSlot));
                     const uint32_t abase = tmem + C::kACol0 + sub * C::kACols;
-                    for (int kk = 0; kk < kvals / 32; ++kk) {
-                        const uint64_t db = umma_sdesc(bbase + 32 * kk);
+                    const uint32_t dbase = tmem + buf * C::kAccCols;
+                    const uint32_t acc0 = u > 0 ? 1u : 0u;
+                    if (kvals == 128) {
 #pragma unroll
-                        for (int m = 0; m < C::kMats; ++m)
-                            umma_s8_ta(tmem + buf * C::kAccCols + m * kTcNMax, abase + m * 32 + 8 * kk, db, idesc,
-                                       (u > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                            for (int m = 0; m < C::kMats; ++m)
+                                umma_s8_ta(dbase + m * kTcNMax, abase + m * 32 + 8 * kk, db0 + 2 * kk, idesc,
+                                           kk > 0 ? 1u : acc0);
+                    } else {
+                        for (int kk = 0; kk < kvals / 32; ++kk)
+#pragma unroll
+                            for (int m = 0; m < C::kMats; ++m)
+                                umma_s8_ta(dbase + m * kTcNMax, abase + m * 32 + 8 * kk, db0 + 2 * kk, idesc,
+                                           kk > 0 ? 1u : acc0);
                     }
                     umma_commit(&sb_empty[sub]);   // the half and the B slot are free once
                     umma_commit(&b_empty[bslot]);  // these MMAs have read them
