@@ -1200,9 +1200,12 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
 // ring of shared-memory B slots (asynchronous 16-byte copies, in the 128-byte-swizzled
 // K-major layout, several halves ahead); 10..13 read an item's accumulators from TMEM
 // once they are complete (warp w owns TMEM lanes 32 (w % 4) ..) and run the epilogue.
-// Keeping the expanded weights out of shared memory leaves it two passes of a quarter
-// of the traffic (the TMA write and the read of the packed codes) plus the B slots.
-// Accumulators are double-buffered in TMEM, so the next item's MMAs overlap an epilogue.
+// With the expanded weights in TMEM, shared memory carries only the packed codes (one
+// TMA write, one read: a quarter of the bytes an expanded s8 tile would move twice) and
+// the B slots.  Accumulators are double-buffered in TMEM, so the next item's MMAs overlap
+// an epilogue.  One tcgen05.mma of this shape costs about the same for any N up to 256
+// and the issuing thread's own instructions add to it, so with ~16-18 tokens per expert
+// the kernel is bound by MMA issue, not by MACs.
 
 constexpr int kTcRows = 128;                    // output rows per item (MMA M)
 constexpr int kTcTok = 32;                      // tokens per item
@@ -1264,14 +1267,7 @@ __device__ __forceinline__ uint32_t umma_idesc_s8(int n)
     return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kTcRows >> 4) << 24);
 }
 
-__device__ __forceinline__ void umma_s8(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-                 "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
-}
-
-// the same with the A operand in tensor memory
+// tcgen05.mma kind::i8 (s8 x s8 -> s32), one CTA, A operand in tensor memory, B by descriptor
 __device__ __forceinline__ void umma_s8_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
                                            uint32_t accumulate)
 {
