@@ -573,7 +573,7 @@ def run_ours(args, w):
             "d2h_bytes_per_step": w.T * w.H * 2,
             "how": "moe_forward_host (pinned host x in, y out) captured in CUDA graphs",
         },
-        "gpu_launches": 3 * K,
+        "gpu_launches": 4 * K,   # per layer call: router, gate/up, down, combine
         "clocks": cl,
         "cpu_baseline": cpu,
     }
