@@ -22,7 +22,8 @@ SO = os.path.join(_HERE, "liboracle.so")
 CFLAGS = ["-O2", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
           "-std=c11"]
 
-INT4, NVFP4 = 0, 1
+INT4, NVFP4, INT8, INT2 = 0, 1, 2, 3
+_CODES_PER_BYTE = {INT4: 2, NVFP4: 2, INT8: 1, INT2: 4}
 
 
 def compile_oracle(src: str = SRC, out: str = SO, include_dir: str = _HERE) -> str:
@@ -85,8 +86,11 @@ class Oracle:
         L = ctypes.CDLL(path)
         L.orc_half_to_double.argtypes = [ctypes.c_uint16]
         L.orc_half_to_double.restype = ctypes.c_double
-        L.orc_int4_at.argtypes = [vp, ctypes.c_long]
-        L.orc_int4_at.restype = ctypes.c_int
+        for f in ("orc_int4_at", "orc_int8_at", "orc_int2_at"):
+            getattr(L, f).argtypes = [vp, ctypes.c_long]
+            getattr(L, f).restype = ctypes.c_int
+        L.orc_quantize_rows.argtypes = [vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp]
+        L.orc_quantize_rows.restype = None
         L.orc_e2m1_to_double.argtypes = [ctypes.c_uint]
         L.orc_e2m1_to_double.restype = ctypes.c_double
         L.orc_e4m3_to_double.argtypes = [ctypes.c_uint8]
@@ -121,6 +125,24 @@ class Oracle:
     def int4_row(self, row_bytes: np.ndarray, K: int) -> np.ndarray:
         row = np.ascontiguousarray(row_bytes, dtype=np.uint8)
         return np.array([self.lib.orc_int4_at(_p(row), k) for k in range(K)], dtype=np.int64)
+
+    def int8_row(self, row_bytes: np.ndarray, K: int) -> np.ndarray:
+        row = np.ascontiguousarray(row_bytes, dtype=np.uint8)
+        return np.array([self.lib.orc_int8_at(_p(row), k) for k in range(K)], dtype=np.int64)
+
+    def int2_row(self, row_bytes: np.ndarray, K: int) -> np.ndarray:
+        row = np.ascontiguousarray(row_bytes, dtype=np.uint8)
+        return np.array([self.lib.orc_int2_at(_p(row), k) for k in range(K)], dtype=np.int64)
+
+    def quantize(self, w: np.ndarray, bits: int):
+        """Per-row symmetric quantisation of fp32 rows [N][K] to bits = 8, 4 or 2.
+        Returns (codes [N][K * bits / 8] uint8, row scales [N] fp32)."""
+        w = np.ascontiguousarray(w, np.float32)
+        N, K = w.shape
+        codes = np.empty((N, K * bits // 8), np.uint8)
+        scale = np.empty(N, np.float32)
+        self.lib.orc_quantize_rows(_p(w), N, K, bits, _p(codes), _p(scale))
+        return codes, scale
 
     def e2m1(self, code: int) -> float:
         return self.lib.orc_e2m1_to_double(code)
@@ -194,9 +216,9 @@ class Oracle:
         keep = []
         codes = np.ascontiguousarray(M["codes"], np.uint8)
         keep.append(codes)
-        N, Kh = codes.shape
-        m = OrcMatrix(format=M["format"], N=N, K=2 * Kh, codes=_p(codes))
-        if M["format"] == INT4:
+        N, Kb = codes.shape
+        m = OrcMatrix(format=M["format"], N=N, K=_CODES_PER_BYTE[M["format"]] * Kb, codes=_p(codes))
+        if M["format"] != NVFP4:
             rs = np.ascontiguousarray(M["row_scale"], np.float32)
             keep.append(rs)
             m.row_scale = _p(rs)

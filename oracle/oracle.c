@@ -42,6 +42,14 @@
  *    sums in ascending index order.
  *  - combine: y_t = shared(x_t) + sum_{j=0..k-1} w_tj * y_{e_tj}(x_t), the shared
  *    expert with weight 1.
+ *  - int8 and int2 codes with one scale per output row (hakusoku page, section
+ *    "実装済み機能": int8/int4/int2 kernels with per-row scales).  Readings: int8 is one
+ *    two's-complement byte per weight; int2 packs four two's-complement codes in
+ *    [-2, 1] per byte, element 4b+i in bits 2i..2i+1 (the int4 order continued).
+ *  - per-row quantisation (hakusoku page, section "実装済み機能": the offline FP8 -> int4
+ *    conversion tool).  Reading: symmetric, scale = max|w| / (2^(bits-1) - 1) rounded
+ *    to fp32, code = round-half-even(w / scale) with that fp32 scale, clamped to the
+ *    code range; an all-zero row gets scale 0 and zero codes.
  *  - adaptive expert top-p (hakusoku page, section "実行・チューニングパラメータ":
  *    the --topp option, which names the idea and its effect but not the rule).
  *    Reading: after top-k, order the k chosen experts by their score s (descending,
@@ -79,6 +87,19 @@ int orc_int4_at(const uint8_t *row, long k)
     return n >= 8 ? n - 16 : n;
 }
 
+int orc_int8_at(const uint8_t *row, long k)
+{
+    int n = row[k];
+    return n >= 128 ? n - 256 : n;
+}
+
+int orc_int2_at(const uint8_t *row, long k)
+{
+    unsigned b = row[k >> 2];
+    int n = (int)((b >> (2 * (k & 3))) & 3u);
+    return n >= 2 ? n - 4 : n;
+}
+
 double orc_e2m1_to_double(unsigned code)
 {
     int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
@@ -95,12 +116,22 @@ double orc_e4m3_to_double(uint8_t b)
     return s ? -v : v;
 }
 
+/* bytes of one row of K codes */
+static size_t row_bytes(int format, long K)
+{
+    return format == ORC_INT8 ? (size_t)K : format == ORC_INT2 ? (size_t)(K / 4) : (size_t)(K / 2);
+}
+
 /* dequantised weight (row n, column k) of one matrix */
 static double wq(const orc_matrix *M, long n, long k)
 {
-    const uint8_t *row = M->codes + (size_t)n * (size_t)(M->K / 2);
+    const uint8_t *row = M->codes + (size_t)n * row_bytes(M->format, M->K);
     if (M->format == ORC_INT4) {
         return (double)orc_int4_at(row, k) * (double)M->row_scale[n];
+    } else if (M->format == ORC_INT8) {
+        return (double)orc_int8_at(row, k) * (double)M->row_scale[n];
+    } else if (M->format == ORC_INT2) {
+        return (double)orc_int2_at(row, k) * (double)M->row_scale[n];
     } else {
         unsigned b = row[k >> 1];
         unsigned c = (k & 1) ? (b >> 4) : (b & 15);
@@ -114,6 +145,38 @@ void orc_dequant_matrix(const orc_matrix *M, double *out)
 {
     for (long n = 0; n < M->N; n++)
         for (long k = 0; k < M->K; k++) out[(size_t)n * (size_t)M->K + (size_t)k] = wq(M, n, k);
+}
+
+/* ------------------------------------------------------------ quantisation */
+
+void orc_quantize_rows(const float *w, int N, int K, int bits, uint8_t *codes, float *scale)
+{
+    int qmax = (1 << (bits - 1)) - 1, qmin = -(1 << (bits - 1));
+    size_t rb = row_bytes(bits == 8 ? ORC_INT8 : bits == 2 ? ORC_INT2 : ORC_INT4, K);
+    memset(codes, 0, rb * (size_t)N);
+    for (int n = 0; n < N; n++) {
+        double amax = 0.0;
+        for (int k = 0; k < K; k++) {
+            double a = fabs((double)w[(size_t)n * K + k]);
+            if (a > amax) amax = a;
+        }
+        float sc = (float)(amax / qmax);
+        scale[n] = sc;
+        uint8_t *row = codes + (size_t)n * rb;
+        for (int k = 0; k < K; k++) {
+            int q = 0;
+            if (sc > 0.0f) {
+                double v = rint((double)w[(size_t)n * K + k] / (double)sc);   /* ties to even */
+                if (v > qmax) v = qmax;
+                if (v < qmin) v = qmin;
+                q = (int)v;
+            }
+            unsigned u = (unsigned)q;
+            if (bits == 8) row[k] = (uint8_t)(u & 255u);
+            else if (bits == 4) row[k >> 1] |= (uint8_t)((u & 15u) << (4 * (k & 1)));
+            else row[k >> 2] |= (uint8_t)((u & 3u) << (2 * (k & 3)));
+        }
+    }
 }
 
 /* ------------------------------------------------------------------ router */
@@ -298,8 +361,8 @@ static orc_matrix routed_matrix(const orc_layer *L, int which, int e)
     M.N = rows;
     M.K = K;
     const uint8_t *codes = which == 0 ? L->g : which == 1 ? L->u : L->d;
-    M.codes = codes + (size_t)e * (size_t)rows * (size_t)(K / 2);
-    if (L->format == ORC_INT4) {
+    M.codes = codes + (size_t)e * (size_t)rows * row_bytes(L->format, K);
+    if (L->format != ORC_NVFP4) {   /* row-scaled integer codes */
         const float *sc = which == 0 ? L->sg : which == 1 ? L->su : L->sd;
         M.row_scale = sc + (size_t)e * (size_t)rows;
     } else {
@@ -319,7 +382,7 @@ static orc_matrix shared_matrix(const orc_layer *L, int which)
     M.N = which == 2 ? L->H : L->I_sh;
     M.K = which == 2 ? L->I_sh : L->H;
     M.codes = which == 0 ? L->sh_g : which == 1 ? L->sh_u : L->sh_d;
-    if (L->format == ORC_INT4) {
+    if (L->format != ORC_NVFP4) {   /* row-scaled integer codes */
         M.row_scale = which == 0 ? L->sh_sg : which == 1 ? L->sh_su : L->sh_sd;
     } else {
         M.block_scale = which == 0 ? L->sh_bg : which == 1 ? L->sh_bu : L->sh_bd;

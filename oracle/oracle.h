@@ -18,12 +18,14 @@
 
 #define ORC_INT4 0
 #define ORC_NVFP4 1
+#define ORC_INT8 2   /* one two's-complement byte per weight, one fp32 scale per row */
+#define ORC_INT2 3   /* four 2-bit two's-complement codes per byte (element 4b+i in bits 2i..2i+1) */
 
 typedef struct {
-    int format;                 /* ORC_INT4 or ORC_NVFP4 */
+    int format;                 /* ORC_INT4, ORC_NVFP4, ORC_INT8 or ORC_INT2 */
     int N, K;                   /* output rows, inputs per row */
-    const uint8_t *codes;       /* [N][K/2] */
-    const float *row_scale;     /* int4: [N] */
+    const uint8_t *codes;       /* [N][K/2] (int4, NVFP4), [N][K] (int8), [N][K/4] (int2) */
+    const float *row_scale;     /* int4, int8, int2: [N] */
     const uint8_t *block_scale; /* NVFP4: [N][K/16] E4M3 */
     float tensor_scale;         /* NVFP4 */
 } orc_matrix;
@@ -64,6 +66,11 @@ typedef struct {
 
 double orc_half_to_double(uint16_t h);
 int orc_int4_at(const uint8_t *row, long k);
+int orc_int8_at(const uint8_t *row, long k);
+int orc_int2_at(const uint8_t *row, long k);
+/* Per-row symmetric quantisation of fp32 rows [N][K] to bits = 8, 4 or 2 two's-complement
+ * codes, packed as the decoders read them, with one fp32 scale per row (see oracle.c). */
+void orc_quantize_rows(const float *w, int N, int K, int bits, uint8_t *codes, float *scale);
 double orc_e2m1_to_double(unsigned code);
 double orc_e4m3_to_double(uint8_t b);
 float orc_sigmoid_f32(float logit);

@@ -48,6 +48,23 @@ def np_dequant_int4(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
     return q.astype(np.float64) * scale.astype(np.float64)[:, None]
 
 
+def np_dequant_int8(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """numpy reading of int8 codes (one two's-complement byte per weight)."""
+    return codes.view(np.int8).astype(np.float64) * scale.astype(np.float64)[:, None]
+
+
+def np_dequant_int2(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """numpy unpacking of int2 codes (four per byte, element 4b+i in bits 2i..2i+1)."""
+    q = np.stack([(codes >> (2 * i)) & 3 for i in range(4)], axis=-1).astype(np.int64)
+    q = q.reshape(codes.shape[0], -1)
+    q = np.where(q >= 2, q - 4, q)
+    return q.astype(np.float64) * scale.astype(np.float64)[:, None]
+
+
+NP_DEQUANT_ROWSCALED = {0: np_dequant_int4, 2: np_dequant_int8, 3: np_dequant_int2}
+BYTES_PER_CODE = {0: 0.5, 1: 0.5, 2: 1.0, 3: 0.25}
+
+
 def _e2m1_table():
     return np.array([float(r.split()[1]) for r in _rows("e2m1_ocp.txt")], np.float64)
 
@@ -72,9 +89,9 @@ def small_layer(E=1, k=1, n_shared=0, H=64, I=32, I_sh=32, fmt=0, scaling=1.0, s
     L = {"Wr": (rng.standard_normal((E, H)) / math.sqrt(H)).astype(np.float32),
          "bias": rng.uniform(-0.1, 0.1, E).astype(np.float32)}
     def mat(rows, K):
-        codes = rng.integers(0, 256, (rows, K // 2), dtype=np.uint8)
-        if fmt == 0:
-            return codes, rng.uniform(0.01, 0.03, rows).astype(np.float32)
+        codes = rng.integers(0, 256, (rows, int(K * BYTES_PER_CODE[fmt])), dtype=np.uint8)
+        if fmt != 1:   # row-scaled integer codes
+            return codes, rng.uniform(0.01, 0.03, rows).astype(np.float32) * (0.0625 if fmt == 2 else 1.0)
         # E4M3 block scales from a small range of normal values (exponent 5..8, any mantissa)
         bs = (rng.integers(5, 9, (rows, K // 16)) << 3 | rng.integers(0, 8, (rows, K // 16)))
         return codes, bs.astype(np.uint8)
@@ -83,7 +100,7 @@ def small_layer(E=1, k=1, n_shared=0, H=64, I=32, I_sh=32, fmt=0, scaling=1.0, s
     d = [mat(H, I) for _ in range(E)]
     L["g"] = np.stack([m[0] for m in g]); L["u"] = np.stack([m[0] for m in u])
     L["d"] = np.stack([m[0] for m in d])
-    if fmt == 0:
+    if fmt != 1:
         L["sg"] = np.stack([m[1] for m in g]); L["su"] = np.stack([m[1] for m in u])
         L["sd"] = np.stack([m[1] for m in d])
     else:
@@ -95,7 +112,7 @@ def small_layer(E=1, k=1, n_shared=0, H=64, I=32, I_sh=32, fmt=0, scaling=1.0, s
     if n_shared:
         gs, us, ds = mat(I_sh, H), mat(I_sh, H), mat(H, I_sh)
         L["sh_g"], L["sh_u"], L["sh_d"] = gs[0], us[0], ds[0]
-        if fmt == 0:
+        if fmt != 1:
             L["sh_sg"], L["sh_su"], L["sh_sd"] = gs[1], us[1], ds[1]
         else:
             L["sh_bg"], L["sh_bu"], L["sh_bd"] = gs[1], us[1], ds[1]
@@ -111,18 +128,19 @@ def small_layer(E=1, k=1, n_shared=0, H=64, I=32, I_sh=32, fmt=0, scaling=1.0, s
 def np_expert(desc, L, e, xd):
     """Dense SwiGLU of routed expert e (or the shared expert if e is None), numpy."""
     fmt = desc["fmt"]
+    dq = NP_DEQUANT_ROWSCALED.get(fmt)
     if e is None:
-        if fmt == 0:
-            Wg = np_dequant_int4(L["sh_g"], L["sh_sg"]); Wu = np_dequant_int4(L["sh_u"], L["sh_su"])
-            Wd = np_dequant_int4(L["sh_d"], L["sh_sd"])
+        if fmt != 1:
+            Wg = dq(L["sh_g"], L["sh_sg"]); Wu = dq(L["sh_u"], L["sh_su"])
+            Wd = dq(L["sh_d"], L["sh_sd"])
         else:
             Wg = np_dequant_nvfp4(L["sh_g"], L["sh_bg"], L["sh_tg"])
             Wu = np_dequant_nvfp4(L["sh_u"], L["sh_bu"], L["sh_tu"])
             Wd = np_dequant_nvfp4(L["sh_d"], L["sh_bd"], L["sh_td"])
     else:
-        if fmt == 0:
-            Wg = np_dequant_int4(L["g"][e], L["sg"][e]); Wu = np_dequant_int4(L["u"][e], L["su"][e])
-            Wd = np_dequant_int4(L["d"][e], L["sd"][e])
+        if fmt != 1:
+            Wg = dq(L["g"][e], L["sg"][e]); Wu = dq(L["u"][e], L["su"][e])
+            Wd = dq(L["d"][e], L["sd"][e])
         else:
             Wg = np_dequant_nvfp4(L["g"][e], L["bg"][e], L["tg"][e])
             Wu = np_dequant_nvfp4(L["u"][e], L["bu"][e], L["tu"][e])
@@ -305,6 +323,55 @@ def pin_route_weights(o):
     assert abs(float(gap[0]) - float(np.float32(0.7) - np.float32(0.5))) < 1e-7, gap
 
 
+# ---------------------------------------------------------------- int8 / int2 and quantisation
+def pin_int8_int2_hand(o):
+    """Hand decodes: int8 bytes 0x00 0x01 0x7F 0x80 0xFF 0xFE 0x40 0xC0 are 0 1 127 -128 -1
+    -2 64 -64; int2 byte 0xE4 (11 10 01 00) holds 0 1 -2 -1 from element 0 up, 0x1B
+    (00 01 10 11) holds -1 -2 1 0; the row scale multiplies."""
+    b8 = np.array([0x00, 0x01, 0x7F, 0x80, 0xFF, 0xFE, 0x40, 0xC0], np.uint8)
+    assert o.int8_row(b8, 8).tolist() == [0, 1, 127, -128, -1, -2, 64, -64]
+    b2 = np.array([0xE4, 0x1B], np.uint8)
+    assert o.int2_row(b2, 8).tolist() == [0, 1, -2, -1, -1, -2, 1, 0]
+    M8 = {"format": 2, "codes": b8.reshape(1, 8), "row_scale": np.float32([0.5])}
+    assert o.dequant(M8)[0].tolist() == [0.0, 0.5, 63.5, -64.0, -0.5, -1.0, 32.0, -32.0]
+    M2 = {"format": 3, "codes": np.array([[0xE4, 0x1B], [0xFF, 0x55]], np.uint8),
+          "row_scale": np.float32([0.25, 2.0])}
+    assert o.dequant(M2).tolist() == [[0.0, 0.25, -0.5, -0.25, -0.25, -0.5, 0.25, 0.0],
+                                      [-2.0, -2.0, -2.0, -2.0, 2.0, 2.0, 2.0, 2.0]]
+
+
+def pin_quantize_hand(o):
+    """Exact rows: scale = max|w| / (2^(bits-1) - 1); codes round half to even."""
+    codes, sc = o.quantize(np.array([[3.0, -7.0, 1.0, 0.5], [1.5, -3.5, 2.5, 0.25],
+                                     [0.0, 0.0, 0.0, 0.0], [0.75, -0.25, 0.0, 1.75]], np.float32), 4)
+    assert sc.tolist() == [1.0, 0.5, 0.0, 0.25]
+    assert [o.int4_row(codes[r], 4).tolist() for r in range(4)] == [[3, -7, 1, 0], [3, -7, 5, 0],
+                                                                     [0, 0, 0, 0], [3, -1, 0, 7]]
+    codes, sc = o.quantize(np.array([[127.0, -0.5, 0.5, 1.5, -2.5, 2.5, -127.0, 3.0]], np.float32), 8)
+    assert sc.tolist() == [1.0]
+    assert o.int8_row(codes[0], 8).tolist() == [127, 0, 0, 2, -2, 2, -127, 3]
+    codes, sc = o.quantize(np.array([[2.0, -1.0, 0.5, 1.5, -2.0, 0.0, 1.0, -3.0]], np.float32), 2)
+    assert sc.tolist() == [3.0]
+    assert o.int2_row(codes[0], 8).tolist() == [1, 0, 0, 0, -1, 0, 0, -1]
+
+
+def pin_quantize_roundtrip(o):
+    """Random rows, every width: codes within range, the largest |w| of a row maps to the
+    largest code magnitude, and dequantised values are within half a step of w."""
+    rng = np.random.default_rng(12)
+    for bits, fmt in ((8, 2), (4, 0), (2, 3)):
+        qmax = 2 ** (bits - 1) - 1
+        w = (rng.standard_normal((6, 32)) * rng.uniform(0.01, 3.0, (6, 1))).astype(np.float32)
+        codes, sc = o.quantize(w, bits)
+        deq = o.dequant({"format": fmt, "codes": codes, "row_scale": sc})
+        for r in range(6):
+            amax = float(np.abs(w[r].astype(np.float64)).max())
+            assert sc[r] == np.float32(amax / qmax)
+            q = np.rint(deq[r] / float(sc[r])).astype(np.int64)
+            assert np.all(np.abs(q) <= qmax) and np.abs(q).max() == qmax
+            assert np.all(np.abs(deq[r] - w[r].astype(np.float64)) <= 0.5 * float(sc[r]) * (1 + 1e-6))
+
+
 # ---------------------------------------------------------------- adaptive top-p
 def _logit_of(p):
     """A float32 logit whose fp32 sigmoid is close to p."""
@@ -423,8 +490,9 @@ def pin_group_bruteforce(o):
 # ---------------------------------------------------------------- FFN and layer
 def pin_dense_equivalence(o):
     """E=1, k=1, no shared expert, scaling 1: w = s/s = 1, so the layer is a dense
-    SwiGLU FFN; with a shared expert and scaling 2.5 it is 2.5*FFN + shared FFN."""
-    for fmt in (0, 1):
+    SwiGLU FFN; with a shared expert and scaling 2.5 it is 2.5*FFN + shared FFN.
+    Every weight format: int4, NVFP4, int8, int2."""
+    for fmt in (0, 1, 2, 3):
         desc, L, x = small_layer(E=1, k=1, n_shared=0, fmt=fmt, scaling=1.0, seed=11 + fmt)
         r = o.forward(desc, L, x, want_h=True)
         xd = x.view(np.float16).astype(np.float64)
@@ -444,7 +512,7 @@ def pin_dense_equivalence(o):
 def pin_layer_composition(o):
     """Several experts: y_t = shared(x_t) + sum_j w_tj * FFN_{e_tj}(x_t) with each
     FFN evaluated densely by numpy and the weights from the (pinned) router."""
-    for fmt in (0, 1):
+    for fmt in (0, 1, 2, 3):
         desc, L, x = small_layer(E=6, k=3, n_shared=1, fmt=fmt, scaling=2.5, seed=31 + fmt)
         r = o.forward(desc, L, x)
         xd = x.view(np.float16).astype(np.float64)
@@ -514,7 +582,8 @@ def pin_topp_layer(o):
 
 
 PINS = [pin_half_exhaustive, pin_int4_hand, pin_e2m1_table, pin_e4m3_exhaustive,
-        pin_nvfp4_hand, pin_sigmoid_closed_forms, pin_router_onehot, pin_router_matmul,
+        pin_nvfp4_hand, pin_int8_int2_hand, pin_quantize_hand, pin_quantize_roundtrip,
+        pin_sigmoid_closed_forms, pin_router_onehot, pin_router_matmul,
         pin_topk_bruteforce, pin_route_weights, pin_topp_hand, pin_topp_boundary,
         pin_topp_bruteforce, pin_group_bruteforce, pin_dense_equivalence,
         pin_layer_composition, pin_union_identity, pin_expert_relabel, pin_forward_token,

@@ -58,6 +58,18 @@ MUTANTS = {
                         "acc += (double)topk_w[(size_t)t * k + (k - 1 - j)] * y_assign"),
     "batched_token_index": ("int a = R->perm[p], t = a / k;", "int a = R->perm[p], t = a % T;"),
     "gap_wrong": ("gap = (float)((double)last - (double)next);", "gap = (float)((double)last);"),
+    # int8 / int2 codes and the quantiser
+    "int8_unsigned": ("return n >= 128 ? n - 256 : n;", "return n;"),
+    "int8_row_stride": ("return format == ORC_INT8 ? (size_t)K :", "return format == ORC_INT8 ? (size_t)(K / 2) :"),
+    "int2_bit_order": ("int n = (int)((b >> (2 * (k & 3))) & 3u);", "int n = (int)((b >> (6 - 2 * (k & 3))) & 3u);"),
+    "int2_unsigned": ("return n >= 2 ? n - 4 : n;", "return n;"),
+    "quant_levels": ("float sc = (float)(amax / qmax);", "float sc = (float)(amax / (qmax + 1));"),
+    "quant_truncate": ("double v = rint((double)w[(size_t)n * K + k] / (double)sc);",
+                       "double v = trunc((double)w[(size_t)n * K + k] / (double)sc);"),
+    "quant_int2_pack": ("row[k >> 2] |= (uint8_t)((u & 3u) << (2 * (k & 3)));",
+                        "row[k >> 2] |= (uint8_t)((u & 3u) << (2 * (3 - (k & 3))));"),
+    "quant_int4_pack": ("row[k >> 1] |= (uint8_t)((u & 15u) << (4 * (k & 1)));",
+                        "row[k >> 1] |= (uint8_t)((u & 15u) << (4 * (1 - (k & 1))));"),
     # adaptive expert top-p
     "topp_le": ("keep[at[r]] = before < top_p * S;", "keep[at[r]] = before <= top_p * S;"),
     "topp_rank_ascending": ("if (si > sj || (si == sj && idx[i] < idx[j])) r++;",
