@@ -298,10 +298,6 @@ Launch ffn_launch(const moe_layer *L, int T, bool gu)
     if (use_tc(d, T)) return {1, L->num_sms};                         // one CTA per SM
     if (use_limbs(d, T)) return {1, L->num_sms * L->occ[0][gu][0]};   // the int8 path has KS = 1 only
     const long i1 = items(4), i4 = items(1);
-#ifdef MOE_FORCE_KS
-    if (MOE_FORCE_KS == 4) return {4, L->num_sms * L->occ[wide][gu][1]};
-    return {1, L->num_sms * L->occ[wide][gu][0]};
-#endif
     if (i1 >= L->num_sms && eff(i1) >= 0.85 * eff(i4)) return {1, L->num_sms * L->occ[wide][gu][0]};
     return {4, L->num_sms * L->occ[wide][gu][1]};
 }
