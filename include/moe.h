@@ -154,7 +154,9 @@ size_t moe_workspace_size(const moe_layer *layer, int T);
 /* Steps 1-2.  x [T][H] fp16.  If logits_in is non-NULL ([T][E] fp32) the router GEMV is
  * skipped and these logits are used (bit-exact selection from given logits).  If
  * logits_out is non-NULL the fp32 logits are written there.  Outputs: topk_idx int32
- * [T][k] (descending selection score), topk_w fp32 [T][k].  0 <= T <= max_tokens. */
+ * [T][k] (descending selection score), topk_w fp32 [T][k].  With the layer's adaptive
+ * top-p active, each token's kept experts come first (in that order) and the remaining
+ * entries are index -1 with weight 0.  0 <= T <= max_tokens. */
 int moe_route(const moe_layer *layer, const uint16_t *x, int T, const float *logits_in,
               float *logits_out, int32_t *topk_idx, float *topk_w, void *workspace,
               size_t workspace_bytes, moe_stream_t stream);
@@ -183,11 +185,12 @@ int moe_route(const moe_layer *layer, const uint16_t *x, int T, const float *log
 int moe_route_static(const moe_layer *layer, const uint16_t *x, int T, const float *logits_in,
                      float *logits_out, int32_t *topk_idx, float *topk_w, moe_stream_t stream);
 
-/* Step 3.  topk_idx [T][k] with values in [0, E) (out-of-range values set
- * MOE_ERR_DEVICE_BOUNDS and are dropped).  Outputs (int32): counts [E], offsets [E+1]
- * (exclusive prefix sum of counts), perm [T*k] (assignment ids a = t*k + j ordered by
- * expert, ascending a inside an expert), unique [E] (experts with counts > 0,
- * ascending; entries past n_unique are unspecified), n_unique [1]. */
+/* Step 3.  topk_idx [T][k] with values in [0, E), or -1 for an entry dropped by top-p
+ * (other out-of-range values set MOE_ERR_DEVICE_BOUNDS and are dropped too).  Outputs
+ * (int32): counts [E], offsets [E+1] (exclusive prefix sum of counts; offsets[E] is the
+ * number of grouped assignments), perm [T*k] (the first offsets[E] entries: assignment
+ * ids a = t*k + j ordered by expert, ascending a inside an expert), unique [E] (experts
+ * with counts > 0, ascending; entries past n_unique are unspecified), n_unique [1]. */
 int moe_group(const moe_layer *layer, const int32_t *topk_idx, int T, int32_t *counts,
               int32_t *offsets, int32_t *perm, int32_t *unique, int32_t *n_unique,
               void *workspace, size_t workspace_bytes, moe_stream_t stream);
@@ -201,7 +204,9 @@ int moe_expert_ffn(const moe_layer *layer, const uint16_t *x, int T, const int32
                    size_t workspace_bytes, moe_stream_t stream);
 
 /* Step 5.  y [T][H] fp16 = y_shared[t] + sum_j topk_w[t][j] * y_assign[t*k + j], summed
- * in fp32 in the order shared, j = 0 .. k-1.  y_shared may be NULL when n_shared = 0. */
+ * in fp32 in the order shared, j = 0 .. k-1; terms with weight 0 (entries dropped by
+ * top-p, whose y_assign rows are never written) are skipped.  y_shared may be NULL when
+ * n_shared = 0. */
 int moe_combine(const moe_layer *layer, const float *y_assign, const float *y_shared,
                 const float *topk_w, int T, uint16_t *y, moe_stream_t stream);
 
