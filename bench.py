@@ -57,8 +57,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"
 # DRAM traffic per launch (bytes) of the dominant kernel from an ncu capture, keyed by
 # workload; valid only while the kernel source hashes to the recorded value.
 NCU_TRAFFIC = {
-    # profiles/ffn_kernel_int4_decode1_e32_full.md: dram read 113,490,176 + write 3,437,824
-    # bytes per gate/up launch (a T=1 step reads the same 9 experts at E=32 as at E=256)
+    # ncu capture of the decode gate/up kernel: dram read 113,490,176 + write 3,437,824
+    # bytes per launch (a T=1 step reads the same 9 experts at E=32 as at E=256)
     "decode1": {"kernel": "gate_up", "bytes": 116928000, "kernel_hash": "9e4eafe6af364447"},
 }
 
@@ -360,28 +360,64 @@ def run_reference(args, w):
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args, w):
+# workloads measured beside the headline one in the default run (the rest of the
+# metric's configurations: T=8 decode, NVFP4 at T=1 and T=16, the T=512 batch)
+EXTRA_CONFIGS = ("decode8", "nvfp4_1", "nvfp4_16", "prefill512")
+MIN_REGION_S = 0.5     # timed regions are repeated until they add up to at least this
+
+
+def region_count(first_ms: float, min_s: float) -> int:
+    """Timed regions to run so that they add up to ``min_s`` seconds, given the slowest
+    rank's first region (at least three)."""
+    return max(3, int(np.ceil(min_s * 1000.0 / max(first_ms, 1e-3))))
+
+
+def timed_regions(run_steps, world, dev, stream, min_s):
+    """Times regions of exactly K steps -- barrier and device synchronisation on both
+    sides, CUDA events on the launch stream -- until they add up to ``min_s`` (at least
+    three regions; every rank runs the same number, decided from the slowest rank's first
+    region).  Returns this rank's per-region milliseconds."""
+    import torch
+
+    def one():
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            run_steps()
+            e1.record(stream)
+        e1.synchronize()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        return e0.elapsed_time(e1)
+
+    ms = [one()]
+    n = region_count(max_over_ranks(world, ms[0]), min_s)
+    for _ in range(n - 1):
+        ms.append(one())
+    return ms
+
+
+def bench_config(args, w, world, dev, stream, host=None, want_e2e=True):
+    """One workload: R rotating layer copies resident in HBM, K steps per timed region."""
     import torch
 
     import w4a16_quantized_expert_b200 as moe
     from w4a16_quantized_expert_b200.device import DeviceLayer
 
-    world, rank, local = dist_setup(args.gpus)
-    dev = torch.device("cuda", local if world > 1 else 0)
     R = args.layers or DEFAULTS.get(w.name, (0, 0, 8))[2]
     K, Wm = args.steps, args.warmup
     desc = {"H": w.H, "I": w.I, "I_sh": w.I_sh, "E": w.E, "k": w.k, "n_shared": w.n_shared,
             "scaling": w.scaling, "fmt": w.fmt, "top_p": w.top_p}
-
-    # ---- inputs resident in HBM
-    host = synth.make_layer(w)
+    if host is None:
+        host = synth.make_layer(w)
     base = DeviceLayer(desc, host, max_tokens=w.T, device=dev)
     layers = [base] + [base.clone_weights() for _ in range(R - 1)]
     xs_host = [synth.make_tokens(w, batch=b) for b in range(R)]
     xs = [torch.from_numpy(x.copy()).to(dev) for x in xs_host]
     ys = [torch.empty_like(x) for x in xs]
     ws = layers[0].workspace(w.T)
-    stream = torch.cuda.Stream(device=dev)
 
     # unique experts per batch (for the byte accounting), from the library's own grouping
     U, A = [], []
@@ -391,138 +427,199 @@ def run_ours(args, w):
             _, _, _, _, nu = base.group(idx, w.T, ws, stream=stream)
             U.append(int(nu.item()))
             A.append(int((idx >= 0).sum().item()))   # fewer than T*k with adaptive top-p
-    U_mean = float(np.mean(U))
-    A_mean = float(np.mean(A))
+    U_mean, A_mean = float(np.mean(U)), float(np.mean(A))
     ab = algorithmic_bytes(w, U_mean)
 
-    # ---- graphs of R consecutive layer calls
-    def capture(n):
+    # ---- graphs of R consecutive layer calls (K steps = reps graphs + a remainder graph)
+    def capture(fn, n):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for i in range(n):
-                layers[i].forward(xs[i], ws, y=ys[i], stream=stream)
+                fn(i)
         return g
+
+    def fwd(i):
+        layers[i].forward(xs[i], ws, y=ys[i], stream=stream)
 
     with torch.cuda.stream(stream):
         for i in range(R):      # eager warm-up of every layer
-            layers[i].forward(xs[i], ws, y=ys[i], stream=stream)
+            fwd(i)
     torch.cuda.synchronize(dev)
-    g_full = capture(R)
-    rem = K % R
-    g_rem = capture(rem) if rem else None
-    reps = K // R
+    rem, reps = K % R, K // R
+    g_full = capture(fwd, R)
+    g_rem = capture(fwd, rem) if rem else None
 
-    with torch.cuda.stream(stream):      # graphs replay on torch's current stream
+    def steps(gf, gr):
+        def run():
+            for _ in range(reps):
+                gf.replay()
+            if gr is not None:
+                gr.replay()
+        return run
+
+    with torch.cuda.stream(stream):      # warm-up steps (graphs replay on the current stream)
         for _ in range(max(1, (Wm + R - 1) // R)):
             g_full.replay()
     torch.cuda.synchronize(dev)
     st = moe.moe_get_device_status(base.handle)
     assert st == moe.MOE_OK, moe.status_string(st)
 
-    clocks = ClockSampler(local if world > 1 else 0)
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
     clocks.start()
-    time.sleep(0.5)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize(dev)
+    time.sleep(0.4)
     t_wall0 = time.time()
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        for _ in range(reps):
-            g_full.replay()
-        if g_rem is not None:
-            g_rem.replay()
-        ev1.record(stream)
-    ev1.synchronize()
-    torch.cuda.synchronize(dev)
+    region_ms = timed_regions(steps(g_full, g_rem), world, dev, stream, args.min_region_s)
     t_wall1 = time.time()
-    barrier(world)
-    ms = ev0.elapsed_time(ev1)
     time.sleep(0.3)
     clocks.stop()
-    ms_max = max_over_ranks(world, ms)
-    ms_step = ms_max / K
-    tokens_per_s = job_tokens_per_s(world, K, w.T, ms_max)
+    ms_region = max_over_ranks(world, float(np.median(region_ms)))
+    ms_step = ms_region / K
     st = moe.moe_get_device_status(base.handle)
     assert st == moe.MOE_OK, moe.status_string(st)
 
-    # ---- per-kernel durations: the same kernels on the same work, launched without PDL
-    # with event-record nodes between them, captured in a graph so that no host launch
-    # gap falls inside a measured interval
-    nk = R * max(1, min(K, 2048) // R)
+    # ---- per-kernel durations: the same kernels on the same work launched without PDL,
+    # event-record nodes between them, captured in a graph (no host gap inside an interval)
+    nk = R * max(1, min(K, 512) // R)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(R)]
     with torch.cuda.stream(stream):
         for e4 in evs:
             for e in e4:
                 e.record(stream)
     torch.cuda.synchronize(dev)
-    gk = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gk, stream=stream):
-        for i in range(R):
-            moe.moe_forward_timed(layers[i].handle, xs[i].data_ptr(), w.T, ys[i].data_ptr(),
-                                  ws.data_ptr(), ws.numel(), stream.cuda_stream,
-                                  [e.cuda_event for e in evs[i]])
+    info = [0, 0]
+
+    def fwd_timed(i):
+        info[:] = moe.moe_forward_timed(layers[i].handle, xs[i].data_ptr(), w.T, ys[i].data_ptr(),
+                                        ws.data_ptr(), ws.numel(), stream.cuda_stream,
+                                        [e.cuda_event for e in evs[i]])
+
+    gk = capture(fwd_timed, R)
     dur = []
     with torch.cuda.stream(stream):
         for _ in range(nk // R):
             gk.replay()
             torch.cuda.synchronize(dev)
             dur += [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(R)]
-    k_ms = np.array(dur).mean(axis=0)            # router, gate_up, down (ms per launch)
-    names = ["router", "gate_up", "down"]
+    parts, launches = info
+    k_ms = np.array(dur).mean(axis=0)
+    if parts == 1:      # one kernel does the whole layer
+        names, k_ms, kbytes = ["layer"], k_ms[:1], [ab["total"]]
+    else:
+        names, kbytes = ["router", "gate_up", "down"], [ab["router"], ab["gate_up"], ab["down"]]
     dom = int(np.argmax(k_ms))
     peaks = load_peaks()
     hbm_peak = float(peaks["hbm_gbs"])
-    dom_bytes = ab[names[dom]]
-    achieved = dom_bytes / (k_ms[dom] * 1e-3) / 1e9
+    achieved = kbytes[dom] / (k_ms[dom] * 1e-3) / 1e9
     tr = NCU_TRAFFIC.get(w.name)
     traffic = (tr["bytes"] if tr and tr.get("kernel") == names[dom] and tr.get("kernel_hash") == kernel_hash()
                else None)
 
     # ---- end to end through the public API with host buffers
-    xh = [torch.from_numpy(x.copy()).pin_memory() for x in xs_host]
-    yh = [torch.empty_like(x).pin_memory() for x in xh]
+    e2e = None
+    if want_e2e:
+        xh = [torch.from_numpy(x.copy()).pin_memory() for x in xs_host]
+        yh = [torch.empty_like(x).pin_memory() for x in xh]
 
-    def capture_host(n):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(n):
-                layers[i].forward_host(xh[i], yh[i], ws, stream=stream)
-        return g
+        def fwd_host(i):
+            layers[i].forward_host(xh[i], yh[i], ws, stream=stream)
 
-    ge = capture_host(R)
-    ge_rem = capture_host(rem) if rem else None
-    with torch.cuda.stream(stream):
-        for _ in range(max(1, (Wm + R - 1) // R)):
-            ge.replay()
+        ge = capture(fwd_host, R)
+        ge_rem = capture(fwd_host, rem) if rem else None
+        with torch.cuda.stream(stream):
+            for _ in range(max(1, (Wm + R - 1) // R)):
+                ge.replay()
+        torch.cuda.synchronize(dev)
+        e_ms = timed_regions(steps(ge, ge_rem), world, dev, stream, args.min_region_s / 2)
+        e2e_ms = max_over_ranks(world, float(np.median(e_ms)))
+        e2e = {"value": job_tokens_per_s(world, K, w.T, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 2,
+               "timed_regions": len(e_ms),
+               "how": "moe_forward_host (pinned host x in, y out) captured in CUDA graphs"}
+        st = moe.moe_get_device_status(base.handle)
+        assert st == moe.MOE_OK, moe.status_string(st)
+        del ge, ge_rem
+
+    tflops = flops(w, A_mean) / (ms_step * 1e-3) / 1e12
+    out = {
+        "w": w, "host": host, "ms_step": ms_step, "region_ms": region_ms, "R": R, "U": U_mean,
+        "ab": ab, "tflops": tflops, "kernels_ms": {n: float(v) for n, v in zip(names, k_ms)},
+        "launches_per_step": launches,
+        "roofline": {
+            "kernel": names[dom], "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
+            "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": traffic,
+            "algorithmic_bytes_per_launch": kbytes[dom],
+            "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] == "measured" else "fallback",
+        },
+        "e2e": e2e, "clocks": clocks.summary(t_wall0, t_wall1), "peaks": peaks,
+        "timed_region_s": float(np.sum(region_ms)) / 1000.0,
+    }
+    del g_full, g_rem, gk
+    for L in layers:
+        L.close()
+    del layers, xs, ys, ws
     torch.cuda.synchronize(dev)
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(reps):
-            ge.replay()
-        if ge_rem is not None:
-            ge_rem.replay()
-        e1.record(stream)
-    e1.synchronize()
-    e2e_ms = max_over_ranks(world, e0.elapsed_time(e1))
-    e2e_value = job_tokens_per_s(world, K, w.T, e2e_ms)
-    st = moe.moe_get_device_status(base.handle)
-    assert st == moe.MOE_OK, moe.status_string(st)
+    torch.cuda.empty_cache()
+    return out
 
+
+def config_entry(world, r, K) -> dict:
+    """A workload's figures for the ``configs`` object of the JSON line."""
+    w, ab, ms = r["w"], r["ab"], r["ms_step"]
+    hbm_peak = r["roofline"]["peak"]
+    qgbs = ab["weights"] / (ms * 1e-3) / 1e9
+    e = {
+        "workload": describe(w), "T": w.T,
+        "ms_per_layer": ms, "tokens_per_s": job_tokens_per_s(world, K, w.T, ms * K),
+        "unique_experts_per_step": r["U"],
+        "quantized_weight_gbs": qgbs, "frac_quantized_of_8tbs": qgbs / 8000.0,
+        "frac_quantized_of_measured": qgbs / hbm_peak,
+        "layer_gbs": ab["total"] / (ms * 1e-3) / 1e9,
+        "kernels_ms": r["kernels_ms"], "roofline": r["roofline"],
+        "tflops": r["tflops"], "timed_regions": len(r["region_ms"]), "steps": K,
+        "clocks": r["clocks"],
+    }
+    if w.T >= 256:     # the batch configuration: tensor throughput against the dense peak
+        pk = float(r["peaks"].get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        e["tflops_frac_of_dense_fp16_peak"] = r["tflops"] / pk
+        e["dense_peak_tflops"] = pk
+    if r["e2e"]:
+        e["e2e_tokens_per_s"] = r["e2e"]["value"]
+    return e
+
+
+def run_ours(args, w):
+    import torch
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    stream = torch.cuda.Stream(device=dev)
+    K, Wm = args.steps, args.warmup
+
+    head = bench_config(args, w, world, dev, stream)
+    extras = {}
+    if w.name == "decode1" and not args.no_configs:
+        shared_host = {}
+        for name in EXTRA_CONFIGS:
+            wx = synth.WORKLOADS[name]
+            key = (wx.seed, wx.fmt, wx.H, wx.I, wx.E, wx.bias)   # nvfp4_1 and nvfp4_16: one layer
+            if key not in shared_host:
+                shared_host.clear()
+                shared_host[key] = synth.make_layer(wx)
+            extras[name] = bench_config(args, wx, world, dev, stream, host=shared_host[key])
     if rank != 0:
         return
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_tokens_per_s(w, host, xs_host, seconds=args.cpu_seconds)
+        xs_host = [synth.make_tokens(w, batch=b) for b in range(4)]
+        cpu = oracle_tokens_per_s(w, head["host"], xs_host, seconds=args.cpu_seconds)
 
+    ab, ms_step = head["ab"], head["ms_step"]
+    hbm_peak = head["roofline"]["peak"]
     layer_gbs = ab["total"] / (ms_step * 1e-3) / 1e9
     weights_gbs = ab["weights"] / (ms_step * 1e-3) / 1e9
-    cl = clocks.summary(t_wall0, t_wall1)
     line = {
         "metric": METRIC,
-        "value": tokens_per_s,
+        "value": job_tokens_per_s(world, K, w.T, ms_step * K),
         "unit": UNIT,
         "n_gpus": world,
         "steps": K,
@@ -537,13 +634,16 @@ def run_ours(args, w):
             "workload": describe(w),
             "T": w.T, "H": w.H, "I": w.I, "E": w.E, "top_k": w.k, "top_p": w.top_p, "n_shared": w.n_shared,
             "weights": "int4" if w.fmt == synth.FMT_INT4 else "nvfp4",
-            "rotating_layers": R,
-            "unique_experts_per_step": U_mean,
-            "l2": f"no flush: {R} layer copies at distinct addresses, "
+            "rotating_layers": head["R"],
+            "unique_experts_per_step": head["U"],
+            "l2": f"no flush: {head['R']} layer copies at distinct addresses, "
                   f"{ab['total'] / 1e6:.0f} MB of weights per step > 126 MB L2",
-            "timing": "CUDA graphs of consecutive layer calls, CUDA events on the launch stream",
+            "timing": f"CUDA graphs of consecutive layer calls, CUDA events on the launch stream; "
+                      f"{len(head['region_ms'])} timed regions of exactly {K} steps, median",
             "parallelism": f"replicas x{world}",
         },
+        "timed_regions": len(head["region_ms"]),
+        "timed_region_s": head["timed_region_s"],
         "hbm": {
             "bytes_per_step": ab["total"],
             "layer_gbs": layer_gbs,
@@ -551,31 +651,16 @@ def run_ours(args, w):
             "peak_gbs": hbm_peak,
             "frac_layer": layer_gbs / hbm_peak,
             "frac_quantized_of_8tbs": weights_gbs / 8000.0,
-            "peak_source": peaks["source"],
+            "peak_source": head["peaks"]["source"],
         },
-        "tflops": flops(w, A_mean) / (ms_step * 1e-3) / 1e12,
-        "kernels_ms": {n: float(v) for n, v in zip(names, k_ms)},
-        "roofline": {
-            "kernel": names[dom],
-            "bound": "hbm",
-            "achieved": achieved,
-            "peak": hbm_peak,
-            "unit": "GB/s",
-            "frac": achieved / hbm_peak,
-            "traffic": traffic,
-            "algorithmic_bytes_per_launch": dom_bytes,
-            "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] == "measured" else "fallback",
-        },
-        "e2e": {
-            "value": e2e_value,
-            "unit": UNIT,
-            "h2d_bytes_per_step": w.T * w.H * 2,
-            "d2h_bytes_per_step": w.T * w.H * 2,
-            "how": "moe_forward_host (pinned host x in, y out) captured in CUDA graphs",
-        },
-        "gpu_launches": 4 * K,   # per layer call: router, gate/up, down, combine
-        "clocks": cl,
+        "tflops": head["tflops"],
+        "kernels_ms": head["kernels_ms"],
+        "roofline": head["roofline"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["launches_per_step"] * K * len(head["region_ms"]),
+        "clocks": head["clocks"],
         "cpu_baseline": cpu,
+        "configs": {name: config_entry(world, r, K) for name, r in extras.items()},
     }
     print(json.dumps(line), flush=True)
 
@@ -594,6 +679,10 @@ def main():
     ap.add_argument("--inter", type=int, default=None, help="override I and I_sh (profiling only)")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="measure the chosen workload only (no other configurations in the line)")
+    ap.add_argument("--min-region-s", type=float, default=MIN_REGION_S,
+                    help="repeat each timed region of K steps until they add up to this")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]

@@ -128,7 +128,11 @@ typedef struct moe_layer moe_layer;   /* opaque handle */
 
 /* ---------------------------------------------------------------- lifetime */
 
-/* Validates desc and weights and builds the handle: TMA descriptors over the caller's
+/* Source: the layer's shape and weight formats -- int4 with per-row scales (hakusoku
+ * page "Show HN: 低速のコンピュータでGLM 5.2を動かす方法", section "実装済み機能"), NVFP4
+ * (648news page "GTX 1070向け35BパラメータMoEモデル推論エンジン公開", section "用語の注釈"),
+ * 256 experts of about 19 MB (hakusoku page, section "Colibrì: ...").
+ * Validates desc and weights and builds the handle: TMA descriptors over the caller's
  * weights and a device status word (the only allocation the library makes).
  * Requirements: H and I (and I_sh) multiples of 64 (int4) or 256 (NVFP4) -- the NVFP4
  * block-scale rows must be 16-byte multiples -- H <= 16384, I, I_sh <= 16384,
@@ -137,11 +141,14 @@ typedef struct moe_layer moe_layer;   /* opaque handle */
  * Returns MOE_OK and *out, or an error code and *out = NULL. */
 int moe_layer_create(const moe_layer_desc *desc, const moe_weights *weights, moe_layer **out);
 
-/* Frees the handle (and its status word).  The caller must ensure no call on it is
+/* Source: none of the pages has a handle; this ends the lifetime moe_layer_create began.
+ * Frees the handle (and its status word).  The caller must ensure no call on it is
  * still running on the GPU.  NULL is accepted. */
 int moe_layer_destroy(moe_layer *layer);
 
-/* Bytes of device workspace any call with T tokens needs (0 if T is out of range).
+/* Source: none of the pages sizes buffers; the workspace holds the intermediate results of
+ * the steps the pages name (logits, top-k, grouping, h, per-expert outputs).
+ * Bytes of device workspace any call with T tokens needs (0 if T is out of range).
  * One workspace serves every entry point; it must be 256-byte aligned, and must not be
  * used by two calls that may run concurrently.  It holds a few completion counters that
  * must be ZERO before the workspace's first use (one cudaMemset of the whole buffer);
@@ -151,7 +158,10 @@ size_t moe_workspace_size(const moe_layer *layer, int T);
 
 /* ---------------------------------------------------------------- staged steps */
 
-/* Steps 1-2.  x [T][H] fp16.  If logits_in is non-NULL ([T][E] fp32) the router GEMV is
+/* Source: DeepSeek-V3-style sigmoid router with a selection bias (hakusoku page, section
+ * "実装済み機能"); routing fused into the small-batch kernels (648news GLM-5.3-Flash vLLM
+ * page, section "Ampere世代のGPU向けに最適化された独自カーネル群").
+ * Steps 1-2.  x [T][H] fp16.  If logits_in is non-NULL ([T][E] fp32) the router GEMV is
  * skipped and these logits are used (bit-exact selection from given logits).  If
  * logits_out is non-NULL the fp32 logits are written there.  Outputs: topk_idx int32
  * [T][k] (descending selection score), topk_w fp32 [T][k].  With the layer's adaptive
@@ -173,9 +183,11 @@ int moe_route(const moe_layer *layer, const uint16_t *x, int T, const float *log
  * Limits: ceil(T / 16) <= 64 and T * n_experts <= 16384 (e.g. T <= 64 with 256
  * experts); larger calls return MOE_ERR_WORKSPACE and launch nothing.  Other arguments
  * and errors as moe_route.
- * The first call on each device looks up the array's address (cudaGetSymbolAddress,
- * which may load the module) and caches it; make that first call before any stream
- * capture begins.
+ * The first call in each CUDA context (each device's primary context, or any other
+ * context the caller makes current) looks up the array's address there
+ * (cudaGetSymbolAddress, which may load the module) and caches it keyed by the context's
+ * unique id, so a context created later, e.g. after cudaDeviceReset, gets its own lookup;
+ * make that first call before any stream capture begins.
  * The scratch is shared by every handle and stream of the device: calls that may
  * overlap in time (other streams, other threads, other handles) race on it and must be
  * serialised by the caller.  Its 64 tile counters must be zero when a call starts: they
@@ -185,7 +197,10 @@ int moe_route(const moe_layer *layer, const uint16_t *x, int T, const float *log
 int moe_route_static(const moe_layer *layer, const uint16_t *x, int T, const float *logits_in,
                      float *logits_out, int32_t *topk_idx, float *topk_w, moe_stream_t stream);
 
-/* Step 3.  topk_idx [T][k] with values in [0, E), or -1 for an entry dropped by top-p
+/* Source: the batch MoE union, each unique expert of a batch read once and applied to all
+ * its tokens (hakusoku page, section "実装済み機能"), in a deterministic order (648news
+ * GLM-5.3-Flash vLLM page, section "Ampere世代のGPU向けに最適化された独自カーネル群").
+ * Step 3.  topk_idx [T][k] with values in [0, E), or -1 for an entry dropped by top-p
  * (other out-of-range values set MOE_ERR_DEVICE_BOUNDS and are dropped too).  Outputs
  * (int32): counts [E], offsets [E+1] (exclusive prefix sum of counts; offsets[E] is the
  * number of grouped assignments), perm [T*k] (the first offsets[E] entries: assignment
@@ -195,7 +210,11 @@ int moe_group(const moe_layer *layer, const int32_t *topk_idx, int T, int32_t *c
               int32_t *offsets, int32_t *perm, int32_t *unique, int32_t *n_unique,
               void *workspace, size_t workspace_bytes, moe_stream_t stream);
 
-/* Step 4 (and the shared expert).  Uses offsets [E+1] and perm [T*k] as moe_group
+/* Source: W4A16, int4 weights with fp16 activations (648news GLM-5.3-Flash vLLM page,
+ * section "OpenAI互換APIで動く320BパラメータのMoE構成"); weights decoded inside the matmul
+ * kernel (648news GTX 1070 page, section "VRAMとシステムメモリで重みを分割する設計"); the
+ * always-on shared expert (hakusoku page, section "実装済み機能").
+ * Step 4 (and the shared expert).  Uses offsets [E+1] and perm [T*k] as moe_group
  * writes them.  y_assign fp32 [T*k][H]: row a = t*k + j holds expert topk_idx[t][j]
  * applied to x[t] (unscaled).  y_shared fp32 [T][H] receives the shared expert (may be
  * NULL when n_shared = 0). */
@@ -203,7 +222,9 @@ int moe_expert_ffn(const moe_layer *layer, const uint16_t *x, int T, const int32
                    const int32_t *perm, float *y_assign, float *y_shared, void *workspace,
                    size_t workspace_bytes, moe_stream_t stream);
 
-/* Step 5.  y [T][H] fp16 = y_shared[t] + sum_j topk_w[t][j] * y_assign[t*k + j], summed
+/* Source: the weighted sum of the routed experts plus the shared expert of the
+ * DeepSeek-V3-style layer (hakusoku page, section "実装済み機能").
+ * Step 5.  y [T][H] fp16 = y_shared[t] + sum_j topk_w[t][j] * y_assign[t*k + j], summed
  * in fp32 in the order shared, j = 0 .. k-1; terms with weight 0 (entries dropped by
  * top-p, whose y_assign rows are never written) are skipped.  y_shared may be NULL when
  * n_shared = 0. */
@@ -212,7 +233,11 @@ int moe_combine(const moe_layer *layer, const float *y_assign, const float *y_sh
 
 /* ---------------------------------------------------------------- fused layer */
 
-/* Steps 1-5 in as few launches as the path allows.  x [T][H] fp16 in, y [T][H] fp16
+/* Source: the whole MoE layer with routing fused into the small-batch kernels (648news
+ * GLM-5.3-Flash vLLM page, section "Ampere世代のGPU向けに最適化された独自カーネル群") and
+ * replayed as one unit per decode step (648news GTX 1070 page, section
+ * "Pascal世代の制約をCUDAグラフとカーネル最適化で克服").
+ * Steps 1-5 in as few launches as the path allows.  x [T][H] fp16 in, y [T][H] fp16
  * out (x and y may not overlap).  Equal within tolerance to the staged path. */
 int moe_forward(const moe_layer *layer, const uint16_t *x, int T, uint16_t *y,
                 void *workspace, size_t workspace_bytes, moe_stream_t stream);
@@ -234,19 +259,36 @@ const char *moe_status_string(int status);
  * debugging, not for the hot path. */
 int moe_get_device_status(const moe_layer *layer, int *status);
 
+/* Where moe_forward (and moe_forward_host) leave the routing and grouping results of a
+ * call with T tokens inside its workspace: byte offsets from the workspace's start of
+ *   logits fp32 [T][E], topk_idx int32 [T][k], topk_w fp32 [T][k]   (as moe_route
+ *                                                 writes them)
+ *   counts int32 [E], offsets int32 [E+1], perm int32 [T*k], unique int32 [E],
+ *   n_unique int32 [1]                           (as moe_group writes them).
+ * The values stay there until the workspace is used by another call.  For tests and
+ * debugging (a check that the grouping the fused path runs is the method's grouping),
+ * not for the hot path.  Returns MOE_ERR_INVALID_ARG for a NULL argument or T out of
+ * [1, max_tokens]. */
+typedef struct moe_ws_routing {
+    size_t logits, topk_idx, topk_w, counts, offsets, perm, unique, n_unique;
+} moe_ws_routing;
+int moe_workspace_routing(const moe_layer *layer, int T, moe_ws_routing *out);
+
 /* Test hook for the bounded waits: launches one block whose consumer waits on an
  * mbarrier that nothing completes, with an iteration limit of max_iters.  The kernel
  * gives up, records MOE_ERR_DEVICE_TIMEOUT in the status word and returns. */
 int moe_debug_wait_timeout(const moe_layer *layer, long long max_iters, moe_stream_t stream);
 
 /* moe_forward for per-kernel timing: the same kernels on the same work, launched without
- * programmatic dependent launch so that events[0..3] (cudaEvent_t handles, recorded on
- * the stream) bracket them: [0] before the router, [1] after the router / before the
- * expert gate/up kernel, [2] after gate/up / before the down kernel (which also
- * combines), [3] after it.  For benchmarks and profiling, not for the hot path. */
+ * programmatic dependent launch, with events[0..3] (cudaEvent_t handles, recorded on the
+ * stream) between them.  info (may be NULL) receives info[0] = the number of timed parts
+ * and info[1] = the number of kernels the call launches.  Three parts: [0, 1] the router,
+ * [1, 2] the gate/up kernel, [2, 3] the down kernel and the combine kernel.  One part:
+ * [0, 1] the single kernel that runs the whole layer; events[2] and events[3] are
+ * recorded right after events[1].  For benchmarks and profiling, not for the hot path. */
 int moe_forward_timed(const moe_layer *layer, const uint16_t *x, int T, uint16_t *y,
                       void *workspace, size_t workspace_bytes, moe_stream_t stream,
-                      void *const events[4]);
+                      void *const events[4], int info[2]);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int moe_version(void);

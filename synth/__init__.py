@@ -80,6 +80,7 @@ def _p(a: np.ndarray) -> int:
 T_X, T_WR, T_BIAS = 1, 2, 3
 T_G, T_U, T_D, T_SG, T_SU, T_SD = 4, 5, 6, 7, 8, 9
 T_SHG, T_SHU, T_SHD, T_SHSG, T_SHSU, T_SHSD = 10, 11, 12, 13, 14, 15
+T_XS = 16   # choices of the edge-case activation rows
 
 
 def _sid(tensor: int, expert: int = 0) -> int:
@@ -260,3 +261,73 @@ def make_layer(w: Workload, experts=None) -> dict:
     layer = {"Wr": Wr, "bias": b}
     layer.update(make_experts(w, experts))
     return layer
+
+
+# ----------------------------------------------------------------- edge-case activations
+STRESS_KINDS = ("outlier", "near_max", "subnormal", "mixed")
+
+
+def make_stress_tokens(w: Workload, T: int, kind: str, batch: int = 0) -> np.ndarray:
+    """fp16 activation rows [T, H] (uint16 bit patterns) at the edges of the fp16 range,
+    for checking that an implementation's activation representation keeps them:
+
+    * ``outlier``: N(0,1) rows in which one or two channels hold +-2^12 .. 2^15 (times
+      a mantissa in [1, 2)), so the rest of the row lies 12 to 16 binary orders below its
+      largest value;
+    * ``near_max``: N(0,1) rows with two channels at +-65504 (the largest finite fp16)
+      and one at +-65472 (the next one down);
+    * ``subnormal``: every value an fp16 subnormal (|x| = m * 2^-24, m in 1..1023);
+    * ``mixed``: N(0,1) rows in which about a quarter of the channels are subnormals.
+
+    Choices (channels, signs, exponents, mantissas) come from the counter-based stream
+    keyed by (seed, T_XS, batch); the N(0,1) parts are ``make_tokens``'s rows."""
+    if kind not in STRESS_KINDS:
+        raise ValueError(kind)
+    x = make_tokens(w, T, batch=batch).copy()
+    H = w.H
+    r = random_bytes(w.seed, _sid(T_XS, batch * 8 + STRESS_KINDS.index(kind)), T * H * 4)
+    r = r.view(np.uint32).reshape(T, H)
+    sign = (r & 1).astype(np.uint16) << 15
+    if kind == "subnormal":
+        m = (((r >> 1) % 1023) + 1).astype(np.uint16)
+        return (sign | m).reshape(T, H)
+    if kind == "mixed":
+        m = (((r >> 1) % 1023) + 1).astype(np.uint16)
+        pick = ((r >> 11) & 3) == 0
+        x[pick] = (sign | m)[pick]
+        return x
+    for t in range(T):
+        c = [int(v % H) for v in r[t, :3] >> 12]
+        if kind == "outlier":
+            n = 1 + int(r[t, 3] & 1)
+            for j in range(n):
+                ex = 12 + int((r[t, 4 + j] >> 4) % 4)                 # 12 .. 15
+                mant = 1.0 + ((int(r[t, 6 + j]) >> 8) % 1024) / 1024.0   # exact in fp16
+                v = np.float16(mant * 2.0 ** ex)
+                x[t, c[j]] = np.array([v], np.float16).view(np.uint16)[0] | int(sign[t, j])
+        else:   # near_max
+            for j, v in enumerate((65504.0, 65504.0, 65472.0)):
+                x[t, c[j]] = np.array([np.float16(v)], np.float16).view(np.uint16)[0] | int(sign[t, j])
+    return x
+
+
+def scale_layer(layer: dict, fmt: int, gate_up: float, down: float, router: float = 1.0) -> dict:
+    """The same layer with every gate/up weight multiplied by ``gate_up``, every down
+    weight by ``down`` and the router weights by ``router`` (powers of two keep the fp32
+    values exact), by scaling the int4 row scales or the NVFP4 per-matrix scales.  Used to
+    keep h and y of edge-case activation rows inside the fp16 range, and the router
+    logits of subnormal rows away from a tie decided by the bias alone."""
+    out = dict(layer)
+    if "Wr" in out:
+        out["Wr"] = (np.asarray(out["Wr"], np.float32) * np.float32(router)).astype(np.float32)
+    if fmt == FMT_INT4:
+        keys_gu, keys_d = ("sg", "su", "sh_sg", "sh_su"), ("sd", "sh_sd")
+    else:
+        keys_gu, keys_d = ("tg", "tu", "sh_tg", "sh_tu"), ("td", "sh_td")
+    for k in keys_gu:
+        if k in out:
+            out[k] = (np.asarray(out[k], np.float32) * np.float32(gate_up)).astype(np.float32)
+    for k in keys_d:
+        if k in out:
+            out[k] = (np.asarray(out[k], np.float32) * np.float32(down)).astype(np.float32)
+    return out

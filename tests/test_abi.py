@@ -110,6 +110,7 @@ def test_null_handle_and_out_of_range_T():
     assert L.moe_forward(None, None, 1, None, None, 0, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_route(None, None, 1, None, None, None, None, None, 0, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_layer_destroy(None) == moe.MOE_OK
+    assert L.moe_workspace_routing(None, 1, None) == moe.MOE_ERR_INVALID_ARG
     st = ctypes.c_int(0)
     assert L.moe_get_device_status(None, ctypes.byref(st)) == moe.MOE_ERR_INVALID_ARG
 
@@ -123,20 +124,24 @@ def test_struct_layouts_match_the_header(tmp_path):
         pytest.skip("no host C compiler")
     fields = [f for f, _ in moe.moe_layer_desc._fields_]
     wfields = [f for f, _ in moe.moe_weights._fields_]
+    rfields = [f for f, _ in moe.moe_ws_routing._fields_]
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "moe.h"', "int main(void) {",
-             '  printf("%zu %zu\\n", sizeof(moe_layer_desc), sizeof(moe_weights));']
+             '  printf("%zu %zu %zu\\n", sizeof(moe_layer_desc), sizeof(moe_weights), sizeof(moe_ws_routing));']
     lines += [f'  printf("%zu\\n", offsetof(moe_layer_desc, {f}));' for f in fields]
     lines += [f'  printf("%zu\\n", offsetof(moe_weights, {f}));' for f in wfields]
+    lines += [f'  printf("%zu\\n", offsetof(moe_ws_routing, {f}));' for f in rfields]
     lines += ["  return 0;", "}"]
     src = tmp_path / "layout.c"
     src.write_text("\n".join(lines) + "\n")
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
     out = subprocess.check_output([str(exe)], text=True).split()
-    sizes, offs = [int(v) for v in out[:2]], [int(v) for v in out[2:]]
-    assert sizes == [ctypes.sizeof(moe.moe_layer_desc), ctypes.sizeof(moe.moe_weights)]
+    sizes, offs = [int(v) for v in out[:3]], [int(v) for v in out[3:]]
+    assert sizes == [ctypes.sizeof(moe.moe_layer_desc), ctypes.sizeof(moe.moe_weights),
+                     ctypes.sizeof(moe.moe_ws_routing)]
     py = [getattr(moe.moe_layer_desc, f).offset for f in fields] + \
-         [getattr(moe.moe_weights, f).offset for f in wfields]
+         [getattr(moe.moe_weights, f).offset for f in wfields] + \
+         [getattr(moe.moe_ws_routing, f).offset for f in rfields]
     assert offs == py
 
 

@@ -43,3 +43,27 @@ def test_prefill512_flops():
     assert bench.flops(W["prefill512"]) == 349_502_963_712
     # with adaptive top-p only the kept pairs count
     assert bench.flops(W["prefill512"], assignments=2048) == 6 * 2048 * 6144 * (2048 + 512) + 2 * 512 * 256 * 6144
+
+
+def test_region_count_covers_the_minimum_time():
+    assert bench.region_count(1.08, 0.5) == 463          # 20 decode steps of 54 us
+    assert bench.region_count(46.0, 0.5) == 11
+    assert bench.region_count(900.0, 0.5) == 3           # never fewer than three
+    assert bench.region_count(0.0, 0.5) >= 3
+
+
+def test_config_entry_figures():
+    w = W["decode8"]
+    ab = bench.algorithmic_bytes(w, 45)
+    r = {"w": w, "ab": ab, "ms_step": 0.2, "U": 45.0, "tflops": 1.0, "region_ms": [4.0] * 7,
+         "kernels_ms": {"layer": 0.19}, "roofline": {"peak": 6538.3}, "clocks": {},
+         "e2e": {"value": 30000.0}, "peaks": {}}
+    e = bench.config_entry(1, r, 20)
+    assert e["tokens_per_s"] == 8 / 0.2e-3
+    assert e["quantized_weight_gbs"] == ab["weights"] / 0.2e-3 / 1e9
+    assert e["frac_quantized_of_8tbs"] == e["quantized_weight_gbs"] / 8000.0
+    assert e["timed_regions"] == 7 and e["e2e_tokens_per_s"] == 30000.0
+    assert "tflops_frac_of_dense_fp16_peak" not in e
+    rp = dict(r, w=W["prefill512"], ab=bench.algorithmic_bytes(W["prefill512"], 228), ms_step=2.3,
+              tflops=150.0, peaks={"bf16_tflops": 1500.0})
+    assert bench.config_entry(1, rp, 20)["tflops_frac_of_dense_fp16_peak"] == 0.1

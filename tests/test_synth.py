@@ -92,3 +92,32 @@ def test_workload_tiny_layer_shapes():
     assert x.shape == (4, 256) and x.dtype == np.uint16
     part = synth.make_experts(w, experts=[3])
     assert np.array_equal(part["g"][3], L["g"][3]) and not part["g"][2].any()
+
+
+def test_stress_tokens_hold_the_promised_values():
+    w = synth.WORKLOADS["decode8"]
+    f = {k: synth.make_stress_tokens(w, 8, k).view(np.float16).astype(np.float64) for k in synth.STRESS_KINDS}
+    for k, v in f.items():
+        assert v.shape == (8, w.H) and np.isfinite(v).all(), k
+    a = np.abs(f["outlier"])
+    top = np.sort(a, axis=1)[:, -1]
+    assert np.all((top >= 2.0 ** 12) & (top < 2.0 ** 16))
+    assert np.all(np.sort(a, axis=1)[:, -3] < 8)              # at most two outliers per row
+    a = np.abs(f["near_max"])
+    assert np.all(a.max(axis=1) == 65504.0) and np.all((a == 65472.0).sum(axis=1) >= 1)
+    a = np.abs(f["subnormal"])
+    assert np.all((a > 0) & (a < 2.0 ** -14)) and np.all(a * 2.0 ** 24 == np.round(a * 2.0 ** 24))
+    a = np.abs(f["mixed"])
+    sub = (a > 0) & (a < 2.0 ** -14)
+    assert 0.15 < sub.mean() < 0.35
+    base = synth.make_tokens(w, 8).view(np.float16).astype(np.float64)
+    assert np.array_equal(f["mixed"][~sub], base[~sub])
+
+
+def test_scale_layer_scales_by_exact_powers_of_two():
+    w = synth.WORKLOADS["tiny"]
+    L = synth.make_layer(w)
+    S = synth.scale_layer(L, w.fmt, 2.0 ** -8, 2.0 ** 3, 2.0 ** 5)
+    assert np.array_equal(S["sg"], L["sg"] * np.float32(2.0 ** -8)) and np.array_equal(S["sh_su"], L["sh_su"] / 256)
+    assert np.array_equal(S["sd"], L["sd"] * 8) and np.array_equal(S["Wr"], L["Wr"] * 32)
+    assert S["g"] is L["g"] and np.array_equal(L["sg"], synth.make_layer(w)["sg"])   # input untouched

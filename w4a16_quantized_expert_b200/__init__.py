@@ -11,8 +11,7 @@ import ctypes
 import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-# W4A16_MOE_LIB selects another build of the same library (e.g. for A/B profiling)
-LIB_PATH = os.environ.get("W4A16_MOE_LIB") or os.path.join(PKG, "libmoe.so")
+LIB_PATH = os.path.join(PKG, "libmoe.so")
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1
@@ -51,6 +50,11 @@ class moe_weights(ctypes.Structure):
     _fields_ = [(f, vp) for f in WEIGHT_FIELDS]
 
 
+class moe_ws_routing(ctypes.Structure):
+    _fields_ = [(f, c_size) for f in ("logits", "topk_idx", "topk_w", "counts", "offsets", "perm", "unique",
+                                      "n_unique")]
+
+
 class MoeError(RuntimeError):
     def __init__(self, code: int, what: str):
         super().__init__(f"{what}: {status_string(code)} ({code})")
@@ -83,12 +87,14 @@ def lib():
         L.moe_combine.argtypes = [vp, vp, vp, vp, c_int, vp, vp]
         L.moe_forward.argtypes = [vp, vp, c_int, vp, vp, c_size, vp]
         L.moe_forward_host.argtypes = [vp, vp, c_int, vp, vp, c_size, vp]
-        L.moe_forward_timed.argtypes = [vp, vp, c_int, vp, vp, c_size, vp, ctypes.POINTER(vp)]
+        L.moe_forward_timed.argtypes = [vp, vp, c_int, vp, vp, c_size, vp, ctypes.POINTER(vp),
+                                        ctypes.POINTER(c_int)]
         L.moe_get_device_status.argtypes = [vp, ctypes.POINTER(c_int)]
         L.moe_debug_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
+        L.moe_workspace_routing.argtypes = [vp, c_int, ctypes.POINTER(moe_ws_routing)]
         for f in ("moe_layer_create", "moe_layer_destroy", "moe_route", "moe_route_static", "moe_group",
                   "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host", "moe_forward_timed",
-                  "moe_get_device_status", "moe_debug_wait_timeout"):
+                  "moe_get_device_status", "moe_debug_wait_timeout", "moe_workspace_routing"):
             getattr(L, f).restype = c_int
         _lib = L
     return _lib
@@ -159,8 +165,11 @@ def moe_forward_host(layer, x_host, T, y_host, ws, ws_bytes, stream=0):
 
 
 def moe_forward_timed(layer, x, T, y, ws, ws_bytes, stream, events):
+    """Returns (timed parts, kernels launched); see include/moe.h."""
     ev = (vp * 4)(*events)
-    _check(lib().moe_forward_timed(layer, x, T, y, ws, ws_bytes, stream, ev), "moe_forward_timed")
+    info = (c_int * 2)(0, 0)
+    _check(lib().moe_forward_timed(layer, x, T, y, ws, ws_bytes, stream, ev, info), "moe_forward_timed")
+    return int(info[0]), int(info[1])
 
 
 def moe_get_device_status(layer) -> int:
@@ -171,3 +180,10 @@ def moe_get_device_status(layer) -> int:
 
 def moe_debug_wait_timeout(layer, max_iters, stream=0):
     _check(lib().moe_debug_wait_timeout(layer, max_iters, stream), "moe_debug_wait_timeout")
+
+
+def moe_workspace_routing(layer, T) -> dict:
+    """Byte offsets of the routing and grouping arrays moe_forward leaves in the workspace."""
+    r = moe_ws_routing()
+    _check(lib().moe_workspace_routing(layer, T, ctypes.byref(r)), "moe_workspace_routing")
+    return {f: getattr(r, f) for f, _ in moe_ws_routing._fields_}

@@ -607,7 +607,7 @@ int moe_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void 
 }
 
 int moe_forward_timed(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void *ws, size_t ws_bytes,
-                      moe_stream_t stream, void *const events[4])
+                      moe_stream_t stream, void *const events[4], int info[2])
 {
     if (!L || T < 0 || T > L->desc.max_tokens) return MOE_ERR_INVALID_ARG;
     if (!events || !events[0] || !events[1] || !events[2] || !events[3]) return MOE_ERR_INVALID_ARG;
@@ -615,6 +615,10 @@ int moe_forward_timed(const moe_layer *L, const uint16_t *x, int T, uint16_t *y,
     if (!x || !y || !aligned16(x)) return MOE_ERR_INVALID_ARG;
     int rc = check_ws(L, T, ws, ws_bytes);
     if (rc) return rc;
+    if (info) {
+        info[0] = 3;   // router | gate/up | down + combine
+        info[1] = 4;
+    }
     return run_forward(L, x, T, y, ws, reinterpret_cast<cudaStream_t>(stream), events);
 }
 
@@ -644,6 +648,21 @@ int moe_get_device_status(const moe_layer *L, int *status)
     if (cudaMemcpy(&v, L->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaMemset(L->d_status, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
     *status = v;
+    return MOE_OK;
+}
+
+int moe_workspace_routing(const moe_layer *L, int T, moe_ws_routing *out)
+{
+    if (!L || !out || T < 1 || T > L->desc.max_tokens) return MOE_ERR_INVALID_ARG;
+    const Ws W = ws_layout(L->desc, T);
+    out->logits = W.logits;
+    out->topk_idx = W.topk_idx;
+    out->topk_w = W.topk_w;
+    out->counts = W.counts;
+    out->offsets = W.offsets;
+    out->perm = W.perm;
+    out->unique = W.unique;
+    out->n_unique = W.n_unique;
     return MOE_OK;
 }
 

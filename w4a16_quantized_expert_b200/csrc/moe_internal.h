@@ -24,7 +24,7 @@ constexpr size_t kStaticRouteScore = 256;
 constexpr size_t kStaticRouteSel = kStaticRouteScore + (size_t)kStaticRouteElems * 4;
 constexpr size_t kStaticRouteLogits = kStaticRouteSel + (size_t)kStaticRouteElems * 4;
 constexpr size_t kStaticRouteBytes = kStaticRouteLogits + (size_t)kStaticRouteElems * 4;
-constexpr int kStaticRouteDevices = 64;   // device ordinals whose scratch address is cached
+constexpr int kStaticRouteContexts = 64;   // CUDA contexts whose scratch address is cached
 constexpr int kRowTile = 16;           // output rows per expert work item (mma M)
 constexpr int kTokChunk = 32;          // tokens per expert work item (4 mma N-tiles)
 

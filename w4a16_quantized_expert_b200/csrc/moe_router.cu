@@ -17,6 +17,8 @@
 // the grouping.  Counters are reset by the CTA that consumes them (atomicInc wraps).
 // The kernel releases its programmatic dependents at once: the expert kernel starts the
 // shared expert while routing is still running.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 #include <math.h>
 
@@ -866,20 +868,70 @@ cudaError_t launch_x_limbs(const uint16_t *x, int T, int H, unsigned char *limbs
 // complete call (atomicInc wraps), the float arrays are written before they are read.
 static __device__ __align__(256) unsigned char g_route_scratch[kStaticRouteBytes];
 
+// The array's device address belongs to the CUDA context that loaded this module: a
+// context created later (after cudaDeviceReset, or a driver-API context of the caller)
+// has its own copy at another address.  The address is therefore cached per context,
+// keyed by the context's process-unique id (cuCtxGetId), never by device ordinal.
+namespace {
+struct CtxFns {
+    PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    PFN_cuCtxGetId_v12000 get_id = nullptr;
+    bool ok = false;
+};
+
+const CtxFns &ctx_fns()
+{
+    static CtxFns f = [] {
+        CtxFns r;
+        cudaDriverEntryPointQueryResult q;
+        void *a = nullptr, *b = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess) {
+            r.get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(a);
+            r.get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(b);
+            r.ok = true;
+        }
+        return r;
+    }();
+    return f;
+}
+}  // namespace
+
 cudaError_t static_route_scratch(void **ptr)
 {
     static std::mutex mu;
-    static void *addr[kStaticRouteDevices] = {};
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kStaticRouteDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        e = cudaGetSymbolAddress(&addr[dev], g_route_scratch);
+    static unsigned long long ids[kStaticRouteContexts] = {};
+    static void *addr[kStaticRouteContexts] = {};
+    static int next = 0;
+    const CtxFns &f = ctx_fns();
+    if (!f.ok) return cudaErrorNotSupported;
+    CUcontext ctx = nullptr;
+    if (f.get_current(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
+    if (!ctx) {
+        // no context is current on this thread yet: the runtime call creates (and makes
+        // current) the device's primary context, whose id is taken below
+        void *a = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&a, g_route_scratch);
         if (e != cudaSuccess) return e;
+        if (f.get_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorUnknown;
     }
-    *ptr = addr[dev];
+    unsigned long long id = 0;
+    if (f.get_id(ctx, &id) != CUDA_SUCCESS) return cudaErrorUnknown;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < kStaticRouteContexts; ++i)
+        if (addr[i] && ids[i] == id) {
+            *ptr = addr[i];
+            return cudaSuccess;
+        }
+    void *a = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&a, g_route_scratch);
+    if (e != cudaSuccess) return e;
+    ids[next] = id;   // the oldest entry gives way when every slot is taken
+    addr[next] = a;
+    next = (next + 1) % kStaticRouteContexts;
+    *ptr = a;
     return cudaSuccess;
 }
 
