@@ -120,7 +120,7 @@ def kernel_hash() -> str:
     stays attached to exactly the code it measured."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "w4a16_quantized_expert_b200", "csrc")
-    for f in ("moe_device.cuh", "moe_internal.h", "moe_ffn.cu"):
+    for f in ("moe_device.cuh", "moe_internal.h", "moe_expert.cuh", "moe_ffn.cu"):
         txt = open(os.path.join(csrc, f), "rb").read()
         if f == "moe_ffn.cu":
             a = txt.find(b"// ============================================================================ tcgen05 path")
@@ -539,6 +539,33 @@ def bench_config(args, w, world, dev, stream, host=None, want_e2e=True):
         assert st == moe.MOE_OK, moe.status_string(st)
         del ge, ge_rem
 
+    # ---- the one-launch decode path on the same layers and tokens (T <= 16)
+    fused = None
+    if w.T <= 16 and not args.no_fused:
+        def fwd_fused(i):
+            layers[i].forward(xs[i], ws, y=ys[i], stream=stream, fused=True)
+
+        with torch.cuda.stream(stream):
+            for i in range(R):
+                fwd_fused(i)
+        torch.cuda.synchronize(dev)
+        gf = capture(fwd_fused, R)
+        gf_rem = capture(fwd_fused, rem) if rem else None
+        with torch.cuda.stream(stream):
+            for _ in range(max(1, (Wm + R - 1) // R)):
+                gf.replay()
+        torch.cuda.synchronize(dev)
+        f_ms = timed_regions(steps(gf, gf_rem), world, dev, stream, args.min_region_s / 2)
+        f_step = max_over_ranks(world, float(np.median(f_ms))) / K
+        st = moe.moe_get_device_status(base.handle)
+        assert st == moe.MOE_OK, moe.status_string(st)
+        fq = ab["weights"] / (f_step * 1e-3) / 1e9
+        fused = {"ms_per_layer": f_step, "tokens_per_s": job_tokens_per_s(world, K, w.T, f_step * K),
+                 "quantized_weight_gbs": fq, "frac_quantized_of_8tbs": fq / 8000.0,
+                 "timed_regions": len(f_ms), "launches_per_step": 1,
+                 "how": "moe_forward_fused (router, experts and combine in one persistent launch)"}
+        del gf, gf_rem
+
     tflops = flops(w, A_mean) / (ms_step * 1e-3) / 1e12
     out = {
         "w": w, "host": host, "ms_step": ms_step, "region_ms": region_ms, "R": R, "U": U_mean,
@@ -550,7 +577,7 @@ def bench_config(args, w, world, dev, stream, host=None, want_e2e=True):
             "algorithmic_bytes_per_launch": kbytes[dom],
             "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] == "measured" else "fallback",
         },
-        "e2e": e2e, "clocks": clocks.summary(t_wall0, t_wall1), "peaks": peaks,
+        "e2e": e2e, "clocks": clocks.summary(t_wall0, t_wall1), "peaks": peaks, "fused": fused,
         "timed_region_s": float(np.sum(region_ms)) / 1000.0,
     }
     del g_full, g_rem, gk
@@ -584,6 +611,8 @@ def config_entry(world, r, K) -> dict:
         e["dense_peak_tflops"] = pk
     if r["e2e"]:
         e["e2e_tokens_per_s"] = r["e2e"]["value"]
+    if r.get("fused"):
+        e["fused_path"] = r["fused"]
     return e
 
 
@@ -660,6 +689,7 @@ def run_ours(args, w):
         "gpu_launches": head["launches_per_step"] * K * len(head["region_ms"]),
         "clocks": head["clocks"],
         "cpu_baseline": cpu,
+        "fused_path": head["fused"],
         "configs": {name: config_entry(world, r, K) for name, r in extras.items()},
     }
     print(json.dumps(line), flush=True)
@@ -681,6 +711,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="measure the chosen workload only (no other configurations in the line)")
+    ap.add_argument("--no-fused", action="store_true",
+                    help="do not also time the one-launch decode path (moe_forward_fused)")
     ap.add_argument("--min-region-s", type=float, default=MIN_REGION_S,
                     help="repeat each timed region of K steps until they add up to this")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -242,6 +242,24 @@ int moe_combine(const moe_layer *layer, const float *y_assign, const float *y_sh
 int moe_forward(const moe_layer *layer, const uint16_t *x, int T, uint16_t *y,
                 void *workspace, size_t workspace_bytes, moe_stream_t stream);
 
+/* Source: as moe_forward (routing fused into the small-batch kernels, one replayed unit per
+ * decode step), taken to one launch.
+ * moe_forward for decode-sized batches (1 <= T <= 16) in ONE persistent launch: router
+ * GEMV, top-k, grouping, gate/up, down and the combine run as one ordered list of work
+ * items, with flags (not grid barriers) between the steps -- the expert weights of the
+ * shared expert stream while routing runs, down items of an expert start while other
+ * experts' gate/up items still run, and each 64-row output tile is combined by the CTA
+ * whose down item completes it.  The routing (logits, top-k, weights, grouping) is the
+ * same bits as moe_forward's.  With int4 weights y is moe_forward's y bit for bit (the
+ * same exact integer sums, the same epilogue and combine order); with NVFP4 the fp32 sums
+ * may run in another order (moe_forward splits K across warps for small layers), within
+ * the layer's tolerance.  Returns MOE_ERR_UNSUPPORTED for T > 16 (and MOE_OK for T = 0).
+ * The grid holds two CTAs per SM and its CTAs wait for one another's flags (bounded waits,
+ * MOE_ERR_DEVICE_TIMEOUT if one gives up): do not run it beside another kernel that keeps
+ * SMs occupied for good. */
+int moe_forward_fused(const moe_layer *layer, const uint16_t *x, int T, uint16_t *y,
+                      void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
 /* moe_forward with HOST activations: enqueues the host->device copy of x_host, the
  * layer and the device->host copy into y_host on the stream (x and y are staged in the
  * workspace).  Returns once enqueued; synchronise the stream before reading y_host.

@@ -21,6 +21,10 @@ activations at the edges of the fp16 range.
    tensor-memory kernel (T = 40) and the NVFP4 path.  The layer's weights are scaled by
    powers of two (synth.scale_layer) so that h and y stay inside the fp16 range; the test
    checks that on the oracle's values first.
+
+3. The one-launch decode path (moe_forward_fused): its own routing and grouping read back
+   the same way, the whole layer against the oracle and against moe_forward (bit for bit
+   with int4 weights), edge-case activations, guard bands and the T > 16 rejection.
 """
 import numpy as np
 import pytest
@@ -70,7 +74,7 @@ GROUP_CASES = [("decode1", 1, 0.0), ("tiny", 4, 0.0), ("decode8", 8, 0.0), ("nvf
 
 
 @pytest.mark.parametrize("name,T,p", GROUP_CASES)
-def test_fused_routing_and_grouping_match_the_oracle(name, T, p):
+def test_forward_routing_and_grouping_match_the_oracle(name, T, p):
     w = _workload(name)
     if p:
         w = w.with_(top_p=p)
@@ -171,4 +175,114 @@ def test_forward_activation_edge_cases(name, T, kind):
     excluded, err = check_y(y_to_f64(y), ref["y"], ref["gap"])
     assert excluded < T, "every token excluded as a near tie"
     print(f"{name} {kind}: excluded {excluded}/{T}, rel err {err:.3g}")
+    dev.close()
+
+
+# ------------------------------------------------------------------ one-launch decode path
+@pytest.mark.parametrize("name,T,p", [("decode1", 1, 0.0), ("tiny", 4, 0.0), ("decode8", 8, 0.0),
+                                      ("nvfp4_16", 16, 0.0), ("tiny", 16, 0.0), ("decode8", 8, 0.7),
+                                      ("tiny", 4, 0.5), ("tiny_e1024", 9, 0.0)])
+def test_fused_path_routing_and_grouping_match_the_oracle(name, T, p):
+    """moe_forward_fused routes and groups in its own router tasks and finishing task."""
+    w = _workload(name)
+    if p:
+        w = w.with_(top_p=p)
+    host = synth.make_layer(w, experts=[0])
+    desc = desc_of(w)
+    dev = DeviceLayer(desc, host, max_tokens=T)
+    x = synth.make_tokens(w, T)
+    ws = dev.workspace(T)
+    dev.forward(torch.from_numpy(x.copy()).cuda(), ws, fused=True)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(dev.handle) == moe.MOE_OK
+    _check_routing_arrays(ws_routing(dev, ws, T), host, desc, x, w)
+    dev.close()
+
+
+FUSED_CASES = [("tiny", 1), ("tiny", 2), ("tiny", 3), ("tiny", 4), ("tiny", 9), ("tiny", 15), ("tiny", 16),
+               ("decode1", 1), ("decode8", 8), ("nvfp4_1", 1), ("nvfp4_16", 16)]
+
+
+@pytest.mark.parametrize("name,T", FUSED_CASES)
+def test_fused_forward_matches_the_oracle_and_moe_forward(name, T):
+    """The whole layer in one launch against the FP64 oracle, and against moe_forward: bit
+    for bit with int4 weights, within tolerance with NVFP4; run twice (counters and flags
+    left ready for the next call)."""
+    w = W[name]
+    x = synth.make_tokens(w, T, batch=T)
+    if name == "tiny":
+        host = synth.make_layer(w)
+    else:
+        logits = oracle.default().router_logits(x, synth.make_router(w)[0])
+        _, _, sel, _ = oracle.default().route(logits, synth.make_router(w)[1], w.k, w.scaling)
+        host = synth.make_layer(w, experts=np.unique(np.argsort(-sel, axis=1, kind="stable")[:, : w.k + 2]))
+    desc = desc_of(w)
+    dev = DeviceLayer(desc, host, max_tokens=max(T, 16))
+    xd = torch.from_numpy(x.copy()).cuda()
+    ws = dev.workspace(T)
+    y_ref = dev.forward(xd, ws)
+    for _ in range(2):
+        y = dev.forward(xd, ws, fused=True)
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_status(dev.handle) == moe.MOE_OK
+        if w.fmt == synth.FMT_INT4:
+            assert torch.equal(y, y_ref), "fused path differs from moe_forward"
+        ref = oracle.default().forward(desc, host, x)
+        excluded, err = check_y(y_to_f64(y), ref["y"], ref["gap"])
+    print(f"{name} T={T} fused: excluded {excluded}/{T}, rel err {err:.3g}")
+    dev.close()
+
+
+@pytest.mark.parametrize("name,T,kind", [("decode1", 1, "outlier"), ("decode1", 1, "subnormal"),
+                                         ("decode8", 8, "near_max"), ("nvfp4_1", 1, "outlier")])
+def test_fused_forward_activation_edge_cases(name, T, kind):
+    w = W[name]
+    fgu, fd, fr = FACTORS[kind]
+    if kind == "subnormal" and w.fmt == synth.FMT_NVFP4:
+        fgu *= 8.0
+    x = synth.make_stress_tokens(w, T, kind)
+    Wr, bias = synth.make_router(w)
+    o = oracle.default()
+    logits = o.router_logits(x, synth.scale_layer({"Wr": Wr}, w.fmt, 1.0, 1.0, fr)["Wr"])
+    _, _, sel, _ = o.route(logits, bias, w.k, w.scaling)
+    host = {"Wr": Wr, "bias": bias}
+    host.update(synth.make_experts(w, np.unique(np.argsort(-sel, axis=1, kind="stable")[:, : w.k + 2])))
+    host = synth.scale_layer(host, w.fmt, fgu, fd, fr)
+    desc = desc_of(w)
+    ref = o.forward(desc, host, x)
+    dev = DeviceLayer(desc, host, max_tokens=T)
+    ws = dev.workspace(T)
+    y = dev.forward(torch.from_numpy(x.copy()).cuda(), ws, fused=True)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(dev.handle) == moe.MOE_OK
+    excluded, err = check_y(y_to_f64(y), ref["y"], ref["gap"])
+    assert excluded < T
+    dev.close()
+
+
+def test_fused_forward_stays_inside_its_buffers_and_rejects_large_batches():
+    w = W["tiny"]
+    T = 16
+    host = synth.make_layer(w)
+    dev = DeviceLayer(desc_of(w), host, max_tokens=32)
+    n = moe.moe_workspace_size(dev.handle, T)
+    G = 4096
+    buf = torch.full((G + n + G,), 0xA5, dtype=torch.uint8, device="cuda")
+    ws = buf[G:G + n]
+    ws.zero_()
+    x = torch.from_numpy(synth.make_tokens(w, T).copy()).cuda()
+    yb = torch.full((T + 2, w.H), 0x5A5A, dtype=torch.int16, device="cuda").view(torch.uint16)
+    for _ in range(3):
+        dev.forward(x, ws, y=yb[1:T + 1], fused=True)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(dev.handle) == moe.MOE_OK
+    b = buf.cpu().numpy()
+    assert np.all(b[:G] == 0xA5) and np.all(b[G + n:] == 0xA5), "write outside the workspace"
+    yh = yb.view(torch.int16).cpu().numpy()
+    assert np.all(yh[0] == 0x5A5A) and np.all(yh[T + 1] == 0x5A5A), "write outside y"
+    x17 = torch.from_numpy(synth.make_tokens(w, 17).copy()).cuda()
+    ws17 = dev.workspace(17)
+    with pytest.raises(moe.MoeError) as e:
+        dev.forward(x17, ws17, fused=True)
+    assert e.value.code == moe.MOE_ERR_UNSUPPORTED
     dev.close()

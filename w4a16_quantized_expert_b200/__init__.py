@@ -86,6 +86,7 @@ def lib():
         L.moe_expert_ffn.argtypes = [vp, vp, c_int, vp, vp, vp, vp, vp, c_size, vp]
         L.moe_combine.argtypes = [vp, vp, vp, vp, c_int, vp, vp]
         L.moe_forward.argtypes = [vp, vp, c_int, vp, vp, c_size, vp]
+        L.moe_forward_fused.argtypes = [vp, vp, c_int, vp, vp, c_size, vp]
         L.moe_forward_host.argtypes = [vp, vp, c_int, vp, vp, c_size, vp]
         L.moe_forward_timed.argtypes = [vp, vp, c_int, vp, vp, c_size, vp, ctypes.POINTER(vp),
                                         ctypes.POINTER(c_int)]
@@ -93,7 +94,7 @@ def lib():
         L.moe_debug_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
         L.moe_workspace_routing.argtypes = [vp, c_int, ctypes.POINTER(moe_ws_routing)]
         for f in ("moe_layer_create", "moe_layer_destroy", "moe_route", "moe_route_static", "moe_group",
-                  "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host", "moe_forward_timed",
+                  "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_fused", "moe_forward_host", "moe_forward_timed",
                   "moe_get_device_status", "moe_debug_wait_timeout", "moe_workspace_routing"):
             getattr(L, f).restype = c_int
         _lib = L
@@ -157,6 +158,10 @@ def moe_combine(layer, y_assign, y_shared, topk_w, T, y, stream=0):
 
 def moe_forward(layer, x, T, y, ws, ws_bytes, stream=0):
     _check(lib().moe_forward(layer, x, T, y, ws, ws_bytes, stream), "moe_forward")
+
+
+def moe_forward_fused(layer, x, T, y, ws, ws_bytes, stream=0):
+    _check(lib().moe_forward_fused(layer, x, T, y, ws, ws_bytes, stream), "moe_forward_fused")
 
 
 def moe_forward_host(layer, x_host, T, y_host, ws, ws_bytes, stream=0):

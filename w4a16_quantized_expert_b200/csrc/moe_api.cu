@@ -24,6 +24,8 @@ cudaError_t ffn_prepare(int fmt, int E, int occ[2][2][2]);
 cudaError_t tc_prepare(int E);
 cudaError_t launch_tc(const LayerMaps &maps, const FfnParams &p, bool gate_up, int grid, bool pdl, cudaStream_t s);
 cudaError_t launch_wait_timeout(int *status, unsigned long long max_iters, cudaStream_t s);
+cudaError_t fused_prepare(int fmt, int *blocks_per_sm);
+cudaError_t launch_fused(const LayerMaps &maps, const FusedParams &p, int grid, bool pdl, cudaStream_t s);
 
 namespace {
 
@@ -34,7 +36,8 @@ size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
 // The counter block sits first and depends only on the handle, so counters keep their
 // place (and their zero value) whatever T successive calls use.
 struct Ws {
-    size_t ctr_tiles, ctr_group, ctr_work, ctr_chunks, h_amax, zrow, ctr_end;
+    size_t ctr_tiles, ctr_group, ctr_work, ctr_chunks, h_amax, f_ctl, f_chunk_ctr, f_chunk_flag, f_tile_ctr, zrow,
+        ctr_end;
     size_t logits, score, sel, topk_idx, topk_w, counts, offsets, perm, unique, n_unique, slots;
     size_t x_perm, h, h_sh, y_assign, y_shared, x_stage, y_stage;
     size_t x_limbs, x_limb_scale, h_limbs, h_limb_scale, hsh_limbs, hsh_limb_scale, total;
@@ -68,6 +71,14 @@ Ws ws_layout(const moe_layer_desc &d, int T)
     w.ctr_work = o; o += 4 * 4;
     w.ctr_chunks = o; o += (size_t)d.max_tokens * (d.top_k + 1) * 4;
     w.h_amax = o; o += (size_t)d.max_tokens * (d.top_k + 1) * 4;
+    // the one-launch decode layer: control words, per-chunk counters and flags, per-tile
+    // counters, each word in a 128-byte line of its own
+    o = up256(o);
+    const size_t fchunks = (size_t)std::min(d.max_tokens, kFusedMaxT) * (d.top_k + 1);
+    w.f_ctl = o; o += 8 * kSyncLine * 4;
+    w.f_chunk_ctr = o; o += fchunks * kSyncLine * 4;
+    w.f_chunk_flag = o; o += fchunks * kSyncLine * 4;
+    w.f_tile_ctr = o; o += (size_t)((d.hidden + 63) / 64) * kSyncLine * 4;
     o = up256(o);
     // a row of zeros read by padding token columns (never written)
     w.zrow = o; o = up256(o + (size_t)std::max(d.hidden, std::max(d.inter, d.inter_shared)) * 2);
@@ -302,6 +313,66 @@ Launch ffn_launch(const moe_layer *L, int T, bool gu)
     return {4, L->num_sms * L->occ[wide][gu][1]};
 }
 
+// The decode-sized layer in one launch (moe_fused.cu).
+bool use_fused(int T) { return T >= 1 && T <= kFusedMaxT; }
+
+int run_fused(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s,
+              void *const *events)
+{
+    const moe_layer_desc &d = L->desc;
+    const Ws W = ws_layout(d, T);
+    FusedParams p = {};
+    p.dk = {0x000F000Fu, 0x00F000F0u, 0x64086408u, 0x64806480u, 0x64086408u, 0x2C002C00u, 0xD480D480u};
+    p.T = T;
+    p.H = d.hidden;
+    p.I = d.inter;
+    p.I_sh = d.inter_shared;
+    p.E = d.n_experts;
+    p.k = d.top_k;
+    p.n_shared = d.n_shared;
+    p.fmt = d.format;
+    p.scaling = d.routed_scaling;
+    p.top_p = (d.top_p > 0.f && d.top_p < 1.f) ? d.top_p : 0.f;
+    p.x = x;
+    p.y = y;
+    p.wt = layer_weights(L);
+    p.logits = at<float>(ws, W.logits);
+    p.score = at<float>(ws, W.score);
+    p.sel = at<float>(ws, W.sel);
+    p.topk_idx = at<int32_t>(ws, W.topk_idx);
+    p.topk_w = at<float>(ws, W.topk_w);
+    p.counts = at<int32_t>(ws, W.counts);
+    p.offsets = at<int32_t>(ws, W.offsets);
+    p.perm = at<int32_t>(ws, W.perm);
+    p.unique = at<int32_t>(ws, W.unique);
+    p.n_unique = at<int32_t>(ws, W.n_unique);
+    p.slots = at<int4>(ws, W.slots);
+    p.x_limbs = at<unsigned char>(ws, W.x_limbs);
+    p.x_limb_scale = at<float>(ws, W.x_limb_scale);
+    p.h = at<__half>(ws, W.h);
+    p.h_sh = at<__half>(ws, W.h_sh);
+    p.h_limbs = at<unsigned char>(ws, W.h_limbs);
+    p.h_limb_scale = at<float>(ws, W.h_limb_scale);
+    p.hsh_limbs = at<unsigned char>(ws, W.hsh_limbs);
+    p.hsh_limb_scale = at<float>(ws, W.hsh_limb_scale);
+    p.h_amax = at<unsigned int>(ws, W.h_amax);
+    p.y_assign = at<float>(ws, W.y_assign);
+    p.y_shared = at<float>(ws, W.y_shared);
+    p.zrow = at<uint16_t>(ws, W.zrow);
+    p.ctl = at<unsigned int>(ws, W.f_ctl);
+    p.chunk_ctr = at<unsigned int>(ws, W.f_chunk_ctr);
+    p.chunk_flag = at<unsigned int>(ws, W.f_chunk_flag);
+    p.tile_ctr = at<unsigned int>(ws, W.f_tile_ctr);
+    p.status = L->d_status;
+    const bool pdl = events == nullptr;
+    if (events) cudaEventRecordWithFlags(reinterpret_cast<cudaEvent_t>(events[0]), s, cudaEventRecordExternal);
+    const cudaError_t e = launch_fused(L->maps, p, L->num_sms * L->occ_fused, pdl, s);
+    if (events)
+        for (int i = 1; i < 4; ++i)
+            cudaEventRecordWithFlags(reinterpret_cast<cudaEvent_t>(events[i]), s, cudaEventRecordExternal);
+    return cuda_status(e);
+}
+
 int run_forward(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s,
                 void *const *events = nullptr)
 {
@@ -438,7 +509,8 @@ int moe_layer_create(const moe_layer_desc *desc, const moe_weights *weights, moe
         return MOE_ERR_CUDA;
     }
     bool occ_ok = router_prepare() == cudaSuccess && ffn_prepare(d.format, d.n_experts, L->occ) == cudaSuccess &&
-                  (d.format != MOE_FMT_INT4_ROWSCALE || tc_prepare(d.n_experts) == cudaSuccess);
+                  (d.format != MOE_FMT_INT4_ROWSCALE || tc_prepare(d.n_experts) == cudaSuccess) &&
+                  fused_prepare(d.format, &L->occ_fused) == cudaSuccess && L->occ_fused >= 1;
     for (int a = 0; a < 2; ++a)
         for (int b = 0; b < 2; ++b)
             for (int c = 0; c < 2; ++c) occ_ok = occ_ok && L->occ[a][b][c] >= 1;
@@ -620,6 +692,18 @@ int moe_forward_timed(const moe_layer *L, const uint16_t *x, int T, uint16_t *y,
         info[1] = 4;
     }
     return run_forward(L, x, T, y, ws, reinterpret_cast<cudaStream_t>(stream), events);
+}
+
+int moe_forward_fused(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void *ws, size_t ws_bytes,
+                      moe_stream_t stream)
+{
+    if (!L || T < 0 || T > L->desc.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!use_fused(T)) return MOE_ERR_UNSUPPORTED;
+    if (!x || !y || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+    int rc = check_ws(L, T, ws, ws_bytes);
+    if (rc) return rc;
+    return run_fused(L, x, T, y, ws, reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
 int moe_forward_host(const moe_layer *L, const uint16_t *x_host, int T, uint16_t *y_host, void *ws,

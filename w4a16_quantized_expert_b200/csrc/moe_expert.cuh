@@ -1,0 +1,238 @@
+// moe_expert.cuh -- pieces of the expert kernels shared by the per-step kernels
+// (moe_ffn.cu) and the fused decode-layer kernel (moe_fused.cu): ring geometry, the
+// int4 / NVFP4 chunk-pair inner loops on the warp MMAs, the consumer barrier and the
+// conversion of finished h rows to int8 limbs.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <math.h>
+
+#include "moe_device.cuh"
+#include "moe_internal.h"
+
+#ifndef MOE_CHAINS
+#define MOE_CHAINS 1
+#endif
+#ifndef MOE_MIN_CTAS
+#define MOE_MIN_CTAS 2
+#endif
+
+namespace moe {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kFfnThreads = (kConsumerWarps + 1) * 32;
+constexpr int kBoxBytes = 128;          // K bytes per TMA box = swizzle span
+constexpr int kBoxSmem = kRowTile * kBoxBytes;     // 2 KB
+constexpr int kScaleBoxBytes = kBoxBytes / 8;      // NVFP4: one E4M3 per 16 weights = 16 B
+constexpr int kScaleBoxSmem = kRowTile * kScaleBoxBytes;   // 256 B
+constexpr int kMatStage = kConsumerWarps * kBoxSmem;       // 8 KB of codes per matrix
+
+template <int FMT, bool GU, int KS, int NNMAX>
+struct FfnCfg {
+    static constexpr int kMats = GU ? 2 : 1;
+    static constexpr int kRW = kConsumerWarps / KS;
+    static constexpr bool kNv = FMT == MOE_FMT_NVFP4;
+    static constexpr int kStageK = KS * kBoxBytes;        // K bytes per stage
+    static constexpr int kCodeBytes = kMats * kMatStage;
+    static constexpr int kScaleBytes = kNv ? kMats * kConsumerWarps * kScaleBoxSmem : 0;
+    // int4 decode variant: the int8 tensor path (weights as s8 bytes, activations as
+    // three int8 limbs; items of at most 8 tokens, KS = 1)
+    static constexpr bool kLimbs = FMT == MOE_FMT_INT4_ROWSCALE && NNMAX == 1 && KS == 1;
+    // decode variant: the producer also copies each stage's slice of the (up to 8) token
+    // rows of the B operand into shared memory, one row per token: fp16 values padded to
+    // 16 bytes, or one 768-byte limb block (the stage's 256 K values, three limbs)
+    static constexpr bool kSmemB = NNMAX == 1 && KS == 1;
+    static constexpr int kBRow = kLimbs ? kLimbBlockBytes : 4 * kStageK + 16;
+    static constexpr int kBBytes = kSmemB ? 8 * kBRow : 0;      // per stage, after the ring (at most)
+    static constexpr int kStageBytes = ((kCodeBytes + kScaleBytes) + 1023) / 1024 * 1024;
+    // Ring depth.  Weights in flight per SM decide the bandwidth (DRAM latency under full
+    // load is about 2.5 us); the int8 path sizes its ring at launch (up to kStagesMax
+    // stages, as many as fit beside a second CTA on the SM, given the B rows per stage).
+    static constexpr int kStages = GU ? (kSmemB ? 3 : 4) : 5;
+    static constexpr int kStagesCap = kLimbs ? (GU ? 6 : 12) : kStages;
+    static constexpr int kZeroRow = kSmemB ? kBRow : 0;   // zero row read by padding lanes
+    static constexpr int kRedFloats = KS > 1 ? kConsumerWarps * kMats * kTokChunk * kRowTile : 0;
+};
+
+constexpr int kStagesMax = 16;   // ring stages any launch may use (mbarrier slots)
+constexpr int kItemQ = 4;        // work items the producer may announce ahead of the consumers
+constexpr int kMaxConvRows = 64; // h rows one conversion handles (tokens of a work item)
+
+// dynamic shared memory of one CTA: ring (weights, then B rows) + zero row + reduction +
+// slot table + header/barriers
+template <int FMT, bool GU, int KS, int NNMAX>
+__host__ __device__ constexpr size_t ffn_smem(int E, int stages, int b_stage)
+{
+    using C = FfnCfg<FMT, GU, KS, NNMAX>;
+    return 1024 + (size_t)stages * (C::kStageBytes + b_stage) + C::kZeroRow + (size_t)C::kRedFloats * 4 +
+           (size_t)4 * 4 * (E + 2) + 64 + 8 + (2 * kStagesMax + 1 + 2 * kItemQ) * 8;
+}
+
+
+// position of h column n inside its 8-column group, in the order the down kernel's
+// B fragments want it (int4: pairs (0,4)(1,5)(2,6)(3,7); NVFP4: natural order)
+template <int FMT>
+__device__ __forceinline__ int h_pos(int n)
+{
+    if (FMT == MOE_FMT_NVFP4) return n;
+    const int m = n & 7;
+    return (n & ~7) | ((m & 3) << 1) | (m >> 2);
+}
+
+// named barrier of the four consumer warps (the producer warp never joins it); NT: the
+// threads that meet there (the tensor-memory kernel's converter warps use it too)
+template <int NT = kConsumerWarps * 32, int ID = 1>
+__device__ __forceinline__ void consumer_sync()
+{
+    asm volatile("bar.sync %0, %1;" ::"n"(ID), "r"(NT) : "memory");
+}
+
+// int4: the fp32 scale of row `row`; NVFP4: the fp32 scale of the whole matrix
+template <int FMT>
+__device__ __forceinline__ float mat_scale(const float *scales, int e, int rows, int row)
+{
+    const int ez = e < 0 ? 0 : e;
+    if (FMT == MOE_FMT_NVFP4) return scales[ez];
+    return scales[(size_t)ez * rows + row];
+}
+
+// Per-thread constants of a consumer warp.
+struct Lane {
+    int lane, g, tq, warp, rw, ks, bx;
+    uint32_t off[4];   // swizzled ldmatrix offsets of chunk pairs 0..3 inside a box
+    DequantK dk;
+};
+
+// B-operand row of each of a thread's four n-tiles
+struct BRows {
+    const uint16_t *r[4];
+};
+
+// One chunk pair (64 weights of each of the warp's 16 rows and of each matrix): ldmatrix,
+// dequantise in registers, NN n-tiles of mma.  X0/X1 hold the n-tile-0 B fragments.
+// independent accumulator chains per (matrix, n-tile): mma.sync results feed the next
+// mma on the same accumulator, so one chain per matrix would serialise a stage's 16 mma
+template <int NN>
+struct Chains {
+    static constexpr int P = MOE_CHAINS;
+};
+
+template <int FMT, bool GU, int KS, int NN, bool PERM>
+__device__ __forceinline__ void chunk_pair(const unsigned char *st, uint32_t abase, const Lane &L, int q, int kel,
+                                           const uint4 &X0, const uint4 &X1, const BRows &brow,
+                                           float (&acc)[GU ? 2 : 1][NN][Chains<NN>::P][4])
+{
+    using C = FfnCfg<FMT, GU, KS, 1>;   // the values used here do not depend on NNMAX
+    uint32_t A[C::kMats][2][2][4];   // [mat][chunk][row g / g+8][pairs]
+#pragma unroll
+    for (int m = 0; m < C::kMats; ++m) {
+        uint32_t r0, r1, r2, r3;
+        ldmatrix_x4(r0, r1, r2, r3, abase + m * kMatStage + L.off[q]);
+        if constexpr (C::kNv) {
+            const unsigned char *sc = st + C::kCodeBytes + (m * kConsumerWarps + L.bx) * kScaleBoxSmem;
+            const int b0 = 4 * q + (L.tq >> 1);       // block of (chunk 2q, word tq)
+            const uint32_t s00 = e4m3_to_half2(sc[L.g * kScaleBoxBytes + b0]);
+            const uint32_t s10 = e4m3_to_half2(sc[(L.g + 8) * kScaleBoxBytes + b0]);
+            const uint32_t s01 = e4m3_to_half2(sc[L.g * kScaleBoxBytes + b0 + 2]);
+            const uint32_t s11 = e4m3_to_half2(sc[(L.g + 8) * kScaleBoxBytes + b0 + 2]);
+            dequant_nvfp4_word(r0, s00, A[m][0][0]);
+            dequant_nvfp4_word(r1, s10, A[m][0][1]);
+            dequant_nvfp4_word(r2, s01, A[m][1][0]);
+            dequant_nvfp4_word(r3, s11, A[m][1][1]);
+        } else {
+            dequant_int4_word(r0, A[m][0][0], L.dk);
+            dequant_int4_word(r1, A[m][0][1], L.dk);
+            dequant_int4_word(r2, A[m][1][0], L.dk);
+            dequant_int4_word(r3, A[m][1][1], L.dk);
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < NN; ++n) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const uint4 X = n == 0 ? (c == 0 ? X0 : X1)
+                                   : __ldg(reinterpret_cast<const uint4 *>(brow.r[n] + kel + 32 * c + 8 * L.tq));
+            uint32_t b00, b01, b10, b11;
+            if constexpr (PERM) {
+                b00 = pack_lo(X.x, X.z);
+                b01 = pack_hi(X.x, X.z);
+                b10 = pack_lo(X.y, X.w);
+                b11 = pack_hi(X.y, X.w);
+            } else {
+                b00 = X.x;
+                b01 = X.y;
+                b10 = X.z;
+                b11 = X.w;
+            }
+            constexpr int P = Chains<NN>::P;
+#pragma unroll
+            for (int m = 0; m < C::kMats; ++m) {
+                mma_16816(acc[m][n][(2 * c) % P], A[m][c][0][0], A[m][c][1][0], A[m][c][0][1], A[m][c][1][1], b00, b01);
+                mma_16816(acc[m][n][(2 * c + 1) % P], A[m][c][0][2], A[m][c][1][2], A[m][c][0][3], A[m][c][1][3], b10, b11);
+            }
+        }
+    }
+}
+
+// int8 path, one chunk pair: 64 K values of each of the warp's 16 rows and of each
+// matrix.  The ldmatrix words become s8 bytes 16 x code: even elements feed one mma,
+// odd elements a second one, with the matching limb bytes of the B operand (the 16
+// bytes at 64 q of the limb block: even elements of chunks 2q and 2q+1, then odd ones).  NN = 1:
+// one n-tile whose columns are (limb, token) = (g / 2, g % 2); NN = 3: n-tile = limb,
+// column = token.  The two mma accumulate 16 x sum(code * limb) exactly in s32, in two
+// independent chains (even and odd elements) so that a stage's mma do not serialise.
+template <bool GU, int NN>
+__device__ __forceinline__ void chunk_pair_limbs(uint32_t abase, const Lane &L, int q, const uint4 (&Bq)[NN],
+                                                 int (&acc)[2][GU ? 2 : 1][NN][4])
+{
+    constexpr int M = GU ? 2 : 1;
+    uint32_t ev[M][4], od[M][4];
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        uint32_t r[4];
+        ldmatrix_x4(r[0], r[1], r[2], r[3], abase + m * kMatStage + L.off[q]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) int4_word_to_s8x16(r[i], ev[m][i], od[m][i]);
+    }
+#pragma unroll
+    for (int n = 0; n < NN; ++n) {
+        const uint4 B = Bq[n];
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            mma_s8(acc[0][m][n], ev[m][0], ev[m][1], ev[m][2], ev[m][3], B.x, B.y);
+            mma_s8(acc[1][m][n], od[m][0], od[m][1], od[m][2], od[m][3], B.z, B.w);
+        }
+    }
+}
+
+// int8 path, gate/up: the ntok h rows of a finished token chunk (fp16, natural order,
+// K values each) -> int8 limb rows and their scales.  The rows' largest magnitudes were
+// gathered by the items that wrote them (atomicMax on the float bits, reset here for the
+// next call).  The four consumer warps.
+template <int NT, int BAR = 1>
+__device__ __noinline__ void convert_h_rows(const __half *src0, size_t src_stride, unsigned char *dst0, float *scale0,
+                                            unsigned *amax0, int ntok, int K, int ltid)
+{
+    __shared__ float s_m[kMaxConvRows];
+    if (ltid < ntok) {
+        s_m[ltid] = __uint_as_float(__ldcg(amax0 + ltid));
+        amax0[ltid] = 0u;
+    }
+    consumer_sync<NT, BAR>();
+    const int nb = (K + kLimbBlockK - 1) / kLimbBlockK;
+    const size_t row_bytes = (size_t)nb * kLimbBlockBytes;
+    for (int j = 0; j < ntok; ++j) {
+        const int sh = limb_shift(s_m[j]);
+        const float scale = pow2f(sh);
+        const __half *src = src0 + j * src_stride;
+        unsigned char *dst = dst0 + j * row_bytes;
+        for (int k8 = 8 * ltid; k8 < nb * kLimbBlockK; k8 += 8 * NT) {
+            const uint4 v = k8 < K ? __ldcg(reinterpret_cast<const uint4 *>(src + k8)) : make_uint4(0u, 0u, 0u, 0u);
+            limb_encode8(v, scale, dst + (size_t)(k8 / kLimbBlockK) * kLimbBlockBytes, k8 % kLimbBlockK);
+        }
+        if (ltid == 0) scale0[j] = pow2f(-sh);
+    }
+    consumer_sync<NT, BAR>();   // s_m is reused by the next conversion
+}
+
+}  // namespace moe

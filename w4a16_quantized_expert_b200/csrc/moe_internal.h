@@ -15,6 +15,8 @@ namespace moe {
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kRouterTokTile = 16;     // tokens per router CTA
+constexpr int kFusedMaxT = 16;         // largest batch the one-launch decode layer takes
+constexpr int kSyncLine = 32;          // words between two synchronisation words (one 128-byte line each)
 constexpr int kRouterMaxDynSmem = 160 * 1024;   // router x staging limit
 // scratch of the allocation-free routing entry point: 64 token-tile counters (256 B),
 // then score, selection score and logits for up to kStaticRouteElems (token, expert) pairs
@@ -119,6 +121,45 @@ struct FfnParams {
     int *status;
 };
 
+// The whole decode-sized layer (T <= kFusedMaxT) in one persistent launch (moe_fused.cu).
+// Work items, claimed in this order: router tasks (one expert's logits for all T tokens;
+// the last one also runs the top-k and the grouping), shared-expert gate/up, routed
+// gate/up, shared-expert down, routed down.  Items of 64 output rows and up to 8 tokens.
+struct FusedParams {
+    DequantK dk;
+    int T, H, I, I_sh, E, k, n_shared, fmt;
+    float scaling, top_p;
+    const uint16_t *x;          // [T][H]
+    uint16_t *y;                // [T][H]
+    LayerWeights wt;
+    float *logits, *score, *sel;                 // [T][E]
+    int32_t *topk_idx;                           // [T][k]
+    float *topk_w;                               // [T][k]
+    int32_t *counts, *offsets, *perm, *unique, *n_unique;
+    int4 *slots;                                 // [E]: (expert, count, offset) of the non-empty experts
+    unsigned char *x_limbs;                      // int4: [T][nblk(H)][3][256]
+    float *x_limb_scale;                         // [T]
+    __half *h;                                   // [T*k][I], rows in perm order
+    __half *h_sh;                                // [T][I_sh]
+    unsigned char *h_limbs, *hsh_limbs;          // int4: limb rows of h and h_sh
+    float *h_limb_scale, *hsh_limb_scale;
+    unsigned int *h_amax;                        // [T*k + T] largest |h| per row (reset after use)
+    float *y_assign;                             // [T*k][H]
+    float *y_shared;                             // [T][H]
+    const uint16_t *zrow;                        // zero halves (padding rows)
+    // Synchronisation words, each alone in its 128-byte line (kSyncLine words apart), so
+    // that polling one never queues behind atomics on another.  Control words: [0] epoch of
+    // the last complete call, [1] epoch whose routing is published, [2] epoch whose x limbs
+    // are complete, [3] router tasks done (wraps), [4] work claims, [5] CTAs done, [6] x-limb
+    // tasks done (wraps).
+    unsigned int *ctl;
+    unsigned int *chunk_ctr;    // [T*k + T] gate/up row tiles done per token chunk (wraps)
+    unsigned int *chunk_flag;   // [T*k + T] epoch whose chunk's h (and its limbs) is complete
+    unsigned int *tile_ctr;     // [H/64] down items done per output row tile (wraps)
+    int *status;
+    int stages, stage_bytes, slot_cap;   // ring slots, bytes per slot, slot-table capacity
+};
+
 struct CombineParams {
     const float *y_assign, *y_shared, *topk_w;
     uint16_t *y;
@@ -136,4 +177,5 @@ struct moe_layer {
     int device;
     int num_sms;
     int occ[2][2][2];   // resident CTAs per SM of the expert kernels [tok_chunk 32][gate_up][ks == 4]
+    int occ_fused;      // resident CTAs per SM of the one-launch decode-layer kernel
 };

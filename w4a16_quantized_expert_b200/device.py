@@ -9,7 +9,7 @@ import numpy as np
 import torch
 
 from . import (MOE_FMT_INT4_ROWSCALE, MOE_FMT_NVFP4, moe_combine, moe_expert_ffn,
-               moe_forward, moe_forward_host, moe_group, moe_layer_create, moe_layer_desc,
+               moe_forward, moe_forward_fused, moe_forward_host, moe_group, moe_layer_create, moe_layer_desc,
                moe_layer_destroy, moe_route, moe_route_static, moe_weights, moe_workspace_size)
 
 # host array key -> moe_weights field
@@ -85,12 +85,14 @@ class DeviceLayer:
         return (stream or torch.cuda.current_stream()).cuda_stream
 
     def forward(self, x: torch.Tensor, ws: torch.Tensor, y: torch.Tensor | None = None,
-                stream=None) -> torch.Tensor:
+                stream=None, fused: bool = False) -> torch.Tensor:
+        """The layer (moe_forward); fused=True: the one-launch decode path
+        (moe_forward_fused, T <= 16)."""
         T = x.shape[0]
         if y is None:
             y = torch.empty_like(x)
-        moe_forward(self.handle, x.data_ptr(), T, y.data_ptr(), ws.data_ptr(), ws.numel(),
-                    self._stream(stream))
+        fn = moe_forward_fused if fused else moe_forward
+        fn(self.handle, x.data_ptr(), T, y.data_ptr(), ws.data_ptr(), ws.numel(), self._stream(stream))
         return y
 
     def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, ws: torch.Tensor,
