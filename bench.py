@@ -50,7 +50,14 @@ DEFAULTS = {
     "prefill2048": (100, 5, 1),
     "decode1_topp": (40000, 400, 8),
     "tiny": (20000, 200, 8),
+    "int8_1": (20000, 400, 4),
+    "int8_8": (8000, 200, 4),
+    "int2_1": (40000, 400, 8),
+    "int2_8": (8000, 200, 8),
 }
+
+FMT_NAMES = {synth.FMT_INT4: "int4", synth.FMT_NVFP4: "nvfp4", synth.FMT_INT8: "int8",
+             synth.FMT_INT2: "int2"}
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
@@ -64,7 +71,7 @@ NCU_TRAFFIC = {
 
 
 def describe(w) -> str:
-    fmt = "int4 row-scale" if w.fmt == synth.FMT_INT4 else "NVFP4 (E2M1 + E4M3/16 + fp32)"
+    fmt = "NVFP4 (E2M1 + E4M3/16 + fp32)" if w.fmt == synth.FMT_NVFP4 else f"{FMT_NAMES[w.fmt]} row-scale"
     bias = "Zipf(1.1) bias in [-0.5,0.5]" if w.bias == "zipf" else "bias U(-0.1,0.1)"
     topp = f", adaptive expert top-p {w.top_p}" if getattr(w, "top_p", 0.0) else ""
     return (f"{w.name}: T={w.T}, H={w.H}, I={w.I}, E={w.E}, top-{w.k}, {w.n_shared} shared "
@@ -75,9 +82,10 @@ def describe(w) -> str:
 def expert_bytes(w, shared=False) -> dict:
     """Bytes of one expert's quantised weights, per matrix group."""
     H, I = w.H, (w.I_sh if shared else w.I)
-    if w.fmt == synth.FMT_INT4:
-        gu = 2 * (I * H // 2) + 2 * I * 4
-        dn = H * I // 2 + H * 4
+    if w.fmt != synth.FMT_NVFP4:   # codes at b bits + one fp32 scale per row
+        b = synth.ROWSCALED_BITS[w.fmt]
+        gu = 2 * (I * H * b // 8) + 2 * I * 4
+        dn = H * I * b // 8 + H * 4
     else:
         gu = 2 * (I * H // 2) + 2 * (I * H // 16) + 2 * 4
         dn = H * I // 2 + H * I // 16 + 4
@@ -294,12 +302,13 @@ def run_reference(args, w):
             I_ = w.I
             RR = R
         out = []
-        if w.fmt == synth.FMT_INT4:
+        if w.fmt != synth.FMT_NVFP4:
+            f, nb = w.fmt, RR * synth.ROWSCALED_BITS[w.fmt] // 8   # code bytes of RR inputs
             sc = (host[key + "sg"], host[key + "su"], host[key + "sd"]) if e is None else \
                  (host["sg"][e], host["su"][e], host["sd"][e])
-            out.append({"format": 0, "codes": np.ascontiguousarray(g[:RR]), "row_scale": sc[0][:RR]})
-            out.append({"format": 0, "codes": np.ascontiguousarray(u[:RR]), "row_scale": sc[1][:RR]})
-            out.append({"format": 0, "codes": np.ascontiguousarray(d[:, : RR // 2]), "row_scale": sc[2]})
+            out.append({"format": f, "codes": np.ascontiguousarray(g[:RR]), "row_scale": sc[0][:RR]})
+            out.append({"format": f, "codes": np.ascontiguousarray(u[:RR]), "row_scale": sc[1][:RR]})
+            out.append({"format": f, "codes": np.ascontiguousarray(d[:, :nb]), "row_scale": sc[2]})
         else:
             if e is None:
                 bs = (host["sh_bg"], host["sh_bu"], host["sh_bd"])
@@ -361,8 +370,9 @@ def run_reference(args, w):
 
 # ------------------------------------------------------------------ our arm
 # workloads measured beside the headline one in the default run (the rest of the
-# metric's configurations: T=8 decode, NVFP4 at T=1 and T=16, the T=512 batch)
-EXTRA_CONFIGS = ("decode8", "nvfp4_1", "nvfp4_16", "prefill512")
+# metric's configurations: T=8 decode, NVFP4 at T=1 and T=16, the T=512 batch; and the
+# int8 and int2 widths at the decode1 shape)
+EXTRA_CONFIGS = ("decode8", "nvfp4_1", "nvfp4_16", "prefill512", "int8_1", "int2_1")
 MIN_REGION_S = 0.5     # timed regions are repeated until they add up to at least this
 
 
@@ -541,7 +551,7 @@ def bench_config(args, w, world, dev, stream, host=None, want_e2e=True):
 
     # ---- the one-launch decode path on the same layers and tokens (T <= 16)
     fused = None
-    if w.T <= 16 and not args.no_fused:
+    if w.T <= 16 and w.fmt in (synth.FMT_INT4, synth.FMT_NVFP4) and not args.no_fused:
         def fwd_fused(i):
             layers[i].forward(xs[i], ws, y=ys[i], stream=stream, fused=True)
 
@@ -662,7 +672,7 @@ def run_ours(args, w):
         "config": {
             "workload": describe(w),
             "T": w.T, "H": w.H, "I": w.I, "E": w.E, "top_k": w.k, "top_p": w.top_p, "n_shared": w.n_shared,
-            "weights": "int4" if w.fmt == synth.FMT_INT4 else "nvfp4",
+            "weights": FMT_NAMES[w.fmt],
             "rotating_layers": head["R"],
             "unique_experts_per_step": head["U"],
             "l2": f"no flush: {head['R']} layer copies at distinct addresses, "

@@ -34,11 +34,13 @@
  *    borrowed: the library never frees them.  Weight pointers given to moe_layer_create
  *    must stay valid and unchanged for the life of the handle.
  *  - Activations are fp16 given as their uint16_t bit patterns, row-major [T][H].
- *  - Quantised matrices are row-major with K (the input dimension) contiguous; two 4-bit
- *    codes per byte, element 2b in the LOW nibble of byte b.  int4 codes are two's
- *    complement in [-8, 7] with one fp32 scale per output row.  NVFP4 codes are E2M1 with
- *    one E4M3 (OCP "FN") scale byte per 16 consecutive K elements of a row and one fp32
- *    scale per (expert, matrix).
+ *  - Quantised matrices are row-major with K (the input dimension) contiguous.  4-bit
+ *    formats hold two codes per byte, element 2b in the LOW nibble of byte b.  int4 codes
+ *    are two's complement in [-8, 7] with one fp32 scale per output row.  int8 codes are
+ *    one two's-complement byte per weight, int2 codes four per byte (element 4b + i in
+ *    bits 2i..2i+1 of byte b, two's complement in [-2, 1]), each with one fp32 scale per
+ *    output row.  NVFP4 codes are E2M1 with one E4M3 (OCP "FN") scale byte per 16
+ *    consecutive K elements of a row and one fp32 scale per (expert, matrix).
  *  - Every call except create/destroy/get_device_status is asynchronous on the caller's
  *    stream, allocates nothing and never synchronises the host, so it may be captured in
  *    a CUDA graph.  A non-zero return means nothing was enqueued.
@@ -75,7 +77,9 @@ enum {
 /* weight formats */
 enum {
     MOE_FMT_INT4_ROWSCALE = 0,   /* int4 codes + fp32 scale per output row */
-    MOE_FMT_NVFP4 = 1            /* E2M1 codes + E4M3 per 16 K-elements + fp32 per matrix */
+    MOE_FMT_NVFP4 = 1,           /* E2M1 codes + E4M3 per 16 K-elements + fp32 per matrix */
+    MOE_FMT_INT8_ROWSCALE = 2,   /* int8 codes + fp32 scale per output row */
+    MOE_FMT_INT2_ROWSCALE = 3    /* int2 codes + fp32 scale per output row */
 };
 
 /* Shape and hyper-parameters of one layer. */
@@ -103,11 +107,12 @@ typedef struct moe_layer_desc {
 /* Device pointers to one layer's parameters (borrowed; see conventions).
  * Routed tensors have a leading expert dimension E; shared ones do not.
  *   router_w     fp32 [E][H]              router_bias fp32 [E]
- *   gate, up     u8   [E][I][H/2]         down        u8   [E][H][I/2]
- *   int4:  gate_scale, up_scale fp32 [E][I];  down_scale fp32 [E][H]
+ *   gate, up     u8   [E][I][H*b/8]       down        u8   [E][H][I*b/8]
+ *          (b = bits per code: 4 for int4 and NVFP4, 8 for int8, 2 for int2)
+ *   int4, int8, int2: gate_scale, up_scale fp32 [E][I];  down_scale fp32 [E][H]
  *   NVFP4: gate_bscale, up_bscale u8 [E][I][H/16]; down_bscale u8 [E][H][I/16];
  *          gate_tscale, up_tscale, down_tscale fp32 [E]
- *   shared_*: the same without E, with I_sh rows (gate/up) or I_sh/2 bytes (down);
+ *   shared_*: the same without E, with I_sh rows (gate/up) or I_sh*b/8 bytes (down);
  *          shared NVFP4 tensor scales are fp32 [1].
  * Pointers that the chosen format or n_shared does not use may be NULL.  Every pointer
  * must be 16-byte aligned. */
@@ -128,13 +133,13 @@ typedef struct moe_layer moe_layer;   /* opaque handle */
 
 /* ---------------------------------------------------------------- lifetime */
 
-/* Source: the layer's shape and weight formats -- int4 with per-row scales (hakusoku
- * page "Show HN: 低速のコンピュータでGLM 5.2を動かす方法", section "実装済み機能"), NVFP4
+/* Source: the layer's shape and weight formats -- int8, int4 and int2 with per-row scales
+ * (hakusoku page "Show HN: 低速のコンピュータでGLM 5.2を動かす方法", section "実装済み機能"), NVFP4
  * (648news page "GTX 1070向け35BパラメータMoEモデル推論エンジン公開", section "用語の注釈"),
  * 256 experts of about 19 MB (hakusoku page, section "Colibrì: ...").
  * Validates desc and weights and builds the handle: TMA descriptors over the caller's
  * weights and a device status word (the only allocation the library makes).
- * Requirements: H and I (and I_sh) multiples of 64 (int4) or 256 (NVFP4) -- the NVFP4
+ * Requirements: H and I (and I_sh) multiples of 64 (int4, int8, int2) or 256 (NVFP4) -- the NVFP4
  * block-scale rows must be 16-byte multiples -- H <= 16384, I, I_sh <= 16384,
  * 1 <= E <= 1024, 1 <= k <= min(E, 32), n_shared in {0, 1}, 1 <= max_tokens <= 65536,
  * all pointers 16-byte aligned.  Uses the current CUDA device.
@@ -253,7 +258,8 @@ int moe_forward(const moe_layer *layer, const uint16_t *x, int T, uint16_t *y,
  * same bits as moe_forward's.  With int4 weights y is moe_forward's y bit for bit (the
  * same exact integer sums, the same epilogue and combine order); with NVFP4 the fp32 sums
  * may run in another order (moe_forward splits K across warps for small layers), within
- * the layer's tolerance.  Returns MOE_ERR_UNSUPPORTED for T > 16 (and MOE_OK for T = 0).
+ * the layer's tolerance.  Returns MOE_ERR_UNSUPPORTED for T > 16 and for int8 or int2
+ * weights (and MOE_OK for T = 0).
  * The grid holds two CTAs per SM and its CTAs wait for one another's flags (bounded waits,
  * MOE_ERR_DEVICE_TIMEOUT if one gives up): do not run it beside another kernel that keeps
  * SMs occupied for good. */

@@ -14,6 +14,8 @@ Workloads (sizes and distributions as the layer is described for GLM-class decod
 * ``nvfp4_1`` / ``nvfp4_16`` -- H=2048, I=512, E=256, k=8, one shared expert, NVFP4,
   T=1 and T=16.
 * ``prefill512`` -- T=512, otherwise as ``decode1``.
+* ``int8_1`` / ``int8_8`` / ``int2_1`` / ``int2_8`` -- the decode1 shape with int8 or int2
+  codes (one fp32 scale per row), T=1 and T=8.
 """
 from __future__ import annotations
 
@@ -30,6 +32,13 @@ _SRC = os.path.join(_HERE, "synth.c")
 
 FMT_INT4 = 0
 FMT_NVFP4 = 1
+FMT_INT8 = 2
+FMT_INT2 = 3
+# bits per code of the row-scaled formats, and the factor on their U(0.01, 0.03) row scales
+# that gives every format about the same weight spread (uniform codes: std 73.9, 4.6 and
+# 1.1 for int8, int4, int2; powers of two keep the scales' fp32 values exact)
+ROWSCALED_BITS = {FMT_INT4: 4, FMT_INT8: 8, FMT_INT2: 2}
+_SCALE_FACTOR = {FMT_INT4: 1.0, FMT_INT8: 1.0 / 16.0, FMT_INT2: 4.0}
 
 
 def build(force: bool = False) -> str:
@@ -167,6 +176,16 @@ WORKLOADS = {
     # larger batch (about 64 tokens per expert): the tensor-memory kernel's compute-heavier regime
     "prefill2048": Workload("prefill2048", 2048, 6144, 2048, 2048, 256, 8, 1, 2.5, FMT_INT4,
                             "uniform", BASE_SEED + 5),
+    # the other row-scaled widths (int8 and int2 kernels with per-row scales: hakusoku page,
+    # section "実装済み機能") at the decode1 shape, one token and eight
+    "int8_1": Workload("int8_1", 1, 6144, 2048, 2048, 256, 8, 1, 2.5, FMT_INT8, "uniform",
+                       BASE_SEED + 6),
+    "int8_8": Workload("int8_8", 8, 6144, 2048, 2048, 256, 8, 1, 2.5, FMT_INT8, "zipf",
+                       BASE_SEED + 6),
+    "int2_1": Workload("int2_1", 1, 6144, 2048, 2048, 256, 8, 1, 2.5, FMT_INT2, "uniform",
+                       BASE_SEED + 7),
+    "int2_8": Workload("int2_8", 8, 6144, 2048, 2048, 256, 8, 1, 2.5, FMT_INT2, "zipf",
+                       BASE_SEED + 7),
 }
 
 
@@ -187,9 +206,12 @@ def make_router(w: Workload):
     return Wr, b
 
 
-def _int4_matrix(seed, tid, sid_scale, e, rows, K, out_q, out_s):
-    out_q[...] = random_bytes(seed, _sid(tid, e), rows * K // 2).reshape(rows, K // 2)
-    out_s[...] = uniform_f32(seed, _sid(sid_scale, e), rows, 0.01, 0.03)
+def _rowscaled_matrix(seed, tid, sid_scale, e, rows, K, fmt, out_q, out_s):
+    """Uniform random code bytes (every code value equally likely) and row scales."""
+    nb = K * ROWSCALED_BITS[fmt] // 8
+    out_q[...] = random_bytes(seed, _sid(tid, e), rows * nb).reshape(rows, nb)
+    s = uniform_f32(seed, _sid(sid_scale, e), rows, 0.01, 0.03)
+    out_s[...] = (s * np.float32(_SCALE_FACTOR[fmt])).astype(np.float32)
 
 
 def _nvfp4_matrix(seed, tid, e, rows, K, out_q, out_b):
@@ -199,39 +221,41 @@ def _nvfp4_matrix(seed, tid, e, rows, K, out_q, out_b):
 
 
 def make_experts(w: Workload, experts=None) -> dict:
-    """Quantised weights of the routed experts (all E, laid out [E][rows][K/2];
+    """Quantised weights of the routed experts (all E, laid out [E][rows][K*bits/8];
     only the listed ``experts`` are filled, the rest stay zero) and of the shared
-    expert.  int4: codes + fp32 row scales.  NVFP4: codes + E4M3 block scales
+    expert.  int8 / int4 / int2: codes + fp32 row scales.  NVFP4: codes + E4M3 block scales
     (one per 16 K-elements) + one fp32 tensor scale per (expert, matrix) equal to
     1/sqrt(fan-in)."""
     E, H, I, Ish = w.E, w.H, w.I, w.I_sh
     ex = range(E) if experts is None else sorted(set(int(e) for e in experts))
     zeros = np.zeros if experts is not None else np.empty
+    bits = ROWSCALED_BITS.get(w.fmt, 4)
     out = {
-        "g": zeros((E, I, H // 2), np.uint8),
-        "u": zeros((E, I, H // 2), np.uint8),
-        "d": zeros((E, H, I // 2), np.uint8),
+        "g": zeros((E, I, H * bits // 8), np.uint8),
+        "u": zeros((E, I, H * bits // 8), np.uint8),
+        "d": zeros((E, H, I * bits // 8), np.uint8),
     }
     shared = w.n_shared > 0
     if shared:
-        out["sh_g"] = np.empty((Ish, H // 2), np.uint8)
-        out["sh_u"] = np.empty((Ish, H // 2), np.uint8)
-        out["sh_d"] = np.empty((H, Ish // 2), np.uint8)
-    if w.fmt == FMT_INT4:
+        out["sh_g"] = np.empty((Ish, H * bits // 8), np.uint8)
+        out["sh_u"] = np.empty((Ish, H * bits // 8), np.uint8)
+        out["sh_d"] = np.empty((H, Ish * bits // 8), np.uint8)
+    if w.fmt in ROWSCALED_BITS:
+        f = w.fmt
         out["sg"] = zeros((E, I), np.float32)
         out["su"] = zeros((E, I), np.float32)
         out["sd"] = zeros((E, H), np.float32)
         for e in ex:
-            _int4_matrix(w.seed, T_G, T_SG, e, I, H, out["g"][e], out["sg"][e])
-            _int4_matrix(w.seed, T_U, T_SU, e, I, H, out["u"][e], out["su"][e])
-            _int4_matrix(w.seed, T_D, T_SD, e, H, I, out["d"][e], out["sd"][e])
+            _rowscaled_matrix(w.seed, T_G, T_SG, e, I, H, f, out["g"][e], out["sg"][e])
+            _rowscaled_matrix(w.seed, T_U, T_SU, e, I, H, f, out["u"][e], out["su"][e])
+            _rowscaled_matrix(w.seed, T_D, T_SD, e, H, I, f, out["d"][e], out["sd"][e])
         if shared:
             out["sh_sg"] = np.empty(Ish, np.float32)
             out["sh_su"] = np.empty(Ish, np.float32)
             out["sh_sd"] = np.empty(H, np.float32)
-            _int4_matrix(w.seed, T_SHG, T_SHSG, 0, Ish, H, out["sh_g"], out["sh_sg"])
-            _int4_matrix(w.seed, T_SHU, T_SHSU, 0, Ish, H, out["sh_u"], out["sh_su"])
-            _int4_matrix(w.seed, T_SHD, T_SHSD, 0, H, Ish, out["sh_d"], out["sh_sd"])
+            _rowscaled_matrix(w.seed, T_SHG, T_SHSG, 0, Ish, H, f, out["sh_g"], out["sh_sg"])
+            _rowscaled_matrix(w.seed, T_SHU, T_SHSU, 0, Ish, H, f, out["sh_u"], out["sh_su"])
+            _rowscaled_matrix(w.seed, T_SHD, T_SHSD, 0, H, Ish, f, out["sh_d"], out["sh_sd"])
     else:
         out["bg"] = zeros((E, I, H // 16), np.uint8)
         out["bu"] = zeros((E, I, H // 16), np.uint8)
@@ -320,7 +344,7 @@ def scale_layer(layer: dict, fmt: int, gate_up: float, down: float, router: floa
     out = dict(layer)
     if "Wr" in out:
         out["Wr"] = (np.asarray(out["Wr"], np.float32) * np.float32(router)).astype(np.float32)
-    if fmt == FMT_INT4:
+    if fmt != FMT_NVFP4:
         keys_gu, keys_d = ("sg", "su", "sh_sg", "sh_su"), ("sd", "sh_sd")
     else:
         keys_gu, keys_d = ("tg", "tu", "sh_tg", "sh_tu"), ("td", "sh_td")

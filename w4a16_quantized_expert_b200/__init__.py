@@ -23,6 +23,8 @@ MOE_ERR_DEVICE_BOUNDS = 6
 
 MOE_FMT_INT4_ROWSCALE = 0
 MOE_FMT_NVFP4 = 1
+MOE_FMT_INT8_ROWSCALE = 2
+MOE_FMT_INT2_ROWSCALE = 3
 
 vp = ctypes.c_void_p
 c_int = ctypes.c_int

@@ -55,9 +55,11 @@ bool use_tc(const moe_layer_desc &d, int T)
 }
 
 // the int4 expert kernels run on the int8 path (activations as limbs) for decode-sized
-// batches (8-token items) and on the tensor-memory kernel
+// batches (8-token items) and on the tensor-memory kernel; int8 and int2 weights run the
+// 8-token int8 path at every batch size
 bool use_limbs(const moe_layer_desc &d, int T)
 {
+    if (d.format == MOE_FMT_INT8_ROWSCALE || d.format == MOE_FMT_INT2_ROWSCALE) return true;
     return d.format == MOE_FMT_INT4_ROWSCALE && (T <= 16 || use_tc(d, T));
 }
 
@@ -150,8 +152,8 @@ bool make_map(CUtensorMap *m, const void *base, int row_bytes, int rows, int exp
 int validate_desc(const moe_layer_desc *d)
 {
     if (!d) return MOE_ERR_INVALID_ARG;
+    if (d->format < MOE_FMT_INT4_ROWSCALE || d->format > MOE_FMT_INT2_ROWSCALE) return MOE_ERR_INVALID_ARG;
     const int kmul = d->format == MOE_FMT_NVFP4 ? 256 : 64;
-    if (d->format != MOE_FMT_INT4_ROWSCALE && d->format != MOE_FMT_NVFP4) return MOE_ERR_INVALID_ARG;
     if (d->hidden <= 0 || d->hidden > 16384 || d->hidden % kmul) return MOE_ERR_INVALID_ARG;
     if (d->inter <= 0 || d->inter > 16384 || d->inter % kmul) return MOE_ERR_INVALID_ARG;
     if (d->n_shared != 0 && d->n_shared != 1) return MOE_ERR_INVALID_ARG;
@@ -172,7 +174,7 @@ int validate_weights(const moe_layer_desc *d, const moe_weights *w)
     int n = 0;
     req[n++] = w->router_w; req[n++] = w->router_bias;
     req[n++] = w->gate; req[n++] = w->up; req[n++] = w->down;
-    if (d->format == MOE_FMT_INT4_ROWSCALE) {
+    if (row_scaled(d->format)) {
         req[n++] = w->gate_scale; req[n++] = w->up_scale; req[n++] = w->down_scale;
     } else {
         req[n++] = w->gate_bscale; req[n++] = w->up_bscale; req[n++] = w->down_bscale;
@@ -180,7 +182,7 @@ int validate_weights(const moe_layer_desc *d, const moe_weights *w)
     }
     if (d->n_shared) {
         req[n++] = w->shared_gate; req[n++] = w->shared_up; req[n++] = w->shared_down;
-        if (d->format == MOE_FMT_INT4_ROWSCALE) {
+        if (row_scaled(d->format)) {
             req[n++] = w->shared_gate_scale; req[n++] = w->shared_up_scale; req[n++] = w->shared_down_scale;
         } else {
             req[n++] = w->shared_gate_bscale; req[n++] = w->shared_up_bscale; req[n++] = w->shared_down_bscale;
@@ -192,9 +194,13 @@ int validate_weights(const moe_layer_desc *d, const moe_weights *w)
     return MOE_OK;
 }
 
-// tokens per expert work item: 8 for decode-sized batches (a one-n-tile kernel with few
-// registers; a bucket of more tokens becomes several items), 32 otherwise
-int tok_chunk(int T) { return T <= 16 ? 8 : kTokChunk; }   // (the tensor-memory kernel sets its own)
+// tokens per expert work item: 8 for decode-sized batches and for int8 / int2 weights (a
+// one-n-tile kernel with few registers; a bucket of more tokens becomes several items), 32
+// otherwise
+int tok_chunk(const moe_layer_desc &d, int T)   // (the tensor-memory kernel sets its own)
+{
+    return (T <= 16 || d.format == MOE_FMT_INT8_ROWSCALE || d.format == MOE_FMT_INT2_ROWSCALE) ? 8 : kTokChunk;
+}
 
 int check_ws(const moe_layer *L, int T, void *ws, size_t bytes)
 {
@@ -257,7 +263,7 @@ FfnParams ffn_params(const moe_layer *L, const uint16_t *x, int T, void *ws)
     p.n_shared = L->desc.n_shared;
     p.fmt = L->desc.format;
     p.dk = {0x000F000Fu, 0x00F000F0u, 0x64086408u, 0x64806480u, 0x64086408u, 0x2C002C00u, 0xD480D480u};
-    p.tok_chunk = tok_chunk(T);
+    p.tok_chunk = tok_chunk(L->desc, T);
     p.x = x;
     p.xb = x;
     p.xb_perm = 0;
@@ -292,7 +298,7 @@ struct Launch {
 Launch ffn_launch(const moe_layer *L, int T, bool gu)
 {
     const moe_layer_desc &d = L->desc;
-    const int tc = tok_chunk(T);
+    const int tc = tok_chunk(d, T);
     const int wide = tc > 8;
     const long slots = (long)std::min<long>(d.n_experts, (long)T * d.top_k);
     const long chunks_sh = (T + tc - 1) / tc;
@@ -313,8 +319,9 @@ Launch ffn_launch(const moe_layer *L, int T, bool gu)
     return {4, L->num_sms * L->occ[wide][gu][1]};
 }
 
-// The decode-sized layer in one launch (moe_fused.cu).
+// The decode-sized layer in one launch (moe_fused.cu): int4 and NVFP4 weights.
 bool use_fused(int T) { return T >= 1 && T <= kFusedMaxT; }
+bool fused_format(int fmt) { return fmt == MOE_FMT_INT4_ROWSCALE || fmt == MOE_FMT_NVFP4; }
 
 int run_fused(const moe_layer *L, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s,
               void *const *events)
@@ -485,15 +492,16 @@ int moe_layer_create(const moe_layer_desc *desc, const moe_weights *weights, moe
     const int H = d.hidden, I = d.inter, Is = d.inter_shared, E = d.n_experts;
     bool ok = true;
     LayerMaps &M = L->maps;
+    const int cb = code_bits(d.format);   // code bytes of a K-long row: K * cb / 8
     for (int r4 = 0; r4 < 2 && ok; ++r4) {
         const int br = r4 ? 4 * kRowTile : kRowTile;
-        ok = make_map(r4 ? &M.g4 : &M.g, w.gate, H / 2, I, E, 128, true, br) &&
-             make_map(r4 ? &M.u4 : &M.u, w.up, H / 2, I, E, 128, true, br) &&
-             make_map(r4 ? &M.d4 : &M.d, w.down, I / 2, H, E, 128, true, br);
+        ok = make_map(r4 ? &M.g4 : &M.g, w.gate, H * cb / 8, I, E, 128, true, br) &&
+             make_map(r4 ? &M.u4 : &M.u, w.up, H * cb / 8, I, E, 128, true, br) &&
+             make_map(r4 ? &M.d4 : &M.d, w.down, I * cb / 8, H, E, 128, true, br);
         if (ok && d.n_shared)
-            ok = make_map(r4 ? &M.sh_g4 : &M.sh_g, w.shared_gate, H / 2, Is, 1, 128, true, br) &&
-                 make_map(r4 ? &M.sh_u4 : &M.sh_u, w.shared_up, H / 2, Is, 1, 128, true, br) &&
-                 make_map(r4 ? &M.sh_d4 : &M.sh_d, w.shared_down, Is / 2, H, 1, 128, true, br);
+            ok = make_map(r4 ? &M.sh_g4 : &M.sh_g, w.shared_gate, H * cb / 8, Is, 1, 128, true, br) &&
+                 make_map(r4 ? &M.sh_u4 : &M.sh_u, w.shared_up, H * cb / 8, Is, 1, 128, true, br) &&
+                 make_map(r4 ? &M.sh_d4 : &M.sh_d, w.shared_down, Is * cb / 8, H, 1, 128, true, br);
         if (ok && d.format == MOE_FMT_NVFP4) {
             ok = make_map(r4 ? &M.gb4 : &M.gb, w.gate_bscale, H / 16, I, E, 16, false, br) &&
                  make_map(r4 ? &M.ub4 : &M.ub, w.up_bscale, H / 16, I, E, 16, false, br) &&
@@ -510,7 +518,8 @@ int moe_layer_create(const moe_layer_desc *desc, const moe_weights *weights, moe
     }
     bool occ_ok = router_prepare() == cudaSuccess && ffn_prepare(d.format, d.n_experts, L->occ) == cudaSuccess &&
                   (d.format != MOE_FMT_INT4_ROWSCALE || tc_prepare(d.n_experts) == cudaSuccess) &&
-                  fused_prepare(d.format, &L->occ_fused) == cudaSuccess && L->occ_fused >= 1;
+                  (!fused_format(d.format) ||
+                   (fused_prepare(d.format, &L->occ_fused) == cudaSuccess && L->occ_fused >= 1));
     for (int a = 0; a < 2; ++a)
         for (int b = 0; b < 2; ++b)
             for (int c = 0; c < 2; ++c) occ_ok = occ_ok && L->occ[a][b][c] >= 1;
@@ -699,7 +708,7 @@ int moe_forward_fused(const moe_layer *L, const uint16_t *x, int T, uint16_t *y,
 {
     if (!L || T < 0 || T > L->desc.max_tokens) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
-    if (!use_fused(T)) return MOE_ERR_UNSUPPORTED;
+    if (!use_fused(T) || !fused_format(L->desc.format)) return MOE_ERR_UNSUPPORTED;
     if (!x || !y || !aligned16(x)) return MOE_ERR_INVALID_ARG;
     int rc = check_ws(L, T, ws, ws_bytes);
     if (rc) return rc;

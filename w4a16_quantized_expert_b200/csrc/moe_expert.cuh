@@ -32,24 +32,32 @@ struct FfnCfg {
     static constexpr int kMats = GU ? 2 : 1;
     static constexpr int kRW = kConsumerWarps / KS;
     static constexpr bool kNv = FMT == MOE_FMT_NVFP4;
-    static constexpr int kStageK = KS * kBoxBytes;        // K bytes per stage
-    static constexpr int kCodeBytes = kMats * kMatStage;
+    // decode variant of the row-scaled formats: the int8 tensor path (weights as s8 bytes,
+    // activations as three int8 limbs; items of at most 8 tokens, KS = 1).  int8 and int2
+    // weights run only this variant.
+    static constexpr bool kLimbs = row_scaled(FMT) && NNMAX == 1 && KS == 1;
+    // K boxes (128 bytes wide) per matrix and stage: a stage covers whole 256-value limb
+    // blocks, so int8 takes two boxes (256 values), int4 one (256), int2 one (512)
+    static constexpr int kBoxesK = (kLimbs && FMT == MOE_FMT_INT8_ROWSCALE) ? 2 : 1;
+    static constexpr int kMatBytes = kBoxesK * kMatStage;     // one matrix's codes per stage
+    static constexpr int kStageK = KS * kBoxesK * kBoxBytes;  // K bytes per stage
+    static constexpr int kStageVals = kStageK * 8 / code_bits(FMT);   // K values per stage
+    static constexpr int kGroups = kStageVals / 64;           // 64-value groups per stage
+    static constexpr int kCodeShift = FMT == MOE_FMT_INT8_ROWSCALE ? 0 : FMT == MOE_FMT_INT2_ROWSCALE ? 6 : 4;
+    static constexpr int kCodeBytes = kMats * kMatBytes;
     static constexpr int kScaleBytes = kNv ? kMats * kConsumerWarps * kScaleBoxSmem : 0;
-    // int4 decode variant: the int8 tensor path (weights as s8 bytes, activations as
-    // three int8 limbs; items of at most 8 tokens, KS = 1)
-    static constexpr bool kLimbs = FMT == MOE_FMT_INT4_ROWSCALE && NNMAX == 1 && KS == 1;
     // decode variant: the producer also copies each stage's slice of the (up to 8) token
     // rows of the B operand into shared memory, one row per token: fp16 values padded to
-    // 16 bytes, or one 768-byte limb block (the stage's 256 K values, three limbs)
+    // 16 bytes, or the limb blocks of the stage's K values (768 bytes per 256 values)
     static constexpr bool kSmemB = NNMAX == 1 && KS == 1;
-    static constexpr int kBRow = kLimbs ? kLimbBlockBytes : 4 * kStageK + 16;
+    static constexpr int kBRow = kLimbs ? kStageVals / kLimbBlockK * kLimbBlockBytes : 4 * kStageK + 16;
     static constexpr int kBBytes = kSmemB ? 8 * kBRow : 0;      // per stage, after the ring (at most)
     static constexpr int kStageBytes = ((kCodeBytes + kScaleBytes) + 1023) / 1024 * 1024;
     // Ring depth.  Weights in flight per SM decide the bandwidth (DRAM latency under full
     // load is about 2.5 us); the int8 path sizes its ring at launch (up to kStagesMax
     // stages, as many as fit beside a second CTA on the SM, given the B rows per stage).
     static constexpr int kStages = GU ? (kSmemB ? 3 : 4) : 5;
-    static constexpr int kStagesCap = kLimbs ? (GU ? 6 : 12) : kStages;
+    static constexpr int kStagesCap = kLimbs ? (GU ? 6 : 12) / kBoxesK : kStages;
     static constexpr int kZeroRow = kSmemB ? kBRow : 0;   // zero row read by padding lanes
     static constexpr int kRedFloats = KS > 1 ? kConsumerWarps * kMats * kTokChunk * kRowTile : 0;
 };
@@ -87,7 +95,7 @@ __device__ __forceinline__ void consumer_sync()
     asm volatile("bar.sync %0, %1;" ::"n"(ID), "r"(NT) : "memory");
 }
 
-// int4: the fp32 scale of row `row`; NVFP4: the fp32 scale of the whole matrix
+// row-scaled formats: the fp32 scale of row `row`; NVFP4: the fp32 scale of the whole matrix
 template <int FMT>
 __device__ __forceinline__ float mat_scale(const float *scales, int e, int rows, int row)
 {
@@ -174,26 +182,82 @@ __device__ __forceinline__ void chunk_pair(const unsigned char *st, uint32_t aba
     }
 }
 
-// int8 path, one chunk pair: 64 K values of each of the warp's 16 rows and of each
-// matrix.  The ldmatrix words become s8 bytes 16 x code: even elements feed one mma,
-// odd elements a second one, with the matching limb bytes of the B operand (the 16
-// bytes at 64 q of the limb block: even elements of chunks 2q and 2q+1, then odd ones).  NN = 1:
-// one n-tile whose columns are (limb, token) = (g / 2, g % 2); NN = 3: n-tile = limb,
-// column = token.  The two mma accumulate 16 x sum(code * limb) exactly in s32, in two
-// independent chains (even and odd elements) so that a stage's mma do not serialise.
-template <bool GU, int NN>
+// int8 path, the A operand of one 64-value group q of a stage, for one matrix whose
+// stage codes start at shared address `mbase` (the warp's 16-row box of each K box):
+// ev[i] / od[i] hold, as s8 bytes 2^shift x code, the even / odd elements of the 8 K
+// values 64 q + 32 c + 8 tq .. +7 of row g (i = 2c) or g + 8 (i = 2c + 1) -- the order of
+// the limb bytes of the B operand.
+//  int4: ldmatrix words (chunk 2q + c of rows g, g + 8), nibbles moved to the top of bytes;
+//  int8: the 8 bytes of each (row, c), split into even and odd bytes;
+//  int2: the 16 bits of each (row, c); rows g and g + 8 are joined in one word and each
+//        2-bit code is moved to the top two bits of its byte.
+// Rows are 128 bytes with the 128-byte swizzle (16-byte unit u of row r at u ^ (r % 8)).
+template <int FMT>
+__device__ __forceinline__ void limb_a_words(uint32_t mbase, const Lane &L, int q, uint32_t (&ev)[4],
+                                             uint32_t (&od)[4])
+{
+    if constexpr (FMT == MOE_FMT_INT8_ROWSCALE) {
+        const uint32_t base = mbase + (q >> 1) * kMatStage;   // K box of the group
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = L.g + 8 * (i & 1), c = i >> 1;
+            const int u = 4 * (q & 1) + 2 * c + (L.tq >> 1);
+            uint32_t lo, hi;
+            asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
+                         : "=r"(lo), "=r"(hi)
+                         : "r"(base + r * kBoxBytes + ((u ^ (r & 7)) << 4) + 8 * (L.tq & 1)));
+            ev[i] = __byte_perm(lo, hi, 0x6420);
+            od[i] = __byte_perm(lo, hi, 0x7531);
+        }
+    } else if constexpr (FMT == MOE_FMT_INT2_ROWSCALE) {
+        constexpr uint32_t kTop = 0xC0C0C0C0u;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            uint32_t v[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int r = L.g + 8 * h;
+                unsigned short b;
+                asm volatile("ld.shared.u16 %0, [%1];"
+                             : "=h"(b)
+                             : "r"(mbase + r * kBoxBytes + ((q ^ (r & 7)) << 4) + 8 * c + 2 * L.tq));
+                v[h] = b;
+            }
+            // bytes 0, 1: row g (codes 0..3, 4..7); bytes 2, 3: row g + 8
+            const uint32_t w = __byte_perm(v[0], v[1], 0x5410);
+            // top two bits of byte b after the shift: code 0 / 4 (<< 6), 2 / 6 (<< 2),
+            // 1 / 5 (<< 4), 3 / 7 (no shift) of the 16-bit row in bytes 2b', 2b' + 1
+            const uint32_t s6 = w << 6, s2 = w << 2, s4 = w << 4;
+            ev[2 * c] = __byte_perm(s6, s2, 0x5140) & kTop;
+            ev[2 * c + 1] = __byte_perm(s6, s2, 0x7362) & kTop;
+            od[2 * c] = __byte_perm(s4, w, 0x5140) & kTop;
+            od[2 * c + 1] = __byte_perm(s4, w, 0x7362) & kTop;
+        }
+    } else {
+        uint32_t r[4];
+        ldmatrix_x4(r[0], r[1], r[2], r[3], mbase + L.off[q]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) int4_word_to_s8x16(r[i], ev[i], od[i]);
+    }
+}
+
+// int8 path, one 64-value group q of a stage: 64 K values of each of the warp's 16 rows
+// and of each matrix.  The A words (limb_a_words) are s8 bytes 2^shift x code: even
+// elements feed one mma, odd elements a second one, with the matching limb bytes of the
+// B operand (the 16 bytes at 64 (q % 4) of the group's limb block: even elements of the
+// two 32-value halves, then odd ones).  NN = 1: one n-tile whose columns are
+// (limb, token) = (g / 2, g % 2); NN = 3: n-tile = limb, column = token.  The two mma
+// accumulate 2^shift x sum(code * limb) exactly in s32, in two independent chains (even
+// and odd elements) so that a stage's mma do not serialise.
+template <int FMT, bool GU, int NN>
 __device__ __forceinline__ void chunk_pair_limbs(uint32_t abase, const Lane &L, int q, const uint4 (&Bq)[NN],
                                                  int (&acc)[2][GU ? 2 : 1][NN][4])
 {
+    using C = FfnCfg<FMT, GU, 1, 1>;
     constexpr int M = GU ? 2 : 1;
     uint32_t ev[M][4], od[M][4];
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-        uint32_t r[4];
-        ldmatrix_x4(r[0], r[1], r[2], r[3], abase + m * kMatStage + L.off[q]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) int4_word_to_s8x16(r[i], ev[m][i], od[m][i]);
-    }
+    for (int m = 0; m < M; ++m) limb_a_words<FMT>(abase + m * C::kMatBytes, L, q, ev[m], od[m]);
 #pragma unroll
     for (int n = 0; n < NN; ++n) {
         const uint4 B = Bq[n];

@@ -445,26 +445,26 @@ __device__ __forceinline__ void settle(const FfnParams &p, Pending &pd, int ltid
     pd.kind = 0;
 }
 
-// One warp's share of one work item on the int8 path (int4 weights, KS = 1, at most 8
-// tokens): the stages, then the epilogue.  NN = 1 for items of 1-2 tokens, 3 otherwise.
-// The accumulators hold 16 x sum(code * limb) per (limb, token); the epilogue forms
+// One warp's share of one work item on the int8 path (int8, int4 or int2 weights, KS = 1,
+// at most 8 tokens): the stages, then the epilogue.  NN = 1 for items of 1-2 tokens, 3
+// otherwise.  The accumulators hold 2^shift x sum(code * limb) per (limb, token) (shift
+// 0, 4, 6 for int8, int4, int2); the epilogue forms
 // sum(code * X) = S0 + 256 S1 + 65536 S2 exactly in 64-bit integers and scales it by
 // 2^-sh and the row scale in fp64.  Gate/up then stores h in fp16 and the last item of
 // a token chunk converts the chunk's h rows to limbs for the down kernel.  Everything
 // the epilogue needs besides the accumulators is loaded before the stages.
-template <bool GU, int NN>
+template <int FMT, bool GU, int NN>
 __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const SlotTable tb, const Item it,
                                                    unsigned char *ring, unsigned char *bring, uint64_t *full,
                                                    uint64_t *empty, int &stage, uint32_t &phase, const Lane L,
                                                    uint32_t zsm, Pending &pd, volatile int *cfail,
                                                    volatile int *abort_flag)
 {
-    using C = FfnCfg<MOE_FMT_INT4_ROWSCALE, GU, 1, 1>;
+    using C = FfnCfg<FMT, GU, 1, 1>;
     const int S = p.stages;
     constexpr int M = C::kMats;
     const bool sh = it.e < 0;
-    const int Kb = it.K / 2;
-    const int nst = (Kb + C::kStageK - 1) / C::kStageK;
+    const int nst = (it.K + C::kStageVals - 1) / C::kStageVals;
     // this lane's B column in n-tile 0: (limb, token); its limb block of each stage sits in
     // the stage's B rows (padding columns read the zero row)
     const int lcol = NN == 1 ? (L.g >> 1) : 0;
@@ -508,15 +508,11 @@ __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const Slo
 
     bool ok = true;
     for (int s = 0; s < nst; ++s) {
-        const int kbox = s * C::kStageK;
-        const int npairs = kbox + kBoxBytes <= Kb ? 4 : (Kb - kbox) / 32;   // K is a multiple of 64
+        // 64-value groups of this stage (K is a multiple of 64)
+        const int ngroups = min(C::kGroups, (it.K - s * C::kStageVals) / 64);
         if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
         const uint32_t bb = bval ? smem_u32(bring + (size_t)stage * p.b_stage) + boff : zsm + 16 * L.tq;
-        uint4 B[4][NN];
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-            for (int n = 0; n < NN; ++n) B[q][n] = lds128(bb + n * kLimbBlockK + 64 * q);
+        // (the zero row is one stage's B row long: every group's offset stays inside it)
         if (GU && s == 0) {
             // the activation scales of the lane's tokens (their ids came with the perm loads)
 #pragma unroll
@@ -527,13 +523,22 @@ __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const Slo
             }
         }
         const uint32_t abase = smem_u32(ring + (size_t)stage * C::kStageBytes + L.bx * kBoxSmem);
-        if (npairs == 4) {
+        // the groups of one 256-value limb block at a time (int2 stages hold two blocks)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) chunk_pair_limbs<GU, NN>(abase, L, q, B[q], acc2);
-        } else {
+        for (int blk = 0; blk < C::kGroups / 4; ++blk) {
+            uint4 B[4][NN];
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                if (q < npairs) chunk_pair_limbs<GU, NN>(abase, L, q, B[q], acc2);
+#pragma unroll
+                for (int n = 0; n < NN; ++n) B[q][n] = lds128(bb + blk * kLimbBlockBytes + n * kLimbBlockK + 64 * q);
+            if (ngroups == C::kGroups) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) chunk_pair_limbs<FMT, GU, NN>(abase, L, 4 * blk + q, B[q], acc2);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (4 * blk + q < ngroups) chunk_pair_limbs<FMT, GU, NN>(abase, L, 4 * blk + q, B[q], acc2);
+            }
         }
         __syncwarp();
         if (L.lane == 0) mbar_arrive(&empty[stage]);
@@ -570,7 +575,7 @@ __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const Slo
             // lanes tq = 0, 1, 2 of a quad hold limbs 0, 1, 2 of tokens c & 1
 #pragma unroll
             for (int m = 0; m < M; ++m) {
-                const int v0 = acc[m][0][c] >> 4;
+                const int v0 = acc[m][0][c] >> C::kCodeShift;
                 const int v1 = __shfl_down_sync(0xffffffffu, v0, 1);
                 const int v2 = __shfl_down_sync(0xffffffffu, v0, 2);
                 Sv[m] = (long long)v0 + 256ll * v1 + 65536ll * v2;
@@ -578,7 +583,8 @@ __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const Slo
         } else {
 #pragma unroll
             for (int m = 0; m < M; ++m)
-                Sv[m] = (long long)(acc[m][0][c] >> 4) + 256ll * (acc[m][1][c] >> 4) + 65536ll * (acc[m][2][c] >> 4);
+                Sv[m] = (long long)(acc[m][0][c] >> C::kCodeShift) + 256ll * (acc[m][1][c] >> C::kCodeShift) +
+                        65536ll * (acc[m][2][c] >> C::kCodeShift);
         }
         const int u = c & 1, h = c >> 1;
         if (!uval[u]) continue;
@@ -748,7 +754,7 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
                 const Item it = (i < n_pre) ? make_item<GU, RW>(p, -1, p.T, 0, i) : decode_item<GU, RW>(p, tb, i);
                 const bool sh = it.e < 0;
                 const int ez = sh ? 0 : it.e;
-                const int Kb = it.K / 2;
+                const int Kb = it.K * code_bits(FMT) / 8;   // code bytes of a row
                 const int nst = (Kb + C::kStageK - 1) / C::kStageK;
                 // decode variant: token rows of the B operand, copied stage by stage
                 const unsigned char *brows[8];
@@ -762,9 +768,12 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
                     }
                 }
                 // bytes of a B row that stage s needs, and where they start
-                auto b_src = [&](int s2) -> size_t { return C::kLimbs ? (size_t)s2 * kLimbBlockBytes : (size_t)4 * s2 * C::kStageK; };
+                // (limb rows end at their last 256-value block: an int2 stage's second block
+                // may lie past it)
+                auto b_src = [&](int s2) -> size_t { return C::kLimbs ? (size_t)s2 * C::kBRow : (size_t)4 * s2 * C::kStageK; };
                 auto b_len = [&](int s2) -> uint32_t {
-                    return C::kLimbs ? (uint32_t)kLimbBlockBytes : 4u * (uint32_t)min(C::kStageK, Kb - s2 * C::kStageK);
+                    return C::kLimbs ? (uint32_t)min((size_t)C::kBRow, limb_row_bytes(it.K) - (size_t)s2 * C::kBRow)
+                                     : 4u * (uint32_t)min(C::kStageK, Kb - s2 * C::kStageK);
                 };
                 // The down kernel starts early (programmatic launch) and its B operand, h,
                 // comes from the gate/up kernel: its first stages get their weights at once
@@ -774,7 +783,8 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
                     if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
                     unconfirmed &= ~(1u << stage);
                     const int kb0 = s * C::kStageK;
-                    const int nks = min(KS, (Kb - kb0 + kBoxBytes - 1) / kBoxBytes);
+                    // K boxes of this stage (KS for the K-split launches, two for int8)
+                    const int nks = min(KS * C::kBoxesK, (Kb - kb0 + kBoxBytes - 1) / kBoxBytes);
                     const uint32_t bbytes = b_len(s);
                     uint32_t tx = (uint32_t)C::kMats * RW * nks * (kBoxSmem + (C::kNv ? kScaleBoxSmem : 0));
                     if constexpr (C::kSmemB) {
@@ -788,10 +798,13 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
                         const CUtensorMap *bm = sh ? (m ? bS1 : bS0) : (m ? bA1 : bA0);
                         for (int rw = 0; rw < (kBox64 ? 1 : RW); ++rw)
                             for (int ks = 0; ks < nks; ++ks) {
-                                // (a 64-row box lands as the four 16-row boxes, stacked)
+                                // (a 64-row box lands as the four 16-row boxes, stacked;
+                                // int8's second K box follows the first)
                                 const int bx = rw * KS + ks;
-                                tma_load_3d(st + m * kMatStage + bx * kBoxSmem, map, &full[stage],
-                                            kb0 + ks * kBoxBytes, it.row0 + rw * kRowTile, ez, pol);
+                                unsigned char *dst = C::kBoxesK > 1 ? st + m * C::kMatBytes + ks * kMatStage
+                                                                    : st + m * kMatStage + bx * kBoxSmem;
+                                tma_load_3d(dst, map, &full[stage], kb0 + ks * kBoxBytes, it.row0 + rw * kRowTile,
+                                            ez, pol);
                                 if (C::kNv)
                                     tma_load_3d(st + C::kCodeBytes + (m * kConsumerWarps + bx) * kScaleBoxSmem, bm,
                                                 &full[stage], (kb0 + ks * kBoxBytes) / 8, it.row0 + rw * kRowTile,
@@ -898,10 +911,11 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
         if constexpr (C::kLimbs) {
             // x limbs come from the router, h limbs from the gate/up kernel
             if (n_item == 0) pdl_wait();
-            const bool ok = it.ntok <= 2 ? consume_item_limbs<GU, 1>(p, tb, it, ring, bring, full, empty, stage, phase,
-                                                                     L, zsm, pend, cfail, abort_flag)
-                                         : consume_item_limbs<GU, 3>(p, tb, it, ring, bring, full, empty, stage, phase,
-                                                                     L, zsm, pend, cfail, abort_flag);
+            const bool ok = it.ntok <= 2
+                                ? consume_item_limbs<FMT, GU, 1>(p, tb, it, ring, bring, full, empty, stage, phase, L,
+                                                                 zsm, pend, cfail, abort_flag)
+                                : consume_item_limbs<FMT, GU, 3>(p, tb, it, ring, bring, full, empty, stage, phase, L,
+                                                                 zsm, pend, cfail, abort_flag);
             if (!ok) break;
             continue;
         } else {
@@ -1637,18 +1651,25 @@ static cudaError_t prepare_fmt(int E, int occ[2][2][2])
     cudaError_t e;
     if ((e = prepare_t<FMT, true, 1, 1>(E, &occ[0][1][0])) != cudaSuccess) return e;
     if ((e = prepare_t<FMT, false, 1, 1>(E, &occ[0][0][0])) != cudaSuccess) return e;
-    if constexpr (FMT == MOE_FMT_INT4_ROWSCALE) {
-        // the int8 path (int4, items of <= 8 tokens) has no K-split variant
-        occ[0][1][1] = occ[0][1][0];
-        occ[0][0][1] = occ[0][0][0];
+    if constexpr (FMT == MOE_FMT_INT8_ROWSCALE || FMT == MOE_FMT_INT2_ROWSCALE) {
+        // int8 and int2 run the int8 path only (8-token items, KS = 1, any batch)
+        for (int w = 0; w < 2; ++w)
+            for (int g = 0; g < 2; ++g) occ[w][g][0] = occ[w][g][1] = occ[0][g][0];
+        return cudaSuccess;
     } else {
-        if ((e = prepare_t<FMT, true, 4, 1>(E, &occ[0][1][1])) != cudaSuccess) return e;
-        if ((e = prepare_t<FMT, false, 4, 1>(E, &occ[0][0][1])) != cudaSuccess) return e;
+        if constexpr (FMT == MOE_FMT_INT4_ROWSCALE) {
+            // the int8 path (int4, items of <= 8 tokens) has no K-split variant
+            occ[0][1][1] = occ[0][1][0];
+            occ[0][0][1] = occ[0][0][0];
+        } else {
+            if ((e = prepare_t<FMT, true, 4, 1>(E, &occ[0][1][1])) != cudaSuccess) return e;
+            if ((e = prepare_t<FMT, false, 4, 1>(E, &occ[0][0][1])) != cudaSuccess) return e;
+        }
+        if ((e = prepare_t<FMT, true, 1, 4>(E, &occ[1][1][0])) != cudaSuccess) return e;
+        if ((e = prepare_t<FMT, true, 4, 4>(E, &occ[1][1][1])) != cudaSuccess) return e;
+        if ((e = prepare_t<FMT, false, 1, 4>(E, &occ[1][0][0])) != cudaSuccess) return e;
+        return prepare_t<FMT, false, 4, 4>(E, &occ[1][0][1]);
     }
-    if ((e = prepare_t<FMT, true, 1, 4>(E, &occ[1][1][0])) != cudaSuccess) return e;
-    if ((e = prepare_t<FMT, true, 4, 4>(E, &occ[1][1][1])) != cudaSuccess) return e;
-    if ((e = prepare_t<FMT, false, 1, 4>(E, &occ[1][0][0])) != cudaSuccess) return e;
-    return prepare_t<FMT, false, 4, 4>(E, &occ[1][0][1]);
 }
 
 template <bool GU>
@@ -1696,22 +1717,33 @@ cudaError_t launch_tc(const LayerMaps &maps, const FfnParams &p0, bool gate_up, 
 
 cudaError_t ffn_prepare(int fmt, int E, int occ[2][2][2])
 {
-    return fmt == MOE_FMT_NVFP4 ? prepare_fmt<MOE_FMT_NVFP4>(E, occ) : prepare_fmt<MOE_FMT_INT4_ROWSCALE>(E, occ);
+    switch (fmt) {
+    case MOE_FMT_NVFP4: return prepare_fmt<MOE_FMT_NVFP4>(E, occ);
+    case MOE_FMT_INT8_ROWSCALE: return prepare_fmt<MOE_FMT_INT8_ROWSCALE>(E, occ);
+    case MOE_FMT_INT2_ROWSCALE: return prepare_fmt<MOE_FMT_INT2_ROWSCALE>(E, occ);
+    default: return prepare_fmt<MOE_FMT_INT4_ROWSCALE>(E, occ);
+    }
 }
 
 template <int FMT>
 static cudaError_t launch_fmt(const LayerMaps &maps, const FfnParams &p, bool gu, int ks, int grid, bool pdl,
                               cudaStream_t s)
 {
-    const bool wide = p.tok_chunk > 8;
-    if (!wide && (ks == 1 || FMT == MOE_FMT_INT4_ROWSCALE))
+    if constexpr (FMT == MOE_FMT_INT8_ROWSCALE || FMT == MOE_FMT_INT2_ROWSCALE) {
+        if (p.tok_chunk != 8 || ks != 1) return cudaErrorInvalidValue;
         return gu ? launch_t<FMT, true, 1, 1>(maps, p, grid, pdl, s) : launch_t<FMT, false, 1, 1>(maps, p, grid, pdl, s);
-    if (!wide) {
-        if constexpr (FMT != MOE_FMT_INT4_ROWSCALE)
-            return gu ? launch_t<FMT, true, 4, 1>(maps, p, grid, pdl, s) : launch_t<FMT, false, 4, 1>(maps, p, grid, pdl, s);
+    } else {
+        const bool wide = p.tok_chunk > 8;
+        if (!wide && (ks == 1 || FMT == MOE_FMT_INT4_ROWSCALE))
+            return gu ? launch_t<FMT, true, 1, 1>(maps, p, grid, pdl, s) : launch_t<FMT, false, 1, 1>(maps, p, grid, pdl, s);
+        if (!wide) {
+            if constexpr (FMT != MOE_FMT_INT4_ROWSCALE)
+                return gu ? launch_t<FMT, true, 4, 1>(maps, p, grid, pdl, s) : launch_t<FMT, false, 4, 1>(maps, p, grid, pdl, s);
+        }
+        if (gu)
+            return ks == 1 ? launch_t<FMT, true, 1, 4>(maps, p, grid, pdl, s) : launch_t<FMT, true, 4, 4>(maps, p, grid, pdl, s);
+        return ks == 1 ? launch_t<FMT, false, 1, 4>(maps, p, grid, pdl, s) : launch_t<FMT, false, 4, 4>(maps, p, grid, pdl, s);
     }
-    if (gu) return ks == 1 ? launch_t<FMT, true, 1, 4>(maps, p, grid, pdl, s) : launch_t<FMT, true, 4, 4>(maps, p, grid, pdl, s);
-    return ks == 1 ? launch_t<FMT, false, 1, 4>(maps, p, grid, pdl, s) : launch_t<FMT, false, 4, 4>(maps, p, grid, pdl, s);
 }
 
 // p.tok_chunk (8 or 32) selects the kernel variant: 8-token items for decode batches,
@@ -1719,8 +1751,12 @@ static cudaError_t launch_fmt(const LayerMaps &maps, const FfnParams &p, bool gu
 cudaError_t launch_ffn(const LayerMaps &maps, const FfnParams &p, bool gate_up, int ks, int grid, bool pdl,
                        cudaStream_t s)
 {
-    return p.fmt == MOE_FMT_NVFP4 ? launch_fmt<MOE_FMT_NVFP4>(maps, p, gate_up, ks, grid, pdl, s)
-                                  : launch_fmt<MOE_FMT_INT4_ROWSCALE>(maps, p, gate_up, ks, grid, pdl, s);
+    switch (p.fmt) {
+    case MOE_FMT_NVFP4: return launch_fmt<MOE_FMT_NVFP4>(maps, p, gate_up, ks, grid, pdl, s);
+    case MOE_FMT_INT8_ROWSCALE: return launch_fmt<MOE_FMT_INT8_ROWSCALE>(maps, p, gate_up, ks, grid, pdl, s);
+    case MOE_FMT_INT2_ROWSCALE: return launch_fmt<MOE_FMT_INT2_ROWSCALE>(maps, p, gate_up, ks, grid, pdl, s);
+    default: return launch_fmt<MOE_FMT_INT4_ROWSCALE>(maps, p, gate_up, ks, grid, pdl, s);
+    }
 }
 
 cudaError_t launch_wait_timeout(int *status, unsigned long long max_iters, cudaStream_t s)

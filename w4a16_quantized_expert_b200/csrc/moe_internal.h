@@ -30,10 +30,19 @@ constexpr int kStaticRouteContexts = 64;   // CUDA contexts whose scratch addres
 constexpr int kRowTile = 16;           // output rows per expert work item (mma M)
 constexpr int kTokChunk = 32;          // tokens per expert work item (4 mma N-tiles)
 
+// bits per weight code of a format
+__host__ __device__ constexpr int code_bits(int fmt)
+{
+    return fmt == MOE_FMT_INT8_ROWSCALE ? 8 : fmt == MOE_FMT_INT2_ROWSCALE ? 2 : 4;
+}
+
+// formats with one fp32 scale per output row (int8, int4, int2)
+__host__ __device__ constexpr bool row_scaled(int fmt) { return fmt != MOE_FMT_NVFP4; }
+
 // Matrices of one layer in one format.  Routed tensors carry a leading expert index.
 struct LayerWeights {
     const float *router_w, *router_bias;
-    // row scales (int4) or tensor scales (NVFP4), routed [E][rows] / [E], shared
+    // row scales (int8, int4, int2) or tensor scales (NVFP4), routed [E][rows] / [E], shared
     const float *g_scale, *u_scale, *d_scale;
     const float *sh_g_scale, *sh_u_scale, *sh_d_scale;
 };
