@@ -271,6 +271,50 @@ def test_forward_host_matches_forward(tiny):
     assert torch.equal(y_dev.cpu(), yh)
 
 
+def test_forward_host_pipelined_calls_share_a_workspace(tiny):
+    """Consecutive host-buffer calls through two handles that share one workspace (the x
+    copies run ahead on a copy stream into two staging buffers used in turn): every y
+    equals the device-buffer forward of its own tokens, for mapped page-locked y (written
+    by the last kernel) and for pageable y (staged copy), eagerly and replayed from a CUDA
+    graph."""
+    T = tiny.T
+    other = tiny.dev.clone_weights()
+    ws = tiny.dev.workspace(T)
+    xs = [synth.make_tokens(tiny.w, T, batch=10 + b) for b in range(6)]
+    refs = []
+    for i, x in enumerate(xs):
+        dev = tiny.dev if i % 2 == 0 else other
+        refs.append(dev.forward(torch.from_numpy(x.copy()).cuda(), ws).cpu())
+    torch.cuda.synchronize()
+    xh = [torch.from_numpy(x.copy()).pin_memory() for x in xs]
+    yh = [torch.zeros_like(x).pin_memory() if i != 3 else torch.zeros_like(x) for i, x in enumerate(xh)]
+    stream = torch.cuda.Stream()
+    for i in range(len(xs)):
+        (tiny.dev if i % 2 == 0 else other).forward_host(xh[i], yh[i], ws, stream=stream)
+    stream.synchronize()
+    for i in range(len(xs)):
+        assert torch.equal(yh[i], refs[i]), f"eager call {i}"
+    # the same calls (mapped y only) captured once and replayed twice
+    for y in yh:
+        y.zero_()
+    yg = [torch.zeros_like(x).pin_memory() for x in xh]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(len(xs)):
+            (tiny.dev if i % 2 == 0 else other).forward_host(xh[i], yg[i], ws, stream=stream)
+    for _ in range(2):
+        for y in yg:
+            y.zero_()
+        with torch.cuda.stream(stream):
+            g.replay()
+        stream.synchronize()
+        for i in range(len(xs)):
+            assert torch.equal(yg[i], refs[i]), f"graph call {i}"
+    del g
+    assert moe.moe_get_device_status(tiny.dev.handle) == moe.MOE_OK
+    other.close()
+
+
 # ------------------------------------------------------------------ special shapes
 def _special(E, k, n_shared, scaling, fmt=0, bias_hot=None, T=6, H=None, I=None):
     H0, I0 = (256, 128) if fmt == 0 else (512, 256)

@@ -37,8 +37,11 @@ struct FfnCfg {
     // weights run only this variant.
     static constexpr bool kLimbs = row_scaled(FMT) && NNMAX == 1 && KS == 1;
     // K boxes (128 bytes wide) per matrix and stage: a stage covers whole 256-value limb
-    // blocks, so int8 takes two boxes (256 values), int4 one (256), int2 one (512)
-    static constexpr int kBoxesK = (kLimbs && FMT == MOE_FMT_INT8_ROWSCALE) ? 2 : 1;
+    // blocks -- int8 two boxes (256 values), int4 two (512), int2 one (512).  Fewer, larger
+    // stages cost less per byte (one full/empty handshake, one B copy per token and stage):
+    // measured on B200, 16-KB down stages beat 8-KB ones by 8% (decode8), and 32 KB is worse
+    // again (fewer stages in flight per CTA).
+    static constexpr int kBoxesK = !kLimbs ? 1 : FMT == MOE_FMT_INT2_ROWSCALE ? 1 : 2;
     static constexpr int kMatBytes = kBoxesK * kMatStage;     // one matrix's codes per stage
     static constexpr int kStageK = KS * kBoxesK * kBoxBytes;  // K bytes per stage
     static constexpr int kStageVals = kStageK * 8 / code_bits(FMT);   // K values per stage
@@ -57,7 +60,7 @@ struct FfnCfg {
     // load is about 2.5 us); the int8 path sizes its ring at launch (up to kStagesMax
     // stages, as many as fit beside a second CTA on the SM, given the B rows per stage).
     static constexpr int kStages = GU ? (kSmemB ? 3 : 4) : 5;
-    static constexpr int kStagesCap = kLimbs ? (GU ? 6 : 12) / kBoxesK : kStages;
+    static constexpr int kStagesCap = kLimbs ? ((GU ? 6 : 12) / kBoxesK < 2 ? 2 : (GU ? 6 : 12) / kBoxesK) : kStages;
     static constexpr int kZeroRow = kSmemB ? kBRow : 0;   // zero row read by padding lanes
     static constexpr int kRedFloats = KS > 1 ? kConsumerWarps * kMats * kTokChunk * kRowTile : 0;
 };
@@ -235,7 +238,7 @@ __device__ __forceinline__ void limb_a_words(uint32_t mbase, const Lane &L, int 
         }
     } else {
         uint32_t r[4];
-        ldmatrix_x4(r[0], r[1], r[2], r[3], mbase + L.off[q]);
+        ldmatrix_x4(r[0], r[1], r[2], r[3], mbase + (q >> 2) * kMatStage + L.off[q & 3]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) int4_word_to_s8x16(r[i], ev[i], od[i]);
     }
