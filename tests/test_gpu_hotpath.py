@@ -67,7 +67,8 @@ def ws_routing(dev, ws, T):
     return out
 
 
-GROUP_CASES = [("decode1", 1, 0.0), ("tiny", 4, 0.0), ("decode8", 8, 0.0), ("nvfp4_16", 16, 0.0),
+GROUP_CASES = [("decode1", 1, 0.0), ("tiny", 1, 0.0), ("tiny_e1024", 1, 0.0), ("nvfp4_1", 1, 0.0),
+               ("decode1", 1, 0.7), ("tiny", 4, 0.0), ("decode8", 8, 0.0), ("nvfp4_16", 16, 0.0),
                ("tiny", 16, 0.0), ("tiny", 17, 0.0), ("tiny", 37, 0.0), ("prefill512", 512, 0.0),
                ("decode8", 8, 0.7), ("tiny", 4, 0.5), ("tiny", 37, 0.5), ("tiny_e1024", 9, 0.0),
                ("tiny_e1024", 40, 0.0)]

@@ -43,6 +43,42 @@ def test_route_bitexact_from_oracle_logits(name, T):
     _route_from_logits(case, T)
 
 
+@pytest.mark.parametrize("E,k,pattern", [(256, 8, "ties"), (256, 8, "all_equal"), (37, 5, "ties"),
+                                          (5, 2, "ties"), (200, 32, "ties"), (256, 1, "random")])
+def test_route_single_token_bitexact(E, k, pattern):
+    """One token (the whole-CTA top-k and the direct grouping): top-k indices, their order
+    and the grouping bit-exact, weights within 1e-6, from oracle logits full of ties
+    (values on a coarse grid, or all equal), so the lower-index rule decides often."""
+    rng = np.random.default_rng(E * 100 + k)
+    if pattern == "all_equal":
+        logits = np.zeros((1, E), np.float32)
+    elif pattern == "ties":
+        logits = (rng.integers(-4, 5, (1, E)) * 0.25).astype(np.float32)
+    else:
+        logits = rng.standard_normal((1, E)).astype(np.float32)
+    w = synth.WORKLOADS["tiny"].with_(E=E, k=k)
+    host = {"Wr": np.zeros((E, 256), np.float32), "bias": np.zeros(E, np.float32)}
+    if pattern == "ties":   # a bias on the same grid: selection ties among unequal scores
+        host["bias"] = (rng.integers(-2, 3, E) * 0.125).astype(np.float32)
+    host.update(synth.make_experts(w, experts=[]))
+    from w4a16_quantized_expert_b200.device import DeviceLayer
+    desc = oracle.desc_of(w)
+    dev = DeviceLayer(desc, host, max_tokens=1)
+    ws = dev.workspace(1)
+    idx, wt, _ = dev.route(None, 1, ws, logits_in=torch.from_numpy(logits).cuda())
+    torch.cuda.synchronize()
+    r_idx, r_w, _, _ = oracle.default().route(logits, host["bias"], k, float(np.float32(w.scaling)))
+    assert np.array_equal(idx.cpu().numpy(), r_idx)
+    check_weights(wt.cpu().numpy(), r_w.astype(np.float64))
+    counts, offsets, perm, unique, nu = dev.group(idx, 1, ws)
+    c_ref, o_ref, p_ref, u_ref = oracle.default().group(r_idx, E)
+    assert np.array_equal(counts.cpu().numpy(), c_ref) and np.array_equal(offsets.cpu().numpy(), o_ref)
+    assert np.array_equal(perm.cpu().numpy()[: len(p_ref)], p_ref)
+    assert int(nu.item()) == len(u_ref) and np.array_equal(unique.cpu().numpy()[: len(u_ref)], u_ref)
+    assert moe.moe_get_device_status(dev.handle) == moe.MOE_OK
+    dev.close()
+
+
 def test_route_gemv_logits(tiny):
     T = tiny.T
     ws = tiny.dev.workspace(T)

@@ -116,6 +116,98 @@ __device__ void group_warp(const int32_t *topk_idx, bool src_smem, int n, int E,
     }
 }
 
+// ---------------------------------------------------------------------------- one token
+// Top-k of a single token by the whole CTA (E <= kRouterThreads, plain top-k): the same
+// selection and order as topk_token -- descending selection score, equal scores to the
+// lower expert index -- from 64-bit keys (score key, then the complement of the expert
+// index), which are all distinct, so every key has one rank.  Each warp first ranks its
+// 32 keys among themselves; the k best of every warp are the only candidates, and their
+// ranks among the 8k candidates are the final ranks.  Two short passes over shared memory
+// replace the k dependent rounds of the one-warp search.  The weights are then formed by
+// warp 0 exactly as topk_token forms them.  sK: kRouterThreads 64-bit words; sC: 8k words.
+__device__ void topk_one_token_cta(const float *sel_row, const float *score_row, int E, int k, float scaling,
+                                   int32_t *idx_out, float *w_out, int *s_topi, float *s_tops,
+                                   unsigned long long *sK, unsigned long long *sC, int tid)
+{
+    const int lane = tid & 31, warp = tid >> 5;
+    constexpr int NW = kRouterThreads / 32;
+    const bool in = tid < E;
+    unsigned long long key = 0ull;
+    float sc = 0.f;
+    if (in) {
+        sc = __ldcg(score_row + tid);
+        key = ((unsigned long long)float_key(__ldcg(sel_row + tid)) << 32) | (unsigned)(0xFFFFFFFFu - (unsigned)tid);
+    }
+    sK[tid] = key;
+    for (int j = tid; j < NW * k; j += kRouterThreads) sC[j] = 0ull;
+    __syncthreads();
+    int r = 0;   // rank inside the warp's 32 keys (absent experts have key 0 and rank last)
+#pragma unroll
+    for (int j = 0; j < 32; ++j) r += sK[warp * 32 + j] > key;
+    const bool cand = in && r < k;
+    if (cand) sC[warp * k + r] = key;
+    __syncthreads();
+    if (cand) {
+        int g = 0;
+#pragma unroll 16
+        for (int j = 0; j < NW * k; ++j) g += sC[j] > key;
+        if (g < k) {
+            s_topi[g] = tid;
+            s_tops[g] = sc;
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int my_idx = 0;
+        float my_score = 0.f;
+        if (lane < k) {
+            my_idx = s_topi[lane];
+            my_score = s_tops[lane];
+        }
+        // combine weights from the unbiased scores, summed in order j = 0..k-1
+        const double s_mine = lane < k ? static_cast<double>(my_score) : 0.0;
+        double sum = 0.0;
+#pragma unroll 8
+        for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, s_mine, j);
+        if (lane < k) {
+            idx_out[lane] = my_idx;
+            w_out[lane] = static_cast<float>(static_cast<double>(scaling) * (s_mine / sum));
+        }
+    }
+}
+
+// Grouping of a single token's k distinct experts (plain top-k), the results group_block
+// gives: the experts in ascending order, one assignment each (perm = their top-k
+// positions), counts and offsets of all E experts.  s_topi holds the top-k experts.
+__device__ void group_one_token(const int *s_topi, int E, int k, int32_t *counts, int32_t *offsets, int32_t *perm,
+                                int32_t *unique, int32_t *n_unique, int4 *slots, int tid)
+{
+    if (tid < k) {
+        const int e = s_topi[tid];
+        int r = 0;   // position of e among the k experts in ascending order
+#pragma unroll 8
+        for (int j = 0; j < k; ++j) r += s_topi[j] < e;
+        perm[r] = tid;
+        unique[r] = e;
+        if (slots) slots[r] = make_int4(e, 1, r, 0);
+    }
+    if (tid == 0) {
+        *n_unique = k;
+        offsets[E] = k;
+    }
+    for (int e = tid; e < E; e += kRouterThreads) {
+        int below = 0, has = 0;
+#pragma unroll 8
+        for (int j = 0; j < k; ++j) {
+            const int f = s_topi[j];
+            below += f < e;
+            has |= f == e;
+        }
+        counts[e] = has;
+        offsets[e] = below;
+    }
+}
+
 // ---------------------------------------------------------------------------- kernels
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p)
 {
@@ -124,8 +216,8 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p)
     __shared__ float red_max[kRouterThreads / 32][kRouterXRows];
     __shared__ float s_amax[kRouterTokTile];
     __shared__ int s_flag;
-    __shared__ int sm_run[kMaxExperts];
-    __shared__ int sm_off[kMaxExperts + 1];
+    __shared__ __align__(8) int sm_run[kMaxExperts];      // (also the single-token top-k's 64-bit keys)
+    __shared__ __align__(8) int sm_off[kMaxExperts + 1];  // (and its candidates)
     __shared__ int s_idx[kRouterTokTile * kMaxTopK];
     __shared__ __align__(8) uint64_t s_bar[2];
 
@@ -288,6 +380,16 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterParams p)
         __syncthreads();
     }
 
+    if (p.T == 1 && p.top_p == 0.f && p.E <= kRouterThreads) {
+        // a single token with plain top-k: the whole CTA selects, then groups directly
+        __shared__ float s_tops[kMaxTopK];
+        topk_one_token_cta(p.sel, p.score, p.E, p.k, p.scaling, p.topk_idx, p.topk_w, s_idx, s_tops,
+                           reinterpret_cast<unsigned long long *>(sm_run),
+                           reinterpret_cast<unsigned long long *>(sm_off), tid);
+        if (p.do_group)
+            group_one_token(s_idx, p.E, p.k, p.counts, p.offsets, p.perm, p.unique, p.n_unique, p.slots, tid);
+        return;
+    }
     for (int t = warp; t < nt; t += kRouterThreads / 32)
         topk_token(p.sel + (size_t)(t0 + t) * p.E, p.score + (size_t)(t0 + t) * p.E, p.E, p.k, p.scaling, p.top_p,
                    p.topk_idx + (size_t)(t0 + t) * p.k, p.topk_w + (size_t)(t0 + t) * p.k, s_idx + t * p.k);
