@@ -370,9 +370,10 @@ def run_reference(args, w):
 
 # ------------------------------------------------------------------ our arm
 # workloads measured beside the headline one in the default run (the rest of the
-# metric's configurations: T=8 decode, NVFP4 at T=1 and T=16, the T=512 batch; and the
-# int8 and int2 widths at the decode1 shape)
-EXTRA_CONFIGS = ("decode8", "nvfp4_1", "nvfp4_16", "prefill512", "int8_1", "int2_1")
+# metric's configurations: T=8 decode, NVFP4 at T=1 and T=16, the T=512 batch; adaptive
+# top-p on decode1; and the int8 and int2 widths at the decode1 shape, T=1 and T=8)
+EXTRA_CONFIGS = ("decode8", "nvfp4_1", "nvfp4_16", "prefill512", "decode1_topp", "int8_1", "int8_8",
+                 "int2_1", "int2_8")
 MIN_REGION_S = 0.5     # timed regions are repeated until they add up to at least this
 
 
@@ -637,14 +638,17 @@ def run_ours(args, w):
     head = bench_config(args, w, world, dev, stream)
     extras = {}
     if w.name == "decode1" and not args.no_configs:
-        shared_host = {}
+        shared_experts = {}
         for name in EXTRA_CONFIGS:
             wx = synth.WORKLOADS[name]
-            key = (wx.seed, wx.fmt, wx.H, wx.I, wx.E, wx.bias)   # nvfp4_1 and nvfp4_16: one layer
-            if key not in shared_host:
-                shared_host.clear()
-                shared_host[key] = synth.make_layer(wx)
-            extras[name] = bench_config(args, wx, world, dev, stream, host=shared_host[key])
+            # workloads that differ only in T, bias or top-p share their experts' weights
+            key = (wx.seed, wx.fmt, wx.H, wx.I, wx.I_sh, wx.E, wx.n_shared)
+            if key not in shared_experts:
+                shared_experts.clear()
+                shared_experts[key] = synth.make_experts(wx)
+            Wr, b = synth.make_router(wx)
+            host = {"Wr": Wr, "bias": b, **shared_experts[key]}
+            extras[name] = bench_config(args, wx, world, dev, stream, host=host)
     if rank != 0:
         return
     cpu = None
