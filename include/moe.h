@@ -266,19 +266,15 @@ int moe_forward(const moe_layer *layer, const uint16_t *x, int T, uint16_t *y,
 int moe_forward_fused(const moe_layer *layer, const uint16_t *x, int T, uint16_t *y,
                       void *workspace, size_t workspace_bytes, moe_stream_t stream);
 
-/* moe_forward with HOST activations: enqueues the host->device copy of x_host, the
- * layer and the transfer of y into y_host; returns once enqueued; synchronise the stream
- * before reading y_host.  x is copied on a copy stream into one of two
- * staging buffers of the workspace, used in turn: the copy for a call waits only for the
- * call two before it on the same workspace (the last user of its buffer, whatever its
- * handle), so it runs while the previous call computes and the layer's kernels keep their
- * launch chain on `stream`.  The library keeps one copy stream and four events per
- * workspace address (up to 64 workspaces; MOE_ERR_CUDA beyond) for the life of the
- * process.  y_host that is
- * page-locked host memory mapped into the device's address space (any cudaHostAlloc /
- * cudaMallocHost allocation on a system with unified addressing) is written by the last
- * kernel directly; other host memory gets a staged device->host copy on `stream`.
- * x_host should be page-locked for its copy to be asynchronous.  Calls that share a
+/* moe_forward with HOST activations: x_host [T][H] in, y_host [T][H] out (fp16 bits);
+ * returns once enqueued; synchronise the stream before reading y_host.  Page-locked host
+ * memory mapped into the device's address space (any cudaHostAlloc / cudaMallocHost
+ * allocation on a system with unified addressing) is read and written by the kernels
+ * themselves: the first kernel of the launch chain fetches x over the bus while the
+ * previous work on the stream finishes and stores it in the workspace once that work is
+ * complete, and the combine kernel writes y_host directly, so the layer keeps its launch
+ * chain.  Other host memory is staged with copies on the stream (synchronous for pageable
+ * memory).  The workspace's staging buffer is reused by every call: calls that share a
  * workspace must be ordered (the same stream, or one capture sequence). */
 int moe_forward_host(const moe_layer *layer, const uint16_t *x_host, int T, uint16_t *y_host,
                      void *workspace, size_t workspace_bytes, moe_stream_t stream);

@@ -308,11 +308,11 @@ def test_forward_host_matches_forward(tiny):
 
 
 def test_forward_host_pipelined_calls_share_a_workspace(tiny):
-    """Consecutive host-buffer calls through two handles that share one workspace (the x
-    copies run ahead on a copy stream into two staging buffers used in turn): every y
-    equals the device-buffer forward of its own tokens, for mapped page-locked y (written
-    by the last kernel) and for pageable y (staged copy), eagerly and replayed from a CUDA
-    graph."""
+    """Consecutive host-buffer calls through two handles that share one workspace (mapped
+    page-locked x fetched by the first kernel of each launch chain, one staging buffer):
+    every y equals the device-buffer forward of its own tokens, for mapped page-locked y
+    (written by the last kernel), pageable y and pageable x (staged copies), eagerly and
+    replayed from a CUDA graph."""
     T = tiny.T
     other = tiny.dev.clone_weights()
     ws = tiny.dev.workspace(T)
@@ -322,7 +322,7 @@ def test_forward_host_pipelined_calls_share_a_workspace(tiny):
         dev = tiny.dev if i % 2 == 0 else other
         refs.append(dev.forward(torch.from_numpy(x.copy()).cuda(), ws).cpu())
     torch.cuda.synchronize()
-    xh = [torch.from_numpy(x.copy()).pin_memory() for x in xs]
+    xh = [torch.from_numpy(x.copy()).pin_memory() if i != 4 else torch.from_numpy(x.copy()) for i, x in enumerate(xs)]
     yh = [torch.zeros_like(x).pin_memory() if i != 3 else torch.zeros_like(x) for i, x in enumerate(xh)]
     stream = torch.cuda.Stream()
     for i in range(len(xs)):
@@ -330,22 +330,29 @@ def test_forward_host_pipelined_calls_share_a_workspace(tiny):
     stream.synchronize()
     for i in range(len(xs)):
         assert torch.equal(yh[i], refs[i]), f"eager call {i}"
-    # the same calls (mapped y only) captured once and replayed twice
+    # the same calls (mapped x and y only) captured once and replayed twice, with new x
+    # contents written into the same host buffers before the second replay
     for y in yh:
         y.zero_()
+    xh[4] = xh[4].pin_memory()
     yg = [torch.zeros_like(x).pin_memory() for x in xh]
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         for i in range(len(xs)):
             (tiny.dev if i % 2 == 0 else other).forward_host(xh[i], yg[i], ws, stream=stream)
-    for _ in range(2):
+    n = len(xs)
+    for rep in range(2):
         for y in yg:
             y.zero_()
         with torch.cuda.stream(stream):
             g.replay()
         stream.synchronize()
-        for i in range(len(xs)):
-            assert torch.equal(yg[i], refs[i]), f"graph call {i}"
+        for i in range(n):   # (the two handles hold the same weights)
+            assert torch.equal(yg[i], refs[(i + rep) % n]), f"graph call {i}, replay {rep}"
+        # the second replay reads new contents of the same host buffers
+        rotated = [xh[(i + 1) % n].clone() for i in range(n)]
+        for i in range(n):
+            xh[i].copy_(rotated[i])
     del g
     assert moe.moe_get_device_status(tiny.dev.handle) == moe.MOE_OK
     other.close()

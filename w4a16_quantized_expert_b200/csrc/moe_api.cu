@@ -7,7 +7,6 @@
 #include <string.h>
 
 #include <algorithm>
-#include <mutex>
 #include <new>
 
 #include "moe_internal.h"
@@ -18,6 +17,7 @@ cudaError_t router_prepare();
 cudaError_t launch_group(const GroupParams &p, cudaStream_t s);
 cudaError_t static_route_scratch(void **ptr);
 cudaError_t launch_combine(const CombineParams &p, bool pdl, cudaStream_t s);
+cudaError_t launch_host_x(const void *src, void *dst, size_t bytes, cudaStream_t s);
 cudaError_t launch_x_limbs(const uint16_t *x, int T, int H, unsigned char *limbs, float *scale, cudaStream_t s);
 cudaError_t launch_ffn(const LayerMaps &maps, const FfnParams &p, bool gate_up, int ks, int grid, bool pdl,
                        cudaStream_t s);
@@ -40,7 +40,7 @@ struct Ws {
     size_t ctr_tiles, ctr_group, ctr_work, ctr_chunks, h_amax, f_ctl, f_chunk_ctr, f_chunk_flag, f_tile_ctr, zrow,
         ctr_end;
     size_t logits, score, sel, topk_idx, topk_w, counts, offsets, perm, unique, n_unique, slots;
-    size_t x_perm, h, h_sh, y_assign, y_shared, x_stage[2], y_stage;
+    size_t x_perm, h, h_sh, y_assign, y_shared, x_stage, y_stage;
     size_t x_limbs, x_limb_scale, h_limbs, h_limb_scale, hsh_limbs, hsh_limb_scale, total;
 };
 
@@ -103,8 +103,7 @@ Ws ws_layout(const moe_layer_desc &d, int T)
     w.h_sh = o; o = up256(o + (size_t)T * d.inter_shared * 2 * (d.n_shared ? 1 : 0));
     w.y_assign = o; o = up256(o + Tk * d.hidden * 4);
     w.y_shared = o; o = up256(o + (size_t)T * d.hidden * 4 * (d.n_shared ? 1 : 0));
-    w.x_stage[0] = o; o = up256(o + (size_t)T * d.hidden * 2);
-    w.x_stage[1] = o; o = up256(o + (size_t)T * d.hidden * 2);
+    w.x_stage = o; o = up256(o + (size_t)T * d.hidden * 2);
     w.y_stage = o; o = up256(o + (size_t)T * d.hidden * 2);
     const bool lb = use_limbs(d, T);
     w.x_limbs = o; o = up256(o + (lb ? (size_t)T * limb_row_bytes(d.hidden) : 0));
@@ -213,52 +212,6 @@ int check_ws(const moe_layer *L, int T, void *ws, size_t bytes)
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-// Copy pipeline of moe_forward_host, one per workspace (keyed by its address; entries live
-// as long as the process): a copy stream, per staging buffer the event at the start of the
-// call that last used it and the event after that call's host->device copy, and what tells
-// whether the previous call was enqueued in the same stream capture.
-struct HostPipe {
-    const void *ws;
-    int device;
-    cudaStream_t copy;
-    cudaEvent_t ev_call[2], ev_x[2];
-    unsigned long long calls;
-    int last_capturing;
-    unsigned long long last_capture_id;
-};
-constexpr int kHostPipes = 64;
-HostPipe g_host_pipes[kHostPipes];
-int g_n_host_pipes = 0;
-std::mutex g_host_mu;
-
-// the entry of workspace ws on the current device (created on first use; NULL if the table
-// is full or a stream or event cannot be created).  Caller holds g_host_mu.
-HostPipe *host_pipe(const void *ws)
-{
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-    for (int i = 0; i < g_n_host_pipes; ++i)
-        if (g_host_pipes[i].ws == ws && g_host_pipes[i].device == dev) return &g_host_pipes[i];
-    if (g_n_host_pipes == kHostPipes) return nullptr;
-    HostPipe hp = {};
-    hp.ws = ws;
-    hp.device = dev;
-    bool ok = cudaStreamCreateWithFlags(&hp.copy, cudaStreamNonBlocking) == cudaSuccess;
-    for (int i = 0; i < 2; ++i) {
-        ok = ok && cudaEventCreateWithFlags(&hp.ev_call[i], cudaEventDisableTiming) == cudaSuccess;
-        ok = ok && cudaEventCreateWithFlags(&hp.ev_x[i], cudaEventDisableTiming) == cudaSuccess;
-    }
-    if (!ok) {
-        for (int i = 0; i < 2; ++i) {
-            if (hp.ev_call[i]) cudaEventDestroy(hp.ev_call[i]);
-            if (hp.ev_x[i]) cudaEventDestroy(hp.ev_x[i]);
-        }
-        if (hp.copy) cudaStreamDestroy(hp.copy);
-        return nullptr;
-    }
-    g_host_pipes[g_n_host_pipes] = hp;
-    return &g_host_pipes[g_n_host_pipes++];
-}
 
 LayerWeights layer_weights(const moe_layer *L)
 {
@@ -775,40 +728,29 @@ int moe_forward_host(const moe_layer *L, const uint16_t *x_host, int T, uint16_t
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const Ws W = ws_layout(L->desc, T);
     const size_t bytes = (size_t)T * L->desc.hidden * 2;
-    // x goes through the workspace's two staging buffers in turn, copied on a copy stream:
-    // the copy of call i waits only until call i-2 on this workspace (the last user of its
-    // buffer, whatever its handle) is done, so it runs while call i-1 computes, and the
-    // layer's kernels keep their programmatic launch chain (the router of call i still
-    // starts behind the previous call's last kernel).
-    std::lock_guard<std::mutex> lock(g_host_mu);
-    HostPipe *hp = host_pipe(ws);
-    if (!hp) return MOE_ERR_CUDA;
-    const int b = (int)(hp->calls & 1u);
-    uint16_t *xd = at<uint16_t>(ws, W.x_stage[b]);
-    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    unsigned long long cid = 0;
-    if (cudaStreamGetCaptureInfo(s, &cs, &cid) != cudaSuccess) return MOE_ERR_CUDA;
-    const int capturing = cs == cudaStreamCaptureStatusActive;
-    // the previous call's start event is usable when that call was enqueued the same way
-    // (both outside a capture, or both inside this capture); else wait for this call's start
-    const bool chained = hp->calls > 0 && hp->last_capturing == capturing && (!capturing || hp->last_capture_id == cid);
-    if (cudaEventRecord(hp->ev_call[b], s) != cudaSuccess) return MOE_ERR_CUDA;
-    if (cudaStreamWaitEvent(hp->copy, chained ? hp->ev_call[b ^ 1] : hp->ev_call[b], 0) != cudaSuccess ||
-        cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, hp->copy) != cudaSuccess ||
-        cudaEventRecord(hp->ev_x[b], hp->copy) != cudaSuccess || cudaStreamWaitEvent(s, hp->ev_x[b], 0) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    hp->calls++;
-    hp->last_capturing = capturing;
-    hp->last_capture_id = cid;
-    // y: page-locked host memory mapped into the device's address space is written by the
-    // combine kernel directly; other host memory gets a staged device->host copy
-    cudaPointerAttributes pa;
-    uint16_t *yd = nullptr;
-    const cudaError_t qe = cudaPointerGetAttributes(&pa, y_host);
-    if (qe != cudaSuccess) cudaGetLastError();   // (an unknown pointer is not an error here)
-    else if (pa.type == cudaMemoryTypeHost && pa.devicePointer) yd = static_cast<uint16_t *>(pa.devicePointer);
-    if (yd) return run_forward(L, xd, T, yd, ws, s);
-    yd = at<uint16_t>(ws, W.y_stage);
+    // page-locked host memory mapped into the device's address space: its device address
+    // (else NULL: a staged copy)
+    auto mapped = [](const void *h) -> const void * {
+        cudaPointerAttributes pa;
+        if (cudaPointerGetAttributes(&pa, h) != cudaSuccess) {
+            cudaGetLastError();   // (an unknown pointer is not an error here)
+            return nullptr;
+        }
+        return (pa.type == cudaMemoryTypeHost && pa.devicePointer && aligned16(pa.devicePointer)) ? pa.devicePointer
+                                                                                                 : nullptr;
+    };
+    uint16_t *xd = at<uint16_t>(ws, W.x_stage);
+    // x: mapped memory is fetched by the first kernel of the launch chain (host_x_kernel:
+    // bus reads overlap the previous layer); other memory is copied on the stream
+    const void *xm = mapped(x_host);
+    const cudaError_t e = xm ? launch_host_x(xm, xd, bytes, s)
+                             : cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    // y: mapped memory is written by the combine kernel directly; other memory gets a
+    // staged device->host copy
+    uint16_t *ym = const_cast<uint16_t *>(static_cast<const uint16_t *>(mapped(y_host)));
+    if (ym) return run_forward(L, xd, T, ym, ws, s);
+    uint16_t *yd = at<uint16_t>(ws, W.y_stage);
     rc = run_forward(L, xd, T, yd, ws, s);
     if (rc) return rc;
     return cuda_status(cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, s));

@@ -743,6 +743,33 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineParams p)
     p.y[i] = __half_as_ushort(__float2half_rn(acc));
 }
 
+// x of a host-buffer call: page-locked host memory mapped into the device's address space
+// -> the workspace's staging buffer, as the first kernel of the layer's launch chain.  Each
+// thread reads its (up to four) 16-byte pieces over the bus first (uncached: the host
+// rewrites the buffer between calls), while the previous layer is still running, and
+// writes them only once that layer is complete (it is the buffer's last reader), so the
+// bus round trip overlaps the previous layer and the router behind keeps its early start.
+__global__ void __launch_bounds__(256) host_x_kernel(const uint4 *src, uint4 *dst, size_t n16)
+{
+    pdl_trigger();   // the router launched behind this kernel may start (it waits for it)
+    const size_t base = (size_t)blockIdx.x * (256 * 4) + threadIdx.x;
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const size_t i = base + (size_t)j * 256;
+        if (i < n16)
+            asm volatile("ld.global.cv.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v[j].x), "=r"(v[j].y), "=r"(v[j].z), "=r"(v[j].w)
+                         : "l"(src + i));
+    }
+    pdl_wait();      // the previous layer no longer reads the staging buffer
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const size_t i = base + (size_t)j * 256;
+        if (i < n16) dst[i] = v[j];
+    }
+}
+
 // x -> int8 limbs on its own (the staged expert entry point, which runs no router):
 // one CTA per token row
 __global__ void __launch_bounds__(kRouterThreads) x_limbs_kernel(const uint16_t *x, int H, unsigned char *limbs,
@@ -898,6 +925,21 @@ cudaError_t launch_group(const GroupParams &p, cudaStream_t s)
 {
     group_kernel<<<1, kRouterThreads, (size_t)(kRouterThreads / 32) * p.E * sizeof(int), s>>>(p);
     return cudaGetLastError();
+}
+
+cudaError_t launch_host_x(const void *src, void *dst, size_t bytes, cudaStream_t s)
+{
+    const size_t n16 = bytes / 16;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((n16 + 1023) / 1024));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, host_x_kernel, static_cast<const uint4 *>(src), static_cast<uint4 *>(dst), n16);
 }
 
 cudaError_t launch_combine(const CombineParams &p, bool pdl, cudaStream_t s)
