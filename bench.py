@@ -10,7 +10,8 @@ int4 weights with per-row fp32 scales (about 19 MB per expert).  The layers rota
 through R copies at distinct HBM addresses and the tokens through R distinct batches, so
 every step streams its ~177 MB of weights from HBM (more than the 126 MB L2).
 
-The timed region replays CUDA graphs of R consecutive layer calls (K steps in all),
+The timed region replays one CUDA graph of exactly K consecutive layer calls (layer
+i mod R at step i; the layers' launch chain runs unbroken through the region),
 bracketed by a barrier and device synchronisation, timed with CUDA events on the launch
 stream; under torchrun every rank runs its own replica (weak scaling) and rank 0 reports
 the maximum time over ranks.  One JSON line is printed.
@@ -441,13 +442,16 @@ def bench_config(args, w, world, dev, stream, host=None, want_e2e=True):
     U_mean, A_mean = float(np.mean(U)), float(np.mean(A))
     ab = algorithmic_bytes(w, U_mean)
 
-    # ---- graphs of R consecutive layer calls (K steps = reps graphs + a remainder graph)
+    # ---- one CUDA graph of exactly K consecutive layer calls (layer i % R at step i), so
+    # that a timed region is one replay and the layers' launch chain runs unbroken
     def capture(fn, n):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for i in range(n):
-                fn(i)
+                fn(i % R)
         return g
+
+    warm_reps = max(1, (Wm + K - 1) // K)   # warm-up replays: at least Wm steps
 
     def fwd(i):
         layers[i].forward(xs[i], ws, y=ys[i], stream=stream)
@@ -456,20 +460,15 @@ def bench_config(args, w, world, dev, stream, host=None, want_e2e=True):
         for i in range(R):      # eager warm-up of every layer
             fwd(i)
     torch.cuda.synchronize(dev)
-    rem, reps = K % R, K // R
-    g_full = capture(fwd, R)
-    g_rem = capture(fwd, rem) if rem else None
+    g_full = capture(fwd, K)
 
-    def steps(gf, gr):
+    def steps(g):
         def run():
-            for _ in range(reps):
-                gf.replay()
-            if gr is not None:
-                gr.replay()
+            g.replay()
         return run
 
     with torch.cuda.stream(stream):      # warm-up steps (graphs replay on the current stream)
-        for _ in range(max(1, (Wm + R - 1) // R)):
+        for _ in range(warm_reps):
             g_full.replay()
     torch.cuda.synchronize(dev)
     st = moe.moe_get_device_status(base.handle)
@@ -479,7 +478,7 @@ def bench_config(args, w, world, dev, stream, host=None, want_e2e=True):
     clocks.start()
     time.sleep(0.4)
     t_wall0 = time.time()
-    region_ms = timed_regions(steps(g_full, g_rem), world, dev, stream, args.min_region_s)
+    region_ms = timed_regions(steps(g_full), world, dev, stream, args.min_region_s)
     t_wall1 = time.time()
     time.sleep(0.3)
     clocks.stop()
@@ -534,21 +533,20 @@ def bench_config(args, w, world, dev, stream, host=None, want_e2e=True):
         def fwd_host(i):
             layers[i].forward_host(xh[i], yh[i], ws, stream=stream)
 
-        ge = capture(fwd_host, R)
-        ge_rem = capture(fwd_host, rem) if rem else None
+        ge = capture(fwd_host, K)
         with torch.cuda.stream(stream):
-            for _ in range(max(1, (Wm + R - 1) // R)):
+            for _ in range(warm_reps):
                 ge.replay()
         torch.cuda.synchronize(dev)
-        e_ms = timed_regions(steps(ge, ge_rem), world, dev, stream, args.min_region_s / 2)
+        e_ms = timed_regions(steps(ge), world, dev, stream, args.min_region_s / 2)
         e2e_ms = max_over_ranks(world, float(np.median(e_ms)))
         e2e = {"value": job_tokens_per_s(world, K, w.T, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": w.T * w.H * 2, "d2h_bytes_per_step": w.T * w.H * 2,
                "timed_regions": len(e_ms),
-               "how": "moe_forward_host (pinned host x in, y out) captured in CUDA graphs"}
+               "how": "moe_forward_host (pinned host x in, y out), one CUDA graph of K calls per region"}
         st = moe.moe_get_device_status(base.handle)
         assert st == moe.MOE_OK, moe.status_string(st)
-        del ge, ge_rem
+        del ge
 
     # ---- the one-launch decode path on the same layers and tokens (T <= 16)
     fused = None
@@ -560,13 +558,12 @@ def bench_config(args, w, world, dev, stream, host=None, want_e2e=True):
             for i in range(R):
                 fwd_fused(i)
         torch.cuda.synchronize(dev)
-        gf = capture(fwd_fused, R)
-        gf_rem = capture(fwd_fused, rem) if rem else None
+        gf = capture(fwd_fused, K)
         with torch.cuda.stream(stream):
-            for _ in range(max(1, (Wm + R - 1) // R)):
+            for _ in range(warm_reps):
                 gf.replay()
         torch.cuda.synchronize(dev)
-        f_ms = timed_regions(steps(gf, gf_rem), world, dev, stream, args.min_region_s / 2)
+        f_ms = timed_regions(steps(gf), world, dev, stream, args.min_region_s / 2)
         f_step = max_over_ranks(world, float(np.median(f_ms))) / K
         st = moe.moe_get_device_status(base.handle)
         assert st == moe.MOE_OK, moe.status_string(st)
@@ -575,7 +572,7 @@ def bench_config(args, w, world, dev, stream, host=None, want_e2e=True):
                  "quantized_weight_gbs": fq, "frac_quantized_of_8tbs": fq / 8000.0,
                  "timed_regions": len(f_ms), "launches_per_step": 1,
                  "how": "moe_forward_fused (router, experts and combine in one persistent launch)"}
-        del gf, gf_rem
+        del gf
 
     tflops = flops(w, A_mean) / (ms_step * 1e-3) / 1e12
     out = {
@@ -591,7 +588,7 @@ def bench_config(args, w, world, dev, stream, host=None, want_e2e=True):
         "e2e": e2e, "clocks": clocks.summary(t_wall0, t_wall1), "peaks": peaks, "fused": fused,
         "timed_region_s": float(np.sum(region_ms)) / 1000.0,
     }
-    del g_full, g_rem, gk
+    del g_full, gk
     for L in layers:
         L.close()
     del layers, xs, ys, ws
@@ -681,8 +678,8 @@ def run_ours(args, w):
             "unique_experts_per_step": head["U"],
             "l2": f"no flush: {head['R']} layer copies at distinct addresses, "
                   f"{ab['total'] / 1e6:.0f} MB of weights per step > 126 MB L2",
-            "timing": f"CUDA graphs of consecutive layer calls, CUDA events on the launch stream; "
-                      f"{len(head['region_ms'])} timed regions of exactly {K} steps, median",
+            "timing": f"one CUDA graph of {K} consecutive layer calls per timed region, CUDA events "
+                      f"on the launch stream; {len(head['region_ms'])} timed regions, median",
             "parallelism": f"replicas x{world}",
         },
         "timed_regions": len(head["region_ms"]),
