@@ -755,6 +755,19 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
                 const bool sh = it.e < 0;
                 const int ez = sh ? 0 : it.e;
                 const int Kb = it.K * code_bits(FMT) / 8;   // code bytes of a row
+                if constexpr (C::kLimbs) {
+                    // the item's row scales, needed by its epilogue: into L2 now, so that the
+                    // consumers' loads do not wait behind the weight stream in the memory queues
+                    const int rows_all = slot_rows<GU>(p, sh);
+#pragma unroll
+                    for (int m = 0; m < C::kMats; ++m) {
+                        const float *sc = GU ? (m ? (sh ? p.wt.sh_u_scale : p.wt.u_scale) : (sh ? p.wt.sh_g_scale : p.wt.g_scale))
+                                             : (sh ? p.wt.sh_d_scale : p.wt.d_scale);
+                        const float *row = sc + (size_t)ez * rows_all + it.row0;
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(row));
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(row + 32));
+                    }
+                }
                 const int nst = (Kb + C::kStageK - 1) / C::kStageK;
                 // decode variant: token rows of the B operand, copied stage by stage
                 const unsigned char *brows[8];
