@@ -396,6 +396,8 @@ def test_forward_special_shapes(E, k, n_shared, scaling, fmt, hot):
     (5, 2, 1, 0, 50, None, None),    # one partial expert tile
     (40, 4, 1, 0, 70, None, None),   # a full and a partial expert tile
     (16, 2, 1, 0, 33, 320, 192),     # H with a partial K chunk; int4 rows not multiples of 128
+    (4, 2, 1, 0, 100, None, None),   # ~50 tokens per expert: 64-token items on tcgen05, ragged
+    (8, 2, 1, 0, 200, 512, 256),     # the same with several 64-token items per expert
 ])
 def test_forward_special_batches(E, k, n_shared, fmt, T, H, I):
     case = _special(E, k, n_shared, 2.5, fmt, None, T=T, H=H, I=I)

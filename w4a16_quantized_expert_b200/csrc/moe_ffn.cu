@@ -1014,12 +1014,11 @@ __global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __
 // the kernel is bound by MMA issue, not by MACs.
 
 constexpr int kTcRows = 128;                    // output rows per item (MMA M)
-constexpr int kTcTok = 32;                      // tokens per item
-constexpr int kTcNMax = 96;                     // 3 x 32 limb columns
+constexpr int kTcTok = 32;                      // tokens per item (batches of few tokens per expert)
+constexpr int kTcTokWide = 64;                  // tokens per item when experts average more than 36
 constexpr int kTcPackMax = 8;                   // packed stages (256 K each) at most
 constexpr int kTcASub = 2;                      // expanded 128-K halves held in TMEM
 constexpr int kTcBMax = 8;                      // B slots at most
-constexpr int kTcBSlot = kTcNMax * 128;         // one B slot: 96 limb rows of 128 K
 constexpr int kTcConv = 8;                      // converter warps (two per TMEM lane quarter)
 constexpr int kTcConvT = kTcConv * 32;
 constexpr int kTcEpi = 4;                       // epilogue warps (one per TMEM lane quarter)
@@ -1027,36 +1026,43 @@ constexpr int kTcThreads = (2 + kTcConv + kTcEpi) * 32;
 // dynamic shared memory the kernel may take (the device's opt-in maximum less a margin
 // for static shared memory)
 constexpr size_t kTcSmemMax = 232448 - 1024;
-static_assert(kTcBSlot % 1024 == 0, "B slots keep the 1024-byte swizzle atoms aligned");
-
-template <bool GU>
+// TOK tokens per item: N = 3 TOK limb columns at most.  With 64-token items (batches of
+// many tokens per expert: each weight byte is read once for twice the tokens, and each MMA
+// carries twice the columns) the gate/up accumulators take 384 of the 512 TMEM columns, so
+// they are single-buffered there (the next item's MMAs wait for the epilogue).
+template <bool GU, int TOK>
 struct TcCfg {
     static constexpr int kMats = GU ? 2 : 1;
+    static constexpr int kNMax = 3 * TOK;                            // limb columns of an item
+    static constexpr int kBSlot = kNMax * 128;                       // one B slot: the limb rows of 128 K
     static constexpr int kPackBytes = kMats * kTcRows * kBoxBytes;   // one 256-K stage of codes
-    static constexpr int kAccCols = kMats * kTcNMax;                 // TMEM columns of one accumulator set
+    static constexpr int kAccCols = kMats * kNMax;                   // TMEM columns of one accumulator set
     static constexpr int kACols = kMats * 32;                        // TMEM columns of one expanded 128-K half
-    static constexpr int kACol0 = 2 * kAccCols;                      // first A column
-    static constexpr int kTmemCols = GU ? 512 : 256;                 // (a power of two)
-    static constexpr int kBSlots = GU ? 4 : 6;
+    static constexpr int kNAcc = 2 * kAccCols + kTcASub * kACols <= 512 ? 2 : 1;   // accumulator sets
+    static constexpr int kACol0 = kNAcc * kAccCols;                  // first A column
+    static constexpr int kTmemCols = kACol0 + kTcASub * kACols <= 256 ? 256 : 512;   // (a power of two)
+    static constexpr int kBSlots = TOK > kTcTok ? 4 : (GU ? 4 : 6);
     static_assert(kACol0 + kTcASub * kACols <= kTmemCols, "TMEM budget");
+    static_assert(kBSlot % 1024 == 0, "B slots keep the 1024-byte swizzle atoms aligned");
+    static_assert(kBSlots <= kTcBMax, "B slot barriers");
 };
 
 // dynamic shared memory of a launch with np packed stages: stages, B slots, slot table,
 // item metadata, barriers
-template <bool GU>
+template <bool GU, int TOK>
 __host__ __device__ constexpr size_t tc_smem(int E, int np)
 {
-    using C = TcCfg<GU>;
-    return 1024 + (size_t)np * C::kPackBytes + (size_t)C::kBSlots * kTcBSlot + (size_t)4 * 4 * (E + 2) + 64 +
-           2 * kTcTok * 16 + 8 + 8 + (2 * kTcPackMax + 2 * kTcASub + kTcBMax + 4 + 2 * kItemQ + 1) * 8;
+    using C = TcCfg<GU, TOK>;
+    return 1024 + (size_t)np * C::kPackBytes + (size_t)C::kBSlots * C::kBSlot + (size_t)4 * 4 * (E + 2) + 64 +
+           2 * TOK * 16 + 8 + 8 + (2 * kTcPackMax + 2 * kTcASub + kTcBMax + 4 + 2 * kItemQ + 1) * 8;
 }
 
 // packed stages of a launch: as many as fit (at most kTcPackMax)
-template <bool GU>
+template <bool GU, int TOK>
 static int tc_pack_stages(int E)
 {
-    const size_t base = tc_smem<GU>(E, 0);
-    const int n = base < kTcSmemMax ? (int)((kTcSmemMax - base) / TcCfg<GU>::kPackBytes) : 0;
+    const size_t base = tc_smem<GU, TOK>(E, 0);
+    const int n = base < kTcSmemMax ? (int)((kTcSmemMax - base) / TcCfg<GU, TOK>::kPackBytes) : 0;
     return n > kTcPackMax ? kTcPackMax : n;
 }
 
@@ -1110,17 +1116,17 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-template <bool GU>
+template <bool GU, int TOK>
 __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_constant__ LayerMaps maps, const FfnParams p)
 {
-    using C = TcCfg<GU>;
+    using C = TcCfg<GU, TOK>;
     constexpr int RW = kTcRows / kRowTile;   // 8: items of 128 rows
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *pack = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int NP = p.stages;                                                  // packed stages of this launch
     unsigned char *bring = pack + (size_t)NP * C::kPackBytes;                 // B slots (1024-aligned: all sizes are)
     constexpr int NB = C::kBSlots;
-    int *tbl = reinterpret_cast<int *>(bring + (size_t)NB * kTcBSlot);
+    int *tbl = reinterpret_cast<int *>(bring + (size_t)NB * C::kBSlot);
     const int E = p.E;
     SlotTable tb;
     tb.e = tbl;
@@ -1131,10 +1137,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
     volatile int *abort_flag = tb.hdr + 2;
     volatile int *cfail = tb.hdr + 3;
     volatile int *q_item = tb.hdr + 4;
-    const unsigned char **s_brow = reinterpret_cast<const unsigned char **>(tb.hdr + 16);   // [2][kTcTok] limb rows
-    float *s_sc = reinterpret_cast<float *>(s_brow + 2 * kTcTok);   // [2][kTcTok] activation scale of each token
-    int *s_id = reinterpret_cast<int *>(s_sc + 2 * kTcTok);         // [2][kTcTok] token (gate/up) or assignment (down)
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(s_id + 2 * kTcTok);
+    const unsigned char **s_brow = reinterpret_cast<const unsigned char **>(tb.hdr + 16);   // [2][TOK] limb rows
+    float *s_sc = reinterpret_cast<float *>(s_brow + 2 * TOK);   // [2][TOK] activation scale of each token
+    int *s_id = reinterpret_cast<int *>(s_sc + 2 * TOK);         // [2][TOK] token (gate/up) or assignment (down)
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(s_id + 2 * TOK);
     uint64_t *bars = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(s_tmem + 2) + 7) & ~uintptr_t(7));
     uint64_t *pk_full = bars, *pk_empty = pk_full + kTcPackMax;
     uint64_t *sb_full = pk_empty + kTcPackMax, *sb_empty = sb_full + kTcASub;   // expanded halves in TMEM
@@ -1260,9 +1266,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
             const Item it = (i < n_pre) ? make_item<GU, RW>(p, -1, p.T, 0, i) : decode_item<GU, RW>(p, tb, i);
             const int n = ((3 * it.ntok + 15) / 16) * 16;
             const uint32_t idesc = umma_idesc_s8(n);
-            const int buf = n_item & 1;
-            // the epilogue of the item two back has released this accumulator set
-            if (!mbar_wait(&acc_empty[buf], (uint32_t)(((n_item >> 1) & 1) ^ 1), p.status)) { ok = false; break; }
+            const int buf = n_item % C::kNAcc;
+            // the epilogue of the item kNAcc back has released this accumulator set
+            if (!mbar_wait(&acc_empty[buf], (uint32_t)(((n_item / C::kNAcc) & 1) ^ 1), p.status)) { ok = false; break; }
             tc_fence_after();
             const int nsub = (it.K + 127) / 128;   // 128-K halves of the packed stages
             for (int u = 0; u < nsub; ++u) {
@@ -1274,7 +1280,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
                     // The issuing thread's own instructions between MMAs add to every MMA's
                     // cost (measured), so the operands are formed once per half: the B
                     // descriptor advances 32 bytes (2 in its 16-byte address field) per step.
-                    const uint64_t db0 = umma_sdesc(smem_u32(bring + (size_t)bslot * kTcBSlot));
+                    const uint64_t db0 = umma_sdesc(smem_u32(bring + (size_t)bslot * C::kBSlot));
                     const uint32_t abase = tmem + C::kACol0 + sub * C::kACols;
                     const uint32_t dbase = tmem + buf * C::kAccCols;
                     const uint32_t acc0 = u > 0 ? 1u : 0u;
@@ -1283,13 +1289,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
                         for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
                             for (int m = 0; m < C::kMats; ++m)
-                                umma_s8_ta(dbase + m * kTcNMax, abase + m * 32 + 8 * kk, db0 + 2 * kk, idesc,
+                                umma_s8_ta(dbase + m * C::kNMax, abase + m * 32 + 8 * kk, db0 + 2 * kk, idesc,
                                            kk > 0 ? 1u : acc0);
                     } else {
                         for (int kk = 0; kk < kvals / 32; ++kk)
 #pragma unroll
                             for (int m = 0; m < C::kMats; ++m)
-                                umma_s8_ta(dbase + m * kTcNMax, abase + m * 32 + 8 * kk, db0 + 2 * kk, idesc,
+                                umma_s8_ta(dbase + m * C::kNMax, abase + m * 32 + 8 * kk, db0 + 2 * kk, idesc,
                                            kk > 0 ? 1u : acc0);
                     }
                     umma_commit(&sb_empty[sub]);   // the half and the B slot are free once
@@ -1349,11 +1355,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
                 // copied into B slot (gsub + half) % NB in the swizzled layout the MMA reads, up
                 // to NB - 2 halves ahead (a slot is refilled two halves after its last use, so the
                 // copies never wait for the MMAs just handed over).  Thread ltid owns pieces
-                // ltid, ltid + 256, ltid + 512 of each half.
-                const unsigned char *bsrc[3];
-                int bdst[3];
+                // ltid + 256 q of each half.
+                constexpr int NQ = 3 * TOK * 8 / kTcConvT;
+                const unsigned char *bsrc[NQ];
+                int bdst[NQ];
 #pragma unroll
-                for (int q = 0; q < 3; ++q) {
+                for (int q = 0; q < NQ; ++q) {
                     const int pc = ltid + q * kTcConvT, jr = pc >> 3, x = pc & 7;
                     bsrc[q] = nullptr;
                     bdst[q] = -1;
@@ -1369,10 +1376,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
                     const int g = gsub + u2, slot = g % NB;
                     if (!mbar_wait(&b_empty[slot], (uint32_t)(((g / NB) & 1) ^ 1), p.status)) ok = false;
                     if (ok) {
-                        unsigned char *sl = bring + (size_t)slot * kTcBSlot;
+                        unsigned char *sl = bring + (size_t)slot * C::kBSlot;
                         const size_t so = (size_t)(u2 >> 1) * kLimbBlockBytes + 128 * (u2 & 1);
 #pragma unroll
-                        for (int q = 0; q < 3; ++q) {
+                        for (int q = 0; q < NQ; ++q) {
                             if (bdst[q] < 0) continue;
                             if (bsrc[q]) cp_async16(sl + bdst[q], bsrc[q] + so);
                             else *reinterpret_cast<uint4 *>(sl + bdst[q]) = make_uint4(0u, 0u, 0u, 0u);
@@ -1465,8 +1472,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
                                     : __ldcg(sh ? p.hsh_limb_scale + bpos : p.h_limb_scale + it.boff + bpos);
                 }
                 consumer_sync<kTcConvT / 2, 2>();
-                const int buf = n_item & 1;
-                if (!mbar_wait(&acc_full[buf], (uint32_t)((n_item >> 1) & 1), p.status)) { ok = false; break; }
+                const int buf = n_item % C::kNAcc;
+                if (!mbar_wait(&acc_full[buf], (uint32_t)((n_item / C::kNAcc) & 1), p.status)) { ok = false; break; }
                 tc_fence_after();
                 const int rows_all = slot_rows<GU>(p, sh);
                 const int ez = sh ? 0 : it.e;
@@ -1485,7 +1492,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
 #pragma unroll
                         for (int c8 = 0; c8 < 3; ++c8) {
                             uint32_t v[8];
-                            tmem_ld8(tbase + m * kTcNMax + 3 * j0 + 8 * c8, v);
+                            tmem_ld8(tbase + m * C::kNMax + 3 * j0 + 8 * c8, v);
 #pragma unroll
                             for (int x = 0; x < 8; ++x) a[m][8 * c8 + x] = v[x];
                         }
@@ -1685,47 +1692,62 @@ static cudaError_t prepare_fmt(int E, int occ[2][2][2])
     }
 }
 
-template <bool GU>
+template <bool GU, int TOK>
 static cudaError_t tc_prepare_t(int E)
 {
     int dev = 0, optin = 0;
     cudaFuncAttributes fa;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, ffn_tc_kernel<GU>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, ffn_tc_kernel<GU, TOK>);
     if (e != cudaSuccess) return e;
-    if (tc_pack_stages<GU>(E) < 2 || tc_smem<GU>(E, tc_pack_stages<GU>(E)) + fa.sharedSizeBytes > (size_t)optin)
+    if (tc_pack_stages<GU, TOK>(E) < 2 || tc_smem<GU, TOK>(E, tc_pack_stages<GU, TOK>(E)) + fa.sharedSizeBytes > (size_t)optin)
         return cudaErrorInvalidValue;
-    e = cudaFuncSetAttribute(ffn_tc_kernel<GU>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
+    e = cudaFuncSetAttribute(ffn_tc_kernel<GU, TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             optin - (int)fa.sharedSizeBytes);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(ffn_tc_kernel<GU>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    return cudaFuncSetAttribute(ffn_tc_kernel<GU, TOK>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
 }
 
 cudaError_t tc_prepare(int E)
 {
-    cudaError_t e = tc_prepare_t<true>(E);
-    return e != cudaSuccess ? e : tc_prepare_t<false>(E);
+    cudaError_t e = tc_prepare_t<true, kTcTok>(E);
+    if (e == cudaSuccess) e = tc_prepare_t<false, kTcTok>(E);
+    if (e == cudaSuccess) e = tc_prepare_t<true, kTcTokWide>(E);
+    return e != cudaSuccess ? e : tc_prepare_t<false, kTcTokWide>(E);
 }
 
-// One CTA per SM (the kernel takes most of the shared memory and all of the TMEM).
-cudaError_t launch_tc(const LayerMaps &maps, const FfnParams &p0, bool gate_up, int grid, bool pdl, cudaStream_t s)
+template <bool GU, int TOK>
+static cudaError_t launch_tc_t(const LayerMaps &maps, const FfnParams &p0, int grid, bool pdl, cudaStream_t s)
 {
     FfnParams p = p0;
-    p.tok_chunk = kTcTok;
-    p.work = p0.work + (gate_up ? 0 : 2);
-    p.stages = gate_up ? tc_pack_stages<true>(p.E) : tc_pack_stages<false>(p.E);
+    p.tok_chunk = TOK;
+    p.work = p0.work + (GU ? 0 : 2);
+    p.stages = tc_pack_stages<GU, TOK>(p.E);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kTcThreads);
-    cfg.dynamicSmemBytes = gate_up ? tc_smem<true>(p.E, p.stages) : tc_smem<false>(p.E, p.stages);
+    cfg.dynamicSmemBytes = tc_smem<GU, TOK>(p.E, p.stages);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return gate_up ? cudaLaunchKernelEx(&cfg, ffn_tc_kernel<true>, maps, p)
-                   : cudaLaunchKernelEx(&cfg, ffn_tc_kernel<false>, maps, p);
+    return cudaLaunchKernelEx(&cfg, ffn_tc_kernel<GU, TOK>, maps, p);
+}
+
+// tokens per item of the tensor-memory kernel: 64 when the routed experts average more
+// than 36 tokens each (T k / E), else 32
+int tc_tokens(const FfnParams &p) { return (long)p.T * p.k > 36l * p.E ? kTcTokWide : kTcTok; }
+
+// One CTA per SM (the kernel takes most of the shared memory and all of the TMEM).
+cudaError_t launch_tc(const LayerMaps &maps, const FfnParams &p, bool gate_up, int grid, bool pdl, cudaStream_t s)
+{
+    if (tc_tokens(p) == kTcTokWide)
+        return gate_up ? launch_tc_t<true, kTcTokWide>(maps, p, grid, pdl, s)
+                       : launch_tc_t<false, kTcTokWide>(maps, p, grid, pdl, s);
+    return gate_up ? launch_tc_t<true, kTcTok>(maps, p, grid, pdl, s) : launch_tc_t<false, kTcTok>(maps, p, grid, pdl, s);
 }
 
 cudaError_t ffn_prepare(int fmt, int E, int occ[2][2][2])
