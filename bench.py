@@ -49,6 +49,7 @@ DEFAULTS = {
     "nvfp4_16": (20000, 400, 16),
     "prefill512": (400, 20, 2),
     "prefill2048": (100, 5, 1),
+    "batch128": (800, 20, 2),
     "decode1_topp": (40000, 400, 8),
     "tiny": (20000, 200, 8),
     "int8_1": (20000, 400, 4),
@@ -373,8 +374,8 @@ def run_reference(args, w):
 # workloads measured beside the headline one in the default run (the rest of the
 # metric's configurations: T=8 decode, NVFP4 at T=1 and T=16, the T=512 batch; adaptive
 # top-p on decode1; and the int8 and int2 widths at the decode1 shape, T=1 and T=8)
-EXTRA_CONFIGS = ("decode8", "nvfp4_1", "nvfp4_16", "prefill512", "decode1_topp", "int8_1", "int8_8",
-                 "int2_1", "int2_8")
+EXTRA_CONFIGS = ("decode8", "nvfp4_1", "nvfp4_16", "prefill512", "batch128", "decode1_topp", "int8_1",
+                 "int8_8", "int2_1", "int2_8")
 MIN_REGION_S = 0.5     # timed regions are repeated until they add up to at least this
 
 

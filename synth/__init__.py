@@ -176,6 +176,10 @@ WORKLOADS = {
     # larger batch (about 64 tokens per expert): the tensor-memory kernel's compute-heavier regime
     "prefill2048": Workload("prefill2048", 2048, 6144, 2048, 2048, 256, 8, 1, 2.5, FMT_INT4,
                             "uniform", BASE_SEED + 5),
+    # a mid-size batch of about 4 tokens per routed expert (128 x 8 / 256): the regime
+    # between the decode batches and prefill512, on the prefill512 layer shape
+    "batch128": Workload("batch128", 128, 6144, 2048, 2048, 256, 8, 1, 2.5, FMT_INT4, "uniform",
+                         BASE_SEED + 8),
     # the other row-scaled widths (int8 and int2 kernels with per-row scales: hakusoku page,
     # section "実装済み機能") at the decode1 shape, one token and eight
     "int8_1": Workload("int8_1", 1, 6144, 2048, 2048, 256, 8, 1, 2.5, FMT_INT8, "uniform",

@@ -17,8 +17,9 @@ activations at the edges of the fp16 range.
    rounded.  Rows with outlier channels 2^12 .. 2^15 above the rest, rows at the largest
    finite fp16 values, rows of fp16 subnormals and rows mixing subnormals with N(0,1)
    values (synth.make_stress_tokens) go through the whole layer and are compared with the
-   FP64 oracle at the layer's tolerance, on the decode kernels (T = 1, 8), the
-   tensor-memory kernel (T = 40) and the NVFP4 path.  The layer's weights are scaled by
+   FP64 oracle at the layer's tolerance, on the decode kernels (T = 1, 8), a 40-token batch
+   on the int8 path (5 tokens per expert) and on the tensor-memory kernel (20 tokens per
+   expert), and the NVFP4 path.  The layer's weights are scaled by
    powers of two (synth.scale_layer) so that h and y stay inside the fp16 range; the test
    checks that on the oracle's values first.
 
@@ -42,6 +43,8 @@ W = synth.WORKLOADS
 E1024 = W["tiny"].with_(E=1024, k=8, name="tiny_e1024")
 BATCH = synth.Workload("stress_batch", 40, 1024, 512, 512, 32, 4, 1, 2.5, synth.FMT_INT4, "uniform",
                        synth.BASE_SEED + 40)
+# the same batch over 8 experts: 20 tokens per expert, past the int8 path's share
+BATCH_TC = BATCH.with_(E=8, name="stress_batch_tc")
 
 
 def _workload(name):
@@ -142,7 +145,8 @@ def _check_routing_arrays(g, host, desc, x, w):
 FACTORS = {"outlier": (2.0 ** -8, 1.0, 1.0), "near_max": (2.0 ** -9, 2.0 ** -2, 1.0),
            "subnormal": (2.0 ** 12, 1.0, 2.0 ** 14), "mixed": (1.0, 1.0, 1.0)}
 
-STRESS_CASES = [(n, T, kind) for n, T in (("decode1", 1), ("stress_batch", 40), ("nvfp4_1", 1))
+STRESS_CASES = [(n, T, kind) for n, T in (("decode1", 1), ("stress_batch", 40), ("stress_batch_tc", 40),
+                                          ("nvfp4_1", 1))
                 for kind in synth.STRESS_KINDS] + \
                [("decode8", 8, "outlier"), ("decode8", 8, "subnormal"), ("decode8", 8, "near_max"),
                 ("nvfp4_16", 16, "outlier"), ("nvfp4_16", 16, "subnormal")]
@@ -150,7 +154,7 @@ STRESS_CASES = [(n, T, kind) for n, T in (("decode1", 1), ("stress_batch", 40), 
 
 @pytest.mark.parametrize("name,T,kind", STRESS_CASES)
 def test_forward_activation_edge_cases(name, T, kind):
-    w = BATCH if name == "stress_batch" else W[name]
+    w = {"stress_batch": BATCH, "stress_batch_tc": BATCH_TC}.get(name) or W[name]
     fgu, fd, fr = FACTORS[kind]
     if kind == "subnormal" and w.fmt == synth.FMT_NVFP4:
         fgu *= 8.0     # NVFP4 weights are about 4x smaller than the int4 ones

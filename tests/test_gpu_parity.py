@@ -251,6 +251,17 @@ def test_forward_prefill512_sampled():
     print(f"prefill512 sampled: excluded {excluded}/{len(tokens)}, rel err {err:.3g}")
 
 
+def test_forward_batch128_sampled():
+    """About 4 tokens per expert at full size: the int8 path's 8-token items, every expert
+    hit, some with two items."""
+    case = Case(W["batch128"])
+    y, _ = _forward(case)
+    tokens = [0, 1, 7, 8, 63, 64, 126, 127]
+    ref = case.oracle_forward(tokens=tokens)
+    excluded, err = check_y(y_to_f64(y)[tokens], ref["y"], ref["gap"])
+    print(f"batch128 sampled: excluded {excluded}/{len(tokens)}, rel err {err:.3g}")
+
+
 def test_forward_prefill2048_sampled():
     """About 64 tokens per expert: several 32-token items per expert row tile."""
     case = Case(W["prefill2048"])
@@ -261,7 +272,9 @@ def test_forward_prefill2048_sampled():
     print(f"prefill2048 sampled: excluded {excluded}/{len(tokens)}, rel err {err:.3g}")
 
 
-@pytest.mark.parametrize("T", [1, 2, 15, 16, 17, 33, 64])
+# (E = 16, k = 2: up to T = 48, six tokens per expert, the int8 path's 8-token items; from
+# T = 49 the tensor-memory kernel)
+@pytest.mark.parametrize("T", [1, 2, 15, 16, 17, 33, 48, 49, 64])
 def test_forward_ragged_T(tiny, T):
     case = Case(W["tiny"], T=T, max_tokens=64, batch=T)
     y, _ = _forward(case)
@@ -395,7 +408,8 @@ def test_forward_special_shapes(E, k, n_shared, scaling, fmt, hot):
     (32, 8, 1, 1, 40, None, None),   # NVFP4, several token tiles
     (5, 2, 1, 0, 50, None, None),    # one partial expert tile
     (40, 4, 1, 0, 70, None, None),   # a full and a partial expert tile
-    (16, 2, 1, 0, 33, 320, 192),     # H with a partial K chunk; int4 rows not multiples of 128
+    (16, 2, 1, 0, 33, 320, 192),     # H with a partial limb block, ~4 tokens per expert (int8 path)
+    (4, 2, 1, 0, 33, 320, 192),      # ~16 tokens per expert, int4 rows not multiples of 128 (f16 path)
     (4, 2, 1, 0, 100, None, None),   # ~50 tokens per expert: 64-token items on tcgen05, ragged
     (8, 2, 1, 0, 200, 512, 256),     # the same with several 64-token items per expert
 ])

@@ -47,21 +47,35 @@ struct Ws {
 // bytes of one row of int8 limbs of a K-long operand (blocks of 256 values, 3 limbs)
 size_t limb_row_bytes(int K) { return (size_t)((K + kLimbBlockK - 1) / kLimbBlockK) * kLimbBlockBytes; }
 
-// Larger int4 batches run the tensor-memory kernel (items of 128 rows and up to 40 tokens),
-// which needs row counts that are multiples of 128.
+// Batches that average at most kFewTokensPerExpert tokens per routed expert (T k <= 6 E)
+// keep the 8-token items of the int8 path: each weight byte is read once per 8 tokens of
+// an expert, and its mma.sync work shrinks with the tokens.  The tensor-memory kernel
+// issues the same MMAs per weight byte however few tokens an item holds, so it pays only
+// with more tokens per expert.  Measured on B200 (H=6144, I=2048, E=256, top-8, int4), layer
+// time int8 path vs tensor-memory kernel: T=32 (1 token per expert) 526 vs 926 us, T=128
+// 1087 vs 1394, T=192 (6) 1431 vs 1521, T=256 (8) 1768 vs 1641, T=512 3135 vs 2306.
+constexpr long kFewTokensPerExpert = 6;
+
+bool few_tokens_per_expert(const moe_layer_desc &d, int T)
+{
+    return (long)T * d.top_k <= kFewTokensPerExpert * d.n_experts;
+}
+
+// Larger int4 batches with more tokens per expert run the tensor-memory kernel (items of
+// 128 rows and 32 or 64 tokens), which needs row counts that are multiples of 128.
 bool use_tc(const moe_layer_desc &d, int T)
 {
-    return d.format == MOE_FMT_INT4_ROWSCALE && T > 16 && d.hidden % 128 == 0 && d.inter % 128 == 0 &&
-           (!d.n_shared || d.inter_shared % 128 == 0);
+    return d.format == MOE_FMT_INT4_ROWSCALE && T > 16 && !few_tokens_per_expert(d, T) && d.hidden % 128 == 0 &&
+           d.inter % 128 == 0 && (!d.n_shared || d.inter_shared % 128 == 0);
 }
 
 // the int4 expert kernels run on the int8 path (activations as limbs) for decode-sized
-// batches (8-token items) and on the tensor-memory kernel; int8 and int2 weights run the
-// 8-token int8 path at every batch size
+// batches and batches of few tokens per expert (8-token items) and on the tensor-memory
+// kernel; int8 and int2 weights run the 8-token int8 path at every batch size
 bool use_limbs(const moe_layer_desc &d, int T)
 {
     if (d.format == MOE_FMT_INT8_ROWSCALE || d.format == MOE_FMT_INT2_ROWSCALE) return true;
-    return d.format == MOE_FMT_INT4_ROWSCALE && (T <= 16 || use_tc(d, T));
+    return d.format == MOE_FMT_INT4_ROWSCALE && (T <= 16 || few_tokens_per_expert(d, T) || use_tc(d, T));
 }
 
 Ws ws_layout(const moe_layer_desc &d, int T)
@@ -105,7 +119,9 @@ Ws ws_layout(const moe_layer_desc &d, int T)
     w.y_shared = o; o = up256(o + (size_t)T * d.hidden * 4 * (d.n_shared ? 1 : 0));
     w.x_stage = o; o = up256(o + (size_t)T * d.hidden * 2);
     w.y_stage = o; o = up256(o + (size_t)T * d.hidden * 2);
-    const bool lb = use_limbs(d, T);
+    // limb buffers for every row-scaled layer: a batch of fewer tokens than T may take the
+    // int8 path where T does not, and the size for T must serve every smaller batch
+    const bool lb = row_scaled(d.format);
     w.x_limbs = o; o = up256(o + (lb ? (size_t)T * limb_row_bytes(d.hidden) : 0));
     w.x_limb_scale = o; o = up256(o + (lb ? (size_t)T * 4 : 0));
     w.h_limbs = o; o = up256(o + (lb ? Tk * limb_row_bytes(d.inter) : 0));
@@ -195,12 +211,11 @@ int validate_weights(const moe_layer_desc *d, const moe_weights *w)
     return MOE_OK;
 }
 
-// tokens per expert work item: 8 for decode-sized batches and for int8 / int2 weights (a
-// one-n-tile kernel with few registers; a bucket of more tokens becomes several items), 32
-// otherwise
+// tokens per expert work item: 8 wherever the int8 path runs (a one-n-tile kernel with few
+// registers; a bucket of more tokens becomes several items), 32 on the f16 path
 int tok_chunk(const moe_layer_desc &d, int T)   // (the tensor-memory kernel sets its own)
 {
-    return (T <= 16 || d.format == MOE_FMT_INT8_ROWSCALE || d.format == MOE_FMT_INT2_ROWSCALE) ? 8 : kTokChunk;
+    return (use_limbs(d, T) && !use_tc(d, T)) ? 8 : kTokChunk;
 }
 
 int check_ws(const moe_layer *L, int T, void *ws, size_t bytes)
