@@ -243,33 +243,48 @@ def test_forward_full_size(name):
 
 
 def test_forward_prefill512_sampled():
+    """~16 tokens per expert (the tensor-memory kernel's 32-token items): every fourth
+    token and the last against the oracle, so that nearly every (expert, token chunk) item
+    holds a checked token."""
     case = Case(W["prefill512"])
     y, _ = _forward(case)
-    tokens = [0, 1, 63, 64, 255, 300, 510, 511]
+    tokens = list(range(0, 512, 4)) + [511]
     ref = case.oracle_forward(tokens=tokens)
     excluded, err = check_y(y_to_f64(y)[tokens], ref["y"], ref["gap"])
     print(f"prefill512 sampled: excluded {excluded}/{len(tokens)}, rel err {err:.3g}")
 
 
-def test_forward_batch128_sampled():
-    """About 4 tokens per expert at full size: the int8 path's 8-token items, every expert
-    hit, some with two items."""
+def test_forward_batch128():
+    """About 4 tokens per expert at full size (the int8 path's 8-token items, some experts
+    with two items): every token against the oracle."""
     case = Case(W["batch128"])
     y, _ = _forward(case)
-    tokens = [0, 1, 7, 8, 63, 64, 126, 127]
-    ref = case.oracle_forward(tokens=tokens)
-    excluded, err = check_y(y_to_f64(y)[tokens], ref["y"], ref["gap"])
-    print(f"batch128 sampled: excluded {excluded}/{len(tokens)}, rel err {err:.3g}")
+    ref = case.oracle_forward(tokens=list(range(128)))
+    excluded, err = check_y(y_to_f64(y), ref["y"], ref["gap"])
+    print(f"batch128: excluded {excluded}/128, rel err {err:.3g}")
 
 
 def test_forward_prefill2048_sampled():
-    """About 64 tokens per expert: several 32-token items per expert row tile."""
+    """About 64 tokens per expert: 64-token items, several per expert row tile; every
+    sixteenth token and the last against the oracle."""
     case = Case(W["prefill2048"])
     y, _ = _forward(case)
-    tokens = [0, 1, 511, 512, 1024, 1535, 2046, 2047]
+    tokens = list(range(0, 2048, 16)) + [2047]
     ref = case.oracle_forward(tokens=tokens)
     excluded, err = check_y(y_to_f64(y)[tokens], ref["y"], ref["gap"])
     print(f"prefill2048 sampled: excluded {excluded}/{len(tokens)}, rel err {err:.3g}")
+
+
+@pytest.mark.parametrize("E,k,T", [(8, 2, 64),    # 16 tokens per expert: the tensor-memory kernel
+                                   (32, 4, 48)])  # 6 tokens per expert: the int8 path
+def test_forward_full_T_at_the_decode_shape(E, k, T):
+    """Every token of a batch at H = 6144, I = 2048 (the stage counts and ring wrap-around
+    of the full-size layer) against the oracle, on both batch paths."""
+    case = Case(W["decode1"].with_(E=E, k=k, T=T, name=f"full_T_{E}_{k}_{T}"))
+    y, _ = _forward(case)
+    ref = case.oracle_forward()
+    excluded, err = check_y(y_to_f64(y), ref["y"], ref["gap"])
+    print(f"E={E} k={k} T={T}: excluded {excluded}/{T}, rel err {err:.3g}")
 
 
 # (E = 16, k = 2: up to T = 48, six tokens per expert, the int8 path's 8-token items; from
