@@ -289,6 +289,25 @@ const char *moe_status_string(int status);
  * debugging, not for the hot path. */
 int moe_get_device_status(const moe_layer *layer, int *status);
 
+/* Source: none of the pages chooses kernels; the choice is this implementation's (measured
+ * crossovers in its design notes).  Which expert kernels (steps 4-6) moe_forward,
+ * moe_forward_host and moe_expert_ffn run for a batch of T tokens of a layer with this
+ * description:
+ *   plan[0]  MOE_PLAN_DECODE (the streaming kernels with 8-token work items: decode-sized
+ *            batches, int4 batches of at most 6 tokens per routed expert, int8 and int2 at
+ *            every T), MOE_PLAN_F16_BATCH (32-token items on the f16 path: NVFP4 above 16
+ *            tokens, int4 shapes the tensor-memory kernel does not take) or
+ *            MOE_PLAN_TENSOR_MEMORY (the tcgen05 kernel: int4 above 16 tokens and more than
+ *            6 tokens per routed expert, H, I, I_sh multiples of 128);
+ *   plan[1]  tokens per work item (8, 32, or 32 / 64 on the tensor-memory kernel);
+ *   plan[2]  1 if activations are carried as exact int8 limbs, 0 for f16.
+ * A pure host function: no handle, no GPU.  Returns MOE_ERR_INVALID_ARG for an invalid
+ * description, a NULL plan or T outside [1, max_tokens]. */
+#define MOE_PLAN_DECODE 0
+#define MOE_PLAN_F16_BATCH 1
+#define MOE_PLAN_TENSOR_MEMORY 2
+int moe_plan(const moe_layer_desc *desc, int T, int plan[3]);
+
 /* Where moe_forward (and moe_forward_host) leave the routing and grouping results of a
  * call with T tokens inside its workspace: byte offsets from the workspace's start of
  *   logits fp32 [T][E], topk_idx int32 [T][k], topk_w fp32 [T][k]   (as moe_route

@@ -104,6 +104,38 @@ def test_unused_pointers_may_be_null():
         assert rc == moe.MOE_ERR_CUDA and h is None
 
 
+D, F, TM = moe.MOE_PLAN_DECODE, moe.MOE_PLAN_F16_BATCH, moe.MOE_PLAN_TENSOR_MEMORY
+BIG = dict(hidden=6144, inter=2048, inter_shared=2048, n_experts=256, top_k=8, max_tokens=4096)
+
+
+@pytest.mark.parametrize("fmt,T,shape,plan", [
+    (0, 1, BIG, (D, 8, 1)), (0, 16, BIG, (D, 8, 1)),
+    (0, 17, BIG, (D, 8, 1)), (0, 128, BIG, (D, 8, 1)), (0, 192, BIG, (D, 8, 1)),  # <= 6 tokens per expert
+    (0, 193, BIG, (TM, 32, 1)), (0, 512, BIG, (TM, 32, 1)),                       # tensor-memory kernel
+    (0, 1152, BIG, (TM, 32, 1)), (0, 1153, BIG, (TM, 64, 1)), (0, 2048, BIG, (TM, 64, 1)),  # > 36 per expert
+    (1, 1, BIG, (D, 8, 0)), (1, 16, BIG, (D, 8, 0)), (1, 17, BIG, (F, 32, 0)),     # NVFP4
+    (2, 1, BIG, (D, 8, 1)), (2, 2048, BIG, (D, 8, 1)), (3, 512, BIG, (D, 8, 1)),   # int8, int2
+    (0, 48, dict(hidden=256, inter=128, inter_shared=128, n_experts=16, top_k=2, max_tokens=64), (D, 8, 1)),
+    (0, 49, dict(hidden=256, inter=128, inter_shared=128, n_experts=16, top_k=2, max_tokens=64), (TM, 32, 1)),
+    (0, 33, dict(hidden=320, inter=192, inter_shared=192, n_experts=4, top_k=2, max_tokens=64), (F, 32, 0)),
+    (0, 33, dict(hidden=320, inter=192, inter_shared=192, n_experts=16, top_k=2, max_tokens=64), (D, 8, 1)),
+])
+def test_plan_of_a_batch(fmt, T, shape, plan):
+    """Which expert kernels a batch runs (a host function: no GPU).  The boundaries are the
+    measured crossovers: at most 6 tokens per routed expert on the 8-token items, 64-token
+    items past 36 tokens per expert, the decode variants for every format up to 16 tokens."""
+    assert moe.moe_plan(_desc(format=fmt, **shape), T) == plan
+
+
+def test_plan_rejects_bad_arguments():
+    with pytest.raises(moe.MoeError):
+        moe.moe_plan(_desc(), 0)
+    with pytest.raises(moe.MoeError):
+        moe.moe_plan(_desc(), 5)            # max_tokens = 4
+    with pytest.raises(moe.MoeError):
+        moe.moe_plan(_desc(hidden=100), 1)  # not a multiple of 64
+
+
 def test_null_handle_and_out_of_range_T():
     L = moe.lib()
     assert L.moe_workspace_size(None, 1) == 0

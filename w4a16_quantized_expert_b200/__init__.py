@@ -25,6 +25,9 @@ MOE_FMT_INT4_ROWSCALE = 0
 MOE_FMT_NVFP4 = 1
 MOE_FMT_INT8_ROWSCALE = 2
 MOE_FMT_INT2_ROWSCALE = 3
+MOE_PLAN_DECODE = 0
+MOE_PLAN_F16_BATCH = 1
+MOE_PLAN_TENSOR_MEMORY = 2
 
 vp = ctypes.c_void_p
 c_int = ctypes.c_int
@@ -95,9 +98,10 @@ def lib():
         L.moe_get_device_status.argtypes = [vp, ctypes.POINTER(c_int)]
         L.moe_debug_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
         L.moe_workspace_routing.argtypes = [vp, c_int, ctypes.POINTER(moe_ws_routing)]
+        L.moe_plan.argtypes = [ctypes.POINTER(moe_layer_desc), c_int, ctypes.POINTER(c_int)]
         for f in ("moe_layer_create", "moe_layer_destroy", "moe_route", "moe_route_static", "moe_group",
                   "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_fused", "moe_forward_host", "moe_forward_timed",
-                  "moe_get_device_status", "moe_debug_wait_timeout", "moe_workspace_routing"):
+                  "moe_get_device_status", "moe_debug_wait_timeout", "moe_workspace_routing", "moe_plan"):
             getattr(L, f).restype = c_int
         _lib = L
     return _lib
@@ -187,6 +191,14 @@ def moe_get_device_status(layer) -> int:
 
 def moe_debug_wait_timeout(layer, max_iters, stream=0):
     _check(lib().moe_debug_wait_timeout(layer, max_iters, stream), "moe_debug_wait_timeout")
+
+
+def moe_plan(desc: moe_layer_desc, T: int) -> tuple:
+    """(kernel family, tokens per work item, int8 limbs) of a batch of T tokens; see
+    include/moe.h."""
+    plan = (c_int * 3)(0, 0, 0)
+    _check(lib().moe_plan(ctypes.byref(desc), T, plan), "moe_plan")
+    return int(plan[0]), int(plan[1]), int(plan[2])
 
 
 def moe_workspace_routing(layer, T) -> dict:

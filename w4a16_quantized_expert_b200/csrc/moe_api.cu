@@ -24,6 +24,7 @@ cudaError_t launch_ffn(const LayerMaps &maps, const FfnParams &p, bool gate_up, 
 cudaError_t ffn_prepare(int fmt, int E, int occ[2][2][2]);
 cudaError_t tc_prepare(int E);
 cudaError_t launch_tc(const LayerMaps &maps, const FfnParams &p, bool gate_up, int grid, bool pdl, cudaStream_t s);
+int tc_tokens(const FfnParams &p);
 cudaError_t launch_wait_timeout(int *status, unsigned long long max_iters, cudaStream_t s);
 cudaError_t fused_prepare(int fmt, int *blocks_per_sm);
 cudaError_t launch_fused(const LayerMaps &maps, const FusedParams &p, int grid, bool pdl, cudaStream_t s);
@@ -211,11 +212,12 @@ int validate_weights(const moe_layer_desc *d, const moe_weights *w)
     return MOE_OK;
 }
 
-// tokens per expert work item: 8 wherever the int8 path runs (a one-n-tile kernel with few
-// registers; a bucket of more tokens becomes several items), 32 on the f16 path
+// tokens per expert work item: 8 for decode-sized batches (every format: the decode
+// variants with their B rows in shared memory) and wherever the int8 path runs (a bucket
+// of more tokens becomes several items), 32 on the f16 path for larger batches
 int tok_chunk(const moe_layer_desc &d, int T)   // (the tensor-memory kernel sets its own)
 {
-    return (use_limbs(d, T) && !use_tc(d, T)) ? 8 : kTokChunk;
+    return (T <= 16 || (use_limbs(d, T) && !use_tc(d, T))) ? 8 : kTokChunk;
 }
 
 int check_ws(const moe_layer *L, int T, void *ws, size_t bytes)
@@ -779,6 +781,25 @@ int moe_get_device_status(const moe_layer *L, int *status)
     if (cudaMemcpy(&v, L->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaMemset(L->d_status, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
     *status = v;
+    return MOE_OK;
+}
+
+int moe_plan(const moe_layer_desc *desc, int T, int plan[3])
+{
+    if (!plan || validate_desc(desc) != MOE_OK || T < 1 || T > desc->max_tokens) return MOE_ERR_INVALID_ARG;
+    const moe_layer_desc &d = *desc;
+    if (use_tc(d, T)) {
+        FfnParams p = {};
+        p.T = T;
+        p.k = d.top_k;
+        p.E = d.n_experts;
+        plan[0] = MOE_PLAN_TENSOR_MEMORY;
+        plan[1] = tc_tokens(p);
+    } else {
+        plan[1] = tok_chunk(d, T);
+        plan[0] = plan[1] > 8 ? MOE_PLAN_F16_BATCH : MOE_PLAN_DECODE;
+    }
+    plan[2] = use_limbs(d, T) ? 1 : 0;
     return MOE_OK;
 }
 
