@@ -207,6 +207,13 @@ def test_expert_ffn(name, T):
     _ffn_vs_oracle(Case(W[name], T=T, experts="routed"), T)
 
 
+@pytest.mark.parametrize("T", [33, 49, 64])
+def test_expert_ffn_batches(T):
+    """The staged expert step on both batch paths (E = 16, k = 2: T = 33 the int8 path,
+    its x limbs made by the staged call itself; T = 49 and 64 the tensor-memory kernel)."""
+    _ffn_vs_oracle(Case(W["tiny"], T=T, max_tokens=64, batch=T), T)
+
+
 def test_combine_tiny(tiny):
     T = tiny.T
     ref = tiny.oracle_forward()
