@@ -1617,6 +1617,10 @@ static void ffn_geometry(int E, int T, int &stages, int &b_stage)
 template <int FMT, bool GU, int KS, int NNMAX>
 static cudaError_t launch_t(const LayerMaps &maps, const FfnParams &p0, int grid, bool pdl, cudaStream_t s)
 {
+    // the int8-path variants read the activation limbs: never launch one without them
+    if (FfnCfg<FMT, GU, KS, NNMAX>::kLimbs && (!p0.limbs || !p0.x_limbs || !p0.x_limb_scale || !p0.h_limbs ||
+                                               !p0.h_limb_scale || !p0.chunk_counters || !p0.h_amax))
+        return cudaErrorInvalidValue;
     FfnParams p = p0;
     ffn_geometry<FMT, GU, KS, NNMAX>(p.E, p.T, p.stages, p.b_stage);
     p.work = p0.work + (GU ? 0 : 2);
