@@ -66,9 +66,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"
 # DRAM traffic per launch (bytes) of the dominant kernel from an ncu capture, keyed by
 # workload; valid only while the kernel source hashes to the recorded value.
 NCU_TRAFFIC = {
-    # ncu capture of the decode gate/up kernel: dram read 113,489,408 + write 3,768,832
+    # ncu capture of the decode gate/up kernel: dram read 113,488,896 + write 3,410,176
     # bytes per launch (a T=1 step reads the same 9 experts at E=32 as at E=256)
-    "decode1": {"kernel": "gate_up", "bytes": 117258240, "kernel_hash": "96511c6fea336837"},
+    "decode1": {"kernel": "gate_up", "bytes": 116899072, "kernel_hash": "12b50175da0b6a30"},
 }
 
 
