@@ -65,6 +65,17 @@ struct FfnCfg {
     static constexpr int kRedFloats = KS > 1 ? kConsumerWarps * kMats * kTokChunk * kRowTile : 0;
 };
 
+// Resident CTAs per SM an expert kernel is compiled for.  The int8-path down kernels run
+// three (about 73 KB of ring each): their consumers, not the weight stream, pace them --
+// measured on B200 with the same bytes in flight per SM, one CTA per SM instead of two
+// made the down kernel 25-48% slower (decode1, decode8), and three instead of two made
+// it 3-11% faster.  The others run two.
+template <int FMT, bool GU, int KS, int NNMAX>
+__host__ __device__ constexpr int ffn_min_ctas()
+{
+    return (!GU && FfnCfg<FMT, GU, KS, NNMAX>::kLimbs) ? 3 : MOE_MIN_CTAS;
+}
+
 constexpr int kStagesMax = 16;   // ring stages any launch may use (mbarrier slots)
 constexpr int kItemQ = 4;        // work items the producer may announce ahead of the consumers
 constexpr int kMaxConvRows = 64; // h rows one conversion handles (tokens of a work item)

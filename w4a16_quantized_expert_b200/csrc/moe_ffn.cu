@@ -650,7 +650,7 @@ __device__ __forceinline__ bool consume_item_limbs(const FfnParams &p, const Slo
 }
 
 template <int FMT, bool GU, int KS, int NNMAX>
-__global__ void __launch_bounds__(kFfnThreads, MOE_MIN_CTAS) ffn_kernel(const __grid_constant__ LayerMaps maps,
+__global__ void __launch_bounds__(kFfnThreads, ffn_min_ctas<FMT, GU, KS, NNMAX>()) ffn_kernel(const __grid_constant__ LayerMaps maps,
                                                           const FfnParams p)
 {
     using C = FfnCfg<FMT, GU, KS, NNMAX>;
@@ -1596,6 +1596,7 @@ __global__ void wait_timeout_kernel(int *status, unsigned long long max_iters)
 // dynamic shared memory a CTA may use so that two fit on one SM (228 KB, 1 KB reserved
 // and up to 1 KB of static shared memory per CTA)
 constexpr size_t kSmemPerCta2 = 112 * 1024;
+constexpr size_t kSmemPerCta3 = 73 * 1024;   // three CTAs per SM (the int8-path down kernels)
 
 // Ring geometry of a launch: the int8 path stages the B rows of min(T, 8) tokens per
 // stage and takes as many stages as fit beside a second CTA (at most its cap).
@@ -1606,7 +1607,8 @@ static void ffn_geometry(int E, int T, int &stages, int &b_stage)
     if constexpr (C::kLimbs) {
         b_stage = (T < 8 ? (T < 1 ? 1 : T) : 8) * C::kBRow;
         const size_t fixed = ffn_smem<FMT, GU, KS, NNMAX>(E, 0, 0);
-        int n = fixed < kSmemPerCta2 ? (int)((kSmemPerCta2 - fixed) / (C::kStageBytes + b_stage)) : 0;
+        const size_t budget = ffn_min_ctas<FMT, GU, KS, NNMAX>() == 3 ? kSmemPerCta3 : kSmemPerCta2;
+        int n = fixed < budget ? (int)((budget - fixed) / (C::kStageBytes + b_stage)) : 0;
         stages = n < 2 ? 2 : (n > C::kStagesCap ? C::kStagesCap : n);
     } else {
         stages = C::kStages;
