@@ -44,18 +44,18 @@ UNIT = "tokens/s"
 # workload -> (default steps, default warmup, rotating layers)
 DEFAULTS = {
     "decode1": (40000, 400, 8),
-    "decode8": (8000, 200, 8),
-    "nvfp4_1": (40000, 400, 32),
-    "nvfp4_16": (20000, 400, 16),
+    "decode8": (4000, 200, 8),
+    "nvfp4_1": (20000, 400, 32),
+    "nvfp4_16": (8000, 400, 16),
     "prefill512": (400, 20, 2),
     "prefill2048": (100, 5, 1),
     "batch128": (800, 20, 2),
-    "decode1_topp": (40000, 400, 8),
+    "decode1_topp": (20000, 400, 8),
     "tiny": (20000, 200, 8),
-    "int8_1": (20000, 400, 4),
-    "int8_8": (8000, 200, 4),
-    "int2_1": (40000, 400, 8),
-    "int2_8": (8000, 200, 8),
+    "int8_1": (10000, 400, 4),
+    "int8_8": (4000, 200, 4),
+    "int2_1": (20000, 400, 8),
+    "int2_8": (4000, 200, 8),
 }
 
 FMT_NAMES = {synth.FMT_INT4: "int4", synth.FMT_NVFP4: "nvfp4", synth.FMT_INT8: "int8",
@@ -625,7 +625,19 @@ def config_entry(world, r, K) -> dict:
     return e
 
 
+def config_steps(name: str, K: int, Wm: int):
+    """Steps and warm-up steps of a workload of the ``configs`` object: the headline's K
+    and W, capped by the workload's own defaults, so that a line with several workloads
+    ends within minutes (the headline workload itself runs exactly K steps)."""
+    d = DEFAULTS.get(name)
+    if d is None:
+        return K, Wm
+    return min(K, d[0]), max(3, min(Wm, d[1]))
+
+
 def run_ours(args, w):
+    import copy
+
     import torch
 
     world, rank, local = dist_setup(args.gpus)
@@ -646,7 +658,10 @@ def run_ours(args, w):
                 shared_experts[key] = synth.make_experts(wx)
             Wr, b = synth.make_router(wx)
             host = {"Wr": Wr, "bias": b, **shared_experts[key]}
-            extras[name] = bench_config(args, wx, world, dev, stream, host=host)
+            ax = copy.copy(args)
+            ax.steps, ax.warmup = config_steps(name, K, Wm)
+            extras[name] = bench_config(ax, wx, world, dev, stream, host=host)
+            extras[name]["K"] = ax.steps
     if rank != 0:
         return
     cpu = None
@@ -702,7 +717,7 @@ def run_ours(args, w):
         "clocks": head["clocks"],
         "cpu_baseline": cpu,
         "fused_path": head["fused"],
-        "configs": {name: config_entry(world, r, K) for name, r in extras.items()},
+        "configs": {name: config_entry(world, r, r["K"]) for name, r in extras.items()},
     }
     print(json.dumps(line), flush=True)
 

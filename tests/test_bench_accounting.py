@@ -67,3 +67,13 @@ def test_config_entry_figures():
     rp = dict(r, w=W["prefill512"], ab=bench.algorithmic_bytes(W["prefill512"], 228), ms_step=2.3,
               tflops=150.0, peaks={"bf16_tflops": 1500.0})
     assert bench.config_entry(1, rp, 20)["tflops_frac_of_dense_fp16_peak"] == 0.1
+
+
+def test_config_steps_are_capped_by_each_workloads_defaults():
+    # the headline's K and W as given; the other workloads of the line at most their own
+    assert bench.config_steps("prefill512", 40000, 400) == (bench.DEFAULTS["prefill512"][0], 20)
+    assert bench.config_steps("decode8", 20, 5) == (20, 5)
+    assert bench.config_steps("int8_8", 20, 1) == (20, 3)          # at least 3 warm-up steps
+    assert bench.config_steps("not_a_workload", 7, 4) == (7, 4)
+    for name in bench.EXTRA_CONFIGS:
+        assert name in bench.DEFAULTS
