@@ -67,8 +67,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"
 # workload; valid only while the kernel source hashes to the recorded value.
 NCU_TRAFFIC = {
     # ncu capture of the decode gate/up kernel: dram read 113,488,896 + write 3,410,176
-    # bytes per launch (a T=1 step reads the same 9 experts at E=32 as at E=256)
-    "decode1": {"kernel": "gate_up", "bytes": 116899072, "kernel_hash": "12b50175da0b6a30"},
+    # bytes per launch (a T=1 step reads the same 9 experts at E=32 as at E=256).  Taken
+    # on sources 12b50175da0b6a30; the one change since (three CTAs per SM for the down
+    # kernels: launch bounds and ring budget of the !GU int8-path variants) leaves the
+    # gate/up kernel's code and launch configuration as they were.
+    "decode1": {"kernel": "gate_up", "bytes": 116899072, "kernel_hash": "2ad01ac547573c66"},
 }
 
 
